@@ -1,0 +1,233 @@
+/*
+ * pa.h — C ABI of libpagedattn: paged KV-cache decode attention for B200 (sm_100a).
+ *
+ * The operations (sources: web pages on PagedAttention):
+ *
+ *   pa_decode            Batched single-token decode attention that reads each
+ *                        sequence's keys and values from a pool of fixed-size
+ *                        blocks through a per-sequence block table ("PagedAttention"
+ *                        concept card, 实现要点: the kernel takes the block table and
+ *                        reads K/V scatter-gather; 核心思想: logical block index to
+ *                        physical block).  The attention math is unchanged
+ *                        ("什么是分页注意力", 边界与常见误解): for query head h of
+ *                        sequence b, o = softmax(scale * q.K^T) V over the sequence's
+ *                        tokens.
+ *   pa_reshape_and_cache Scatter the step's new K/V rows into their slots (each step
+ *                        computes one key and value per token and caches them:
+ *                        "什么是 LLM 中的分页注意力", 快速回顾:KV 缓存; slot addressing
+ *                        as in its section 块表).
+ *   pa_copy_blocks       Copy-on-write copy of whole blocks before a forked sequence
+ *                        writes into a block it shares (concept card, 实现要点;
+ *                        "深入解析 PagedAttention", 多序列共享).
+ *   pa_alloc_*           Host-side block allocator with reference counts: on-demand
+ *                        blocks, fork = share + refcount, free at refcount 0, copy on
+ *                        write ("深入解析 PagedAttention", 核心创新 and 多序列共享;
+ *                        concept card, 带来的能力 and 实现要点).
+ *
+ * Conventions shared by every entry point
+ *   - Device pointers are caller-owned.  No entry point allocates or frees device
+ *     memory, and none synchronises: kernels are queued on `stream` and the call
+ *     returns.  The split-context workspace is caller-provided
+ *     (pa_decode_workspace_size).
+ *   - Every function returns a pa_status; no exception or abort crosses the ABI.
+ *     Argument errors are detected on the host before anything is queued, and a
+ *     failing call changes no state.
+ *   - Data corruption that only the device can see (a block id outside
+ *     [0, num_blocks), a sequence length outside [0, max_blocks*block_size], a slot
+ *     outside the pool) never faults: the kernel ORs a PA_DEVERR_* bit into
+ *     *dev_err_flag (if non-NULL), skips or clamps the access, and the affected
+ *     output is unspecified.  Read the flag after synchronising and map it with
+ *     pa_status_from_device_flag.
+ *   - Layouts (row-major, innermost last):
+ *       q, out          [B][Hq][D]
+ *       k_pool, v_pool  [num_blocks][block_size][Hkv][D]
+ *       block_tables    [B][max_blocks] int32; entries at logical index
+ *                       >= ceil(seq_lens[b] / block_size) are never read (may be -1)
+ *       seq_lens        [B] int32, tokens of sequence b including this step's token
+ *       key, value      [T][Hkv][D]
+ *       slot_mapping    [T] int64; slot s = physical block (s / block_size), offset
+ *                       (s % block_size); s < 0 skips the token
+ *       pairs           [n][2] int32 (src, dst) physical block ids
+ *   - Query head h reads KV head h / (Hq / Hkv) (grouped-query attention).
+ *   - Element types: PA_BF16 (bfloat16 storage, fp32 arithmetic, one final rounding
+ *     to bfloat16) or PA_F32 (fp32 throughout, no TF32).  All of q, pools and out
+ *     share the dtype.  Supported: D in {64, 128}; block_size in {4, 8, 16, 32};
+ *     Hq % Hkv == 0; q/out/pool/key/value pointers 16-byte aligned.
+ */
+#ifndef PAGED_KV_CACHE_350_B200_PA_H
+#define PAGED_KV_CACHE_350_B200_PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same underlying type as cudaStream_t; NULL means the legacy default stream. */
+typedef struct CUstream_st* pa_stream_t;
+
+typedef enum pa_status {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,    /* bad size, pointer, alignment or combination */
+  PA_ERR_UNSUPPORTED = 2,    /* valid but not implemented (e.g. D not in {64,128}) */
+  PA_ERR_OUT_OF_BLOCKS = 3,  /* allocator has no free block; state unchanged */
+  PA_ERR_BAD_BLOCK_ID = 4,   /* device flag: a block id outside [0, num_blocks) */
+  PA_ERR_CUDA = 5,           /* a CUDA runtime call failed (launch, driver entry point) */
+  PA_ERR_NOT_FOUND = 6,      /* allocator: unknown sequence id */
+  PA_ERR_EXISTS = 7,         /* allocator: sequence id already in use */
+  PA_ERR_BAD_SEQ_LEN = 8,    /* device flag: seq_lens[b] outside [0, max_blocks*block_size] */
+  PA_ERR_BAD_SLOT = 9,       /* device flag: slot >= num_blocks*block_size */
+  PA_ERR_TIMEOUT = 10        /* device flag: a bounded pipeline wait gave up */
+} pa_status;
+
+typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
+
+/* Bits a kernel ORs into *dev_err_flag. */
+#define PA_DEVERR_BAD_BLOCK_ID 0x1
+#define PA_DEVERR_BAD_SEQ_LEN 0x2
+#define PA_DEVERR_BAD_SLOT 0x4
+#define PA_DEVERR_TIMEOUT 0x8
+
+/* Static, NUL-terminated description of a status. */
+const char* pa_status_string(pa_status status);
+
+/* Map a device error flag word to the status of its lowest set bit (PA_OK if 0). */
+pa_status pa_status_from_device_flag(int32_t flag);
+
+/* Library version string, e.g. "0.1.0". */
+const char* pa_version(void);
+
+/* ---------------------------------------------------------------------------
+ * Decode attention
+ * ------------------------------------------------------------------------- */
+
+typedef enum pa_decode_path {
+  PA_PATH_AUTO = 0,     /* tensor-core path when eligible, else the CUDA-core path */
+  PA_PATH_GENERIC = 1,  /* CUDA-core path (any supported shape and dtype) */
+  PA_PATH_TENSOR = 2    /* bf16 tensor-core path: Hq/Hkv <= 16, block_size in {8,16,32};
+                           PA_ERR_UNSUPPORTED if not eligible */
+} pa_decode_path;
+
+typedef struct pa_decode_opts {
+  /* Tokens per context partition.  0 = automatic.  Otherwise a positive multiple of
+   * block_size (and of 16 on the tensor-core path).  A sequence longer than one
+   * partition is split; each partition writes a partial (max, sum, unnormalised
+   * output) to the workspace and a reduce kernel merges them by log-sum-exp. */
+  int partition_tokens;
+  int path;             /* pa_decode_path */
+} pa_decode_opts;
+
+/* Bytes of workspace pa_decode needs for a batch of B sequences of at most
+ * max_seq_len tokens.  partition_tokens as in pa_decode_opts (0 = the automatic
+ * choice; its bound holds for every automatic choice).  Returns 0 when no split is
+ * possible and (size_t)-1 for invalid arguments. */
+size_t pa_decode_workspace_size(int B, int Hq, int D, int max_seq_len, int block_size,
+                                int partition_tokens);
+
+/* out[b][h][:] = sum_t softmax_t(scale * q[b][h].k_t) v_t over t < seq_lens[b], with
+ * k_t = k_pool[block_tables[b][t / block_size]][t % block_size][h / (Hq/Hkv)][:]
+ * (v_t likewise).  seq_lens[b] == 0 gives a zero row.  `workspace` may be NULL when
+ * workspace_bytes is 0; with the automatic partitioning an insufficient workspace
+ * makes every sequence a single partition.  dev_err_flag may be NULL. */
+pa_status pa_decode(void* out, const void* q, const void* k_pool, const void* v_pool,
+                    const int32_t* block_tables, const int32_t* seq_lens, int B, int Hq,
+                    int Hkv, int D, int block_size, int max_blocks, int num_blocks,
+                    float scale, pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                    int32_t* dev_err_flag, pa_stream_t stream);
+
+/* What pa_decode_ex would launch for these arguments (host only, queues nothing):
+ * the path taken, the partition size, the partitions of the longest possible
+ * sequence, and the number of kernel launches (1, or 2 with the reduce). */
+typedef struct pa_decode_plan_info {
+  int path;              /* PA_PATH_GENERIC or PA_PATH_TENSOR */
+  int partition_tokens;
+  int max_parts;
+  int launches;
+} pa_decode_plan_info;
+
+pa_status pa_decode_plan(int B, int Hq, int Hkv, int D, int block_size, int max_blocks,
+                         pa_dtype dtype, size_t workspace_bytes, const pa_decode_opts* opts,
+                         pa_decode_plan_info* info);
+
+/* pa_decode with explicit options (opts may be NULL = defaults). */
+pa_status pa_decode_ex(void* out, const void* q, const void* k_pool, const void* v_pool,
+                       const int32_t* block_tables, const int32_t* seq_lens, int B, int Hq,
+                       int Hkv, int D, int block_size, int max_blocks, int num_blocks,
+                       float scale, pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                       int32_t* dev_err_flag, pa_stream_t stream, const pa_decode_opts* opts);
+
+/* ---------------------------------------------------------------------------
+ * Cache maintenance
+ * ------------------------------------------------------------------------- */
+
+/* For t < T with s = slot_mapping[t] >= 0: k_pool[s / block_size][s % block_size][:][:]
+ * = key[t][:][:], same for value.  Non-negative slots must be distinct within a call. */
+pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_pool, void* v_pool,
+                               const int64_t* slot_mapping, int T, int Hkv, int D,
+                               int block_size, int num_blocks, pa_dtype dtype,
+                               int32_t* dev_err_flag, pa_stream_t stream);
+
+/* For i < n: block pairs[i][1] of both pools = block pairs[i][0] (all block_size slots,
+ * every head).  `pairs` is a DEVICE array.  Destinations must be distinct and no
+ * destination may also be a source in the same call. */
+pa_status pa_copy_blocks(void* k_pool, void* v_pool, const int32_t* pairs, int n,
+                         int block_size, int Hkv, int D, int num_blocks, pa_dtype dtype,
+                         int32_t* dev_err_flag, pa_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Host block allocator (opaque, library-owned; destroy with pa_alloc_destroy)
+ *
+ * Policy: the free list is a LIFO stack whose initial pops return 0, 1, 2, ... or,
+ * with shuffle_seed != 0, a Fisher-Yates permutation drawn from splitmix64(seed)
+ * (index next() % (i+1) for i = n-1 .. 1).  A sequence of n tokens holds
+ * ceil(n / block_size) blocks.  Appending takes a fresh block when the last block is
+ * full (or absent); when the last block is partial and shared (refcount > 1) the
+ * append copies on write: it takes a fresh block dst, reports (src, dst), decrements
+ * refcount(src) and points the table at dst.  Freed blocks are pushed in table order
+ * when their refcount reaches 0.  A failing call changes no state.  Not thread-safe.
+ * ------------------------------------------------------------------------- */
+
+typedef struct pa_allocator pa_allocator;
+
+pa_status pa_alloc_create(int num_blocks, int block_size, uint64_t shuffle_seed,
+                          pa_allocator** out);
+/* Like pa_alloc_create with an explicit initial pop order (a permutation of
+ * [0, num_blocks), host array, copied). */
+pa_status pa_alloc_create_ordered(int num_blocks, int block_size, const int32_t* pop_order,
+                                  pa_allocator** out);
+void pa_alloc_destroy(pa_allocator* a);
+
+/* Register a sequence already holding num_tokens tokens: ceil(num_tokens/bs) fresh blocks. */
+pa_status pa_alloc_add_seq(pa_allocator* a, int64_t seq_id, int num_tokens);
+/* child shares every block of parent (refcount +1 each) and its token count. */
+pa_status pa_alloc_fork(pa_allocator* a, int64_t parent_id, int64_t child_id);
+/* Reserve the slot of the sequence's next token; *cow_src = *cow_dst = -1 if no copy. */
+pa_status pa_alloc_append_slot(pa_allocator* a, int64_t seq_id, int64_t* slot,
+                               int32_t* cow_src, int32_t* cow_dst);
+/* append_slot for n distinct sequences, in order, all or nothing: on any error no
+ * sequence is changed.  Writes slot_mapping[n]; copy pairs to cow_pairs[2*k..] (room
+ * for n pairs) and their count to *n_pairs. */
+pa_status pa_alloc_append_slots(pa_allocator* a, const int64_t* seq_ids, int n,
+                                int64_t* slot_mapping, int32_t* cow_pairs, int* n_pairs);
+/* Drop a sequence; blocks whose refcount reaches 0 return to the free list. */
+pa_status pa_alloc_free_seq(pa_allocator* a, int64_t seq_id);
+
+/* Copy the sequence's table (up to cap entries) to out; *n = its length, *num_tokens. */
+pa_status pa_alloc_block_table(const pa_allocator* a, int64_t seq_id, int32_t* out, int cap,
+                               int* n, int* num_tokens);
+/* Fill block_tables[n][max_blocks] (padded with -1) and seq_lens[n] for n sequences. */
+pa_status pa_alloc_block_tables(const pa_allocator* a, const int64_t* seq_ids, int n,
+                                int32_t* block_tables, int max_blocks, int32_t* seq_lens);
+int pa_alloc_refcount(const pa_allocator* a, int32_t block);   /* -1 if out of range */
+int pa_alloc_num_free(const pa_allocator* a);
+/* Sum over live sequences of (blocks * block_size - tokens). */
+int64_t pa_alloc_internal_waste_slots(const pa_allocator* a);
+/* Free stack bottom-to-top into out (up to cap); returns its length. */
+int pa_alloc_free_list(const pa_allocator* a, int32_t* out, int cap);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGED_KV_CACHE_350_B200_PA_H */

@@ -1,0 +1,333 @@
+"""ctypes binding of libpagedattn (include/pa.h): argument marshalling only.
+
+Every function keeps the C name and takes torch tensors (device memory and
+streams come from PyTorch); shapes are read from the tensors, pointers and
+sizes are passed to the C ABI, and a non-OK status raises ``PAError``.  No
+computation happens here.  If the shared library is missing this module
+raises at import: there is no fallback path.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedattn.so")
+
+# pa_status
+PA_OK = 0
+PA_ERR_INVALID_ARG = 1
+PA_ERR_UNSUPPORTED = 2
+PA_ERR_OUT_OF_BLOCKS = 3
+PA_ERR_BAD_BLOCK_ID = 4
+PA_ERR_CUDA = 5
+PA_ERR_NOT_FOUND = 6
+PA_ERR_EXISTS = 7
+PA_ERR_BAD_SEQ_LEN = 8
+PA_ERR_BAD_SLOT = 9
+PA_ERR_TIMEOUT = 10
+
+# pa_dtype
+PA_F32 = 0
+PA_BF16 = 1
+
+# pa_decode_path
+PA_PATH_AUTO = 0
+PA_PATH_GENERIC = 1
+PA_PATH_TENSOR = 2
+
+# device error flag bits
+PA_DEVERR_BAD_BLOCK_ID = 0x1
+PA_DEVERR_BAD_SEQ_LEN = 0x2
+PA_DEVERR_BAD_SLOT = 0x4
+PA_DEVERR_TIMEOUT = 0x8
+
+
+class PAError(RuntimeError):
+    def __init__(self, status, where=""):
+        self.status = status
+        msg = lib.pa_status_string(status).decode() if lib is not None else str(status)
+        super().__init__(f"{where}: {msg} (status {status})" if where else msg)
+
+
+class pa_decode_opts(ctypes.Structure):
+    _fields_ = [("partition_tokens", ctypes.c_int), ("path", ctypes.c_int)]
+
+
+class pa_decode_plan_info(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int), ("partition_tokens", ctypes.c_int),
+                ("max_parts", ctypes.c_int), ("launches", ctypes.c_int)]
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(
+            f"libpagedattn.so not found at {_LIB_PATH}; build it with "
+            "`python -m paged_kv_cache_350_b200.build` (there is no non-CUDA fallback)")
+    L = ctypes.CDLL(_LIB_PATH)
+    vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    pi32 = ctypes.POINTER(ctypes.c_int32)
+    pi64 = ctypes.POINTER(ctypes.c_int64)
+    pint = ctypes.POINTER(ctypes.c_int)
+    sig = {
+        "pa_status_string": (ctypes.c_char_p, [i32]),
+        "pa_status_from_device_flag": (i32, [ctypes.c_int32]),
+        "pa_version": (ctypes.c_char_p, []),
+        "pa_decode_workspace_size": (sz, [i32, i32, i32, i32, i32, i32]),
+        "pa_decode": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32,
+                            vp, sz, vp, vp]),
+        "pa_decode_ex": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32,
+                               i32, vp, sz, vp, vp, ctypes.POINTER(pa_decode_opts)]),
+        "pa_decode_plan": (i32, [i32, i32, i32, i32, i32, i32, i32, sz,
+                                 ctypes.POINTER(pa_decode_opts), ctypes.POINTER(pa_decode_plan_info)]),
+        "pa_reshape_and_cache": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]),
+        "pa_copy_blocks": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]),
+        "pa_alloc_create": (i32, [i32, i32, ctypes.c_uint64, ctypes.POINTER(vp)]),
+        "pa_alloc_create_ordered": (i32, [i32, i32, pi32, ctypes.POINTER(vp)]),
+        "pa_alloc_destroy": (None, [vp]),
+        "pa_alloc_add_seq": (i32, [vp, i64, i32]),
+        "pa_alloc_fork": (i32, [vp, i64, i64]),
+        "pa_alloc_append_slot": (i32, [vp, i64, pi64, pi32, pi32]),
+        "pa_alloc_append_slots": (i32, [vp, pi64, i32, pi64, pi32, pint]),
+        "pa_alloc_free_seq": (i32, [vp, i64]),
+        "pa_alloc_block_table": (i32, [vp, i64, pi32, i32, pint, pint]),
+        "pa_alloc_block_tables": (i32, [vp, pi64, i32, pi32, i32, pi32]),
+        "pa_alloc_refcount": (i32, [vp, ctypes.c_int32]),
+        "pa_alloc_num_free": (i32, [vp]),
+        "pa_alloc_internal_waste_slots": (i64, [vp]),
+        "pa_alloc_free_list": (i32, [vp, pi32, i32]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    return L
+
+
+lib = None
+lib = _load()
+
+#: every symbol include/pa.h declares
+EXPORTED = (
+    "pa_status_string", "pa_status_from_device_flag", "pa_version", "pa_decode_workspace_size",
+    "pa_decode", "pa_decode_ex", "pa_decode_plan", "pa_reshape_and_cache", "pa_copy_blocks", "pa_alloc_create",
+    "pa_alloc_create_ordered", "pa_alloc_destroy", "pa_alloc_add_seq", "pa_alloc_fork",
+    "pa_alloc_append_slot", "pa_alloc_append_slots", "pa_alloc_free_seq", "pa_alloc_block_table",
+    "pa_alloc_block_tables", "pa_alloc_refcount", "pa_alloc_num_free",
+    "pa_alloc_internal_waste_slots", "pa_alloc_free_list",
+)
+
+
+def _check(status, where):
+    if status != PA_OK:
+        raise PAError(status, where)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dtype_of(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return PA_BF16
+    if t.dtype == torch.float32:
+        return PA_F32
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def _need(cond, msg):
+    if not cond:
+        raise ValueError(msg)
+
+
+# ---------------------------------------------------------------------------
+# decode
+# ---------------------------------------------------------------------------
+
+def pa_decode_workspace_size(B, Hq, D, max_seq_len, block_size, partition_tokens=0):
+    n = lib.pa_decode_workspace_size(B, Hq, D, max_seq_len, block_size, partition_tokens)
+    if n == ctypes.c_size_t(-1).value:
+        raise PAError(PA_ERR_INVALID_ARG, "pa_decode_workspace_size")
+    return n
+
+
+def pa_decode_plan(B, Hq, Hkv, D, block_size, max_blocks, dtype, workspace_bytes=0,
+                   partition_tokens=0, path=PA_PATH_AUTO):
+    """dict(path, partition_tokens, max_parts, launches) that pa_decode would use."""
+    info = pa_decode_plan_info()
+    opts = pa_decode_opts(partition_tokens, path)
+    _check(lib.pa_decode_plan(B, Hq, Hkv, D, block_size, max_blocks, dtype, workspace_bytes,
+                              ctypes.byref(opts), ctypes.byref(info)), "pa_decode_plan")
+    return {"path": info.path, "partition_tokens": info.partition_tokens,
+            "max_parts": info.max_parts, "launches": info.launches}
+
+
+def pa_decode(out, q, k_pool, v_pool, block_tables, seq_lens, scale, workspace=None,
+              err_flag=None, stream=None, partition_tokens=0, path=PA_PATH_AUTO):
+    """out[B,Hq,D] = paged decode attention of q[B,Hq,D] over the pools (see include/pa.h)."""
+    import torch
+    _need(q.dim() == 3 and out.shape == q.shape, "q/out must be [B, Hq, D]")
+    _need(k_pool.dim() == 4 and v_pool.shape == k_pool.shape, "pools must be [NB, bs, Hkv, D]")
+    _need(block_tables.dim() == 2 and block_tables.dtype == torch.int32, "block_tables int32 [B, MB]")
+    _need(seq_lens.dtype == torch.int32 and seq_lens.numel() == q.shape[0], "seq_lens int32 [B]")
+    for t in (out, q, k_pool, v_pool, block_tables, seq_lens):
+        _need(t.is_contiguous(), "tensors must be contiguous")
+    _need(q.dtype == out.dtype == k_pool.dtype == v_pool.dtype, "q, out and pools share a dtype")
+    B, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_pool.shape
+    _need(D2 == D, "head dim mismatch")
+    _need(block_tables.shape[0] == B, "block_tables rows != B")
+    wbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    opts = pa_decode_opts(partition_tokens, path)
+    st = lib.pa_decode_ex(_ptr(out), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables),
+                          _ptr(seq_lens), B, Hq, Hkv, D, bs, block_tables.shape[1], NB,
+                          float(scale), _dtype_of(q), _ptr(workspace), wbytes, _ptr(err_flag),
+                          _stream(stream), ctypes.byref(opts))
+    _check(st, "pa_decode")
+    return out
+
+
+def pa_reshape_and_cache(key, value, k_pool, v_pool, slot_mapping, err_flag=None, stream=None):
+    """Scatter key/value [T,Hkv,D] into the pools at slot_mapping[T] (int64; < 0 skips)."""
+    import torch
+    _need(key.dim() == 3 and value.shape == key.shape, "key/value must be [T, Hkv, D]")
+    _need(slot_mapping.dtype == torch.int64 and slot_mapping.numel() == key.shape[0],
+          "slot_mapping int64 [T]")
+    _need(key.dtype == value.dtype == k_pool.dtype == v_pool.dtype, "dtype mismatch")
+    for t in (key, value, k_pool, v_pool, slot_mapping):
+        _need(t.is_contiguous(), "tensors must be contiguous")
+    NB, bs, Hkv, D = k_pool.shape
+    _need(key.shape[1:] == (Hkv, D), "key rows must be [Hkv, D] of the pool")
+    st = lib.pa_reshape_and_cache(_ptr(key), _ptr(value), _ptr(k_pool), _ptr(v_pool),
+                                  _ptr(slot_mapping), key.shape[0], Hkv, D, bs, NB,
+                                  _dtype_of(key), _ptr(err_flag), _stream(stream))
+    _check(st, "pa_reshape_and_cache")
+
+
+def pa_copy_blocks(k_pool, v_pool, pairs, err_flag=None, stream=None):
+    """Copy whole blocks pairs[i][0] -> pairs[i][1] (device int32 [n, 2]) in both pools."""
+    import torch
+    _need(pairs.dtype == torch.int32 and (pairs.numel() == 0 or pairs.shape[-1] == 2),
+          "pairs int32 [n, 2]")
+    _need(pairs.is_contiguous() and k_pool.is_contiguous() and v_pool.is_contiguous(),
+          "tensors must be contiguous")
+    NB, bs, Hkv, D = k_pool.shape
+    n = pairs.numel() // 2
+    st = lib.pa_copy_blocks(_ptr(k_pool), _ptr(v_pool), _ptr(pairs), n, bs, Hkv, D, NB,
+                            _dtype_of(k_pool), _ptr(err_flag), _stream(stream))
+    _check(st, "pa_copy_blocks")
+
+
+def pa_status_from_device_flag(flag):
+    return lib.pa_status_from_device_flag(int(flag))
+
+
+# ---------------------------------------------------------------------------
+# host allocator
+# ---------------------------------------------------------------------------
+
+def _i32p(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
+def _i64p(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
+
+
+class Allocator:
+    """The pa_alloc_* block allocator (C++), one handle per pool."""
+
+    def __init__(self, num_blocks, block_size, shuffle_seed=0, pop_order=None):
+        h = ctypes.c_void_p()
+        if pop_order is not None:
+            order = np.ascontiguousarray(pop_order, dtype=np.int32)
+            _need(order.size == num_blocks, "pop_order must list every block")
+            st = lib.pa_alloc_create_ordered(num_blocks, block_size, _i32p(order), ctypes.byref(h))
+        else:
+            st = lib.pa_alloc_create(num_blocks, block_size, ctypes.c_uint64(shuffle_seed),
+                                     ctypes.byref(h))
+        _check(st, "pa_alloc_create")
+        self._h = h
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib.pa_alloc_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def add_seq(self, seq_id, num_tokens):
+        _check(lib.pa_alloc_add_seq(self._h, seq_id, num_tokens), "pa_alloc_add_seq")
+
+    def fork(self, parent_id, child_id):
+        _check(lib.pa_alloc_fork(self._h, parent_id, child_id), "pa_alloc_fork")
+
+    def append_slot(self, seq_id):
+        slot, src, dst = ctypes.c_int64(), ctypes.c_int32(), ctypes.c_int32()
+        _check(lib.pa_alloc_append_slot(self._h, seq_id, ctypes.byref(slot), ctypes.byref(src),
+                                        ctypes.byref(dst)), "pa_alloc_append_slot")
+        return slot.value, src.value, dst.value
+
+    def append_slots(self, seq_ids, slot_out=None, pairs_out=None):
+        """append_slot for every id, all or nothing; returns (slots int64[n], pairs int32[k,2])."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = ids.size
+        slots = slot_out if slot_out is not None else np.empty(n, dtype=np.int64)
+        pairs = pairs_out if pairs_out is not None else np.empty((max(n, 1), 2), dtype=np.int32)
+        k = ctypes.c_int()
+        _check(lib.pa_alloc_append_slots(self._h, _i64p(ids), n, _i64p(slots), _i32p(pairs),
+                                         ctypes.byref(k)), "pa_alloc_append_slots")
+        return slots[:n], pairs[: k.value]
+
+    def free_seq(self, seq_id):
+        _check(lib.pa_alloc_free_seq(self._h, seq_id), "pa_alloc_free_seq")
+
+    def block_table(self, seq_id):
+        n, ntok = ctypes.c_int(), ctypes.c_int()
+        _check(lib.pa_alloc_block_table(self._h, seq_id, None, 0, ctypes.byref(n),
+                                        ctypes.byref(ntok)), "pa_alloc_block_table")
+        out = np.empty(max(n.value, 1), dtype=np.int32)
+        _check(lib.pa_alloc_block_table(self._h, seq_id, _i32p(out), n.value, ctypes.byref(n),
+                                        ctypes.byref(ntok)), "pa_alloc_block_table")
+        return out[: n.value].tolist(), ntok.value
+
+    def block_tables(self, seq_ids, max_blocks, tables_out=None, lens_out=None):
+        """Padded tables int32[n, max_blocks] (-1 tail) and seq_lens int32[n]."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = ids.size
+        tables = tables_out if tables_out is not None else np.empty((n, max_blocks), np.int32)
+        lens = lens_out if lens_out is not None else np.empty(n, np.int32)
+        _check(lib.pa_alloc_block_tables(self._h, _i64p(ids), n, _i32p(tables), max_blocks,
+                                         _i32p(lens)), "pa_alloc_block_tables")
+        return tables, lens
+
+    def refcount(self, block):
+        return lib.pa_alloc_refcount(self._h, block)
+
+    def num_free(self):
+        return lib.pa_alloc_num_free(self._h)
+
+    def internal_waste_slots(self):
+        return lib.pa_alloc_internal_waste_slots(self._h)
+
+    def free_list(self):
+        n = lib.pa_alloc_free_list(self._h, None, 0)
+        out = np.empty(max(n, 1), dtype=np.int32)
+        lib.pa_alloc_free_list(self._h, _i32p(out), n)
+        return out[:n].tolist()

@@ -1,0 +1,285 @@
+// Host block allocator with reference counts for a paged KV pool.
+//
+// Blocks are handed out on demand, one when the previous is full ("PagedAttention"
+// concept card, 带来的能力; "什么是 LLM 中的分页注意力", 使用分页注意力).  A fork shares
+// every block and raises its refcount; a block returns to the free list when its count
+// reaches 0; before a sequence writes into a partial block it still shares, the block
+// is copied (copy on write) so the sibling's prefix stays intact ("深入解析
+// PagedAttention", 核心创新 / 多序列共享; concept card, 实现要点).  The exact policy
+// (LIFO free list, splitmix64 Fisher-Yates shuffle, when a copy happens) is stated in
+// include/pa.h.  Every failing call leaves the state unchanged.
+
+#include <algorithm>
+#include <cstring>
+#include <new>
+#include <unordered_map>
+#include <unordered_set>
+#include <vector>
+
+#include "pa.h"
+
+namespace {
+
+struct Seq {
+  std::vector<int32_t> table;
+  int64_t ntok = 0;
+};
+
+// splitmix64 (Steele, Lea & Flood, OOPSLA 2014).
+struct SplitMix64 {
+  uint64_t state;
+  uint64_t next() {
+    uint64_t z = (state += 0x9E3779B97F4A7C15ull);
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+  }
+};
+
+}  // namespace
+
+struct pa_allocator {
+  int num_blocks = 0;
+  int block_size = 0;
+  std::vector<int32_t> free_stack;  // back() is popped first
+  std::vector<int32_t> ref;
+  std::unordered_map<int64_t, Seq> seqs;
+
+  int32_t pop() {
+    int32_t b = free_stack.back();
+    free_stack.pop_back();
+    ref[b] = 1;
+    return b;
+  }
+};
+
+namespace {
+
+bool init_from_order(pa_allocator* a, int num_blocks, int block_size,
+                     const std::vector<int32_t>& pop_order) {
+  a->num_blocks = num_blocks;
+  a->block_size = block_size;
+  a->ref.assign(num_blocks, 0);
+  a->free_stack.assign(pop_order.rbegin(), pop_order.rend());
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_alloc_create(int num_blocks, int block_size, uint64_t shuffle_seed,
+                          pa_allocator** out) {
+  if (!out || num_blocks <= 0 || block_size <= 0) return PA_ERR_INVALID_ARG;
+  std::vector<int32_t> order(num_blocks);
+  for (int i = 0; i < num_blocks; ++i) order[i] = i;
+  if (shuffle_seed != 0) {
+    SplitMix64 rng{shuffle_seed};
+    for (int i = num_blocks - 1; i > 0; --i) {
+      int j = static_cast<int>(rng.next() % static_cast<uint64_t>(i + 1));
+      std::swap(order[i], order[j]);
+    }
+  }
+  pa_allocator* a = new (std::nothrow) pa_allocator();
+  if (!a) return PA_ERR_INVALID_ARG;
+  init_from_order(a, num_blocks, block_size, order);
+  *out = a;
+  return PA_OK;
+}
+
+pa_status pa_alloc_create_ordered(int num_blocks, int block_size, const int32_t* pop_order,
+                                  pa_allocator** out) {
+  if (!out || !pop_order || num_blocks <= 0 || block_size <= 0) return PA_ERR_INVALID_ARG;
+  std::vector<int32_t> order(pop_order, pop_order + num_blocks);
+  std::vector<char> seen(num_blocks, 0);
+  for (int32_t b : order) {
+    if (b < 0 || b >= num_blocks || seen[b]) return PA_ERR_INVALID_ARG;
+    seen[b] = 1;
+  }
+  pa_allocator* a = new (std::nothrow) pa_allocator();
+  if (!a) return PA_ERR_INVALID_ARG;
+  init_from_order(a, num_blocks, block_size, order);
+  *out = a;
+  return PA_OK;
+}
+
+void pa_alloc_destroy(pa_allocator* a) { delete a; }
+
+pa_status pa_alloc_add_seq(pa_allocator* a, int64_t seq_id, int num_tokens) {
+  if (!a || num_tokens < 0) return PA_ERR_INVALID_ARG;
+  if (a->seqs.count(seq_id)) return PA_ERR_EXISTS;
+  int64_t need = (static_cast<int64_t>(num_tokens) + a->block_size - 1) / a->block_size;
+  if (need > static_cast<int64_t>(a->free_stack.size())) return PA_ERR_OUT_OF_BLOCKS;
+  Seq s;
+  s.table.reserve(need + 1);
+  for (int64_t i = 0; i < need; ++i) s.table.push_back(a->pop());
+  s.ntok = num_tokens;
+  a->seqs.emplace(seq_id, std::move(s));
+  return PA_OK;
+}
+
+pa_status pa_alloc_fork(pa_allocator* a, int64_t parent_id, int64_t child_id) {
+  if (!a) return PA_ERR_INVALID_ARG;
+  auto it = a->seqs.find(parent_id);
+  if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
+  if (a->seqs.count(child_id)) return PA_ERR_EXISTS;
+  Seq child = it->second;  // copy before emplace (rehash may move the parent)
+  for (int32_t b : child.table) a->ref[b] += 1;
+  a->seqs.emplace(child_id, std::move(child));
+  return PA_OK;
+}
+
+static void append_one(pa_allocator* a, Seq& s, int64_t* slot, int32_t* src, int32_t* dst) {
+  const int bs = a->block_size;
+  const int off = static_cast<int>(s.ntok % bs);
+  int32_t phys;
+  *src = -1;
+  *dst = -1;
+  if (off == 0) {
+    phys = a->pop();
+    s.table.push_back(phys);
+  } else {
+    int32_t last = s.table.back();
+    if (a->ref[last] > 1) {
+      phys = a->pop();
+      a->ref[last] -= 1;
+      s.table.back() = phys;
+      *src = last;
+      *dst = phys;
+    } else {
+      phys = last;
+    }
+  }
+  s.ntok += 1;
+  *slot = static_cast<int64_t>(phys) * bs + off;
+}
+
+pa_status pa_alloc_append_slot(pa_allocator* a, int64_t seq_id, int64_t* slot,
+                               int32_t* cow_src, int32_t* cow_dst) {
+  if (!a || !slot || !cow_src || !cow_dst) return PA_ERR_INVALID_ARG;
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
+  Seq& s = it->second;
+  const bool needs_block =
+      (s.ntok % a->block_size == 0) || (a->ref[s.table.back()] > 1);
+  if (needs_block && a->free_stack.empty()) return PA_ERR_OUT_OF_BLOCKS;
+  append_one(a, s, slot, cow_src, cow_dst);
+  return PA_OK;
+}
+
+pa_status pa_alloc_append_slots(pa_allocator* a, const int64_t* seq_ids, int n,
+                                int64_t* slot_mapping, int32_t* cow_pairs, int* n_pairs) {
+  if (!a || n < 0 || (n > 0 && (!seq_ids || !slot_mapping || !cow_pairs)) || !n_pairs)
+    return PA_ERR_INVALID_ARG;
+  // Dry run: resolve every sequence, reject duplicates, and count the fresh blocks the
+  // batch takes, replaying the refcount drops of earlier copies in the same batch.
+  std::vector<Seq*> rows(n);
+  std::unordered_set<int64_t> seen;
+  seen.reserve(static_cast<size_t>(n) * 2);
+  std::unordered_map<int32_t, int> dropped;
+  int64_t need = 0;
+  for (int i = 0; i < n; ++i) {
+    auto it = a->seqs.find(seq_ids[i]);
+    if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
+    if (!seen.insert(seq_ids[i]).second) return PA_ERR_INVALID_ARG;
+    Seq& s = it->second;
+    rows[i] = &s;
+    if (s.ntok % a->block_size == 0) {
+      need += 1;
+    } else {
+      int32_t last = s.table.back();
+      auto d = dropped.find(last);
+      int drop = d == dropped.end() ? 0 : d->second;
+      if (a->ref[last] - drop > 1) {
+        need += 1;
+        dropped[last] = drop + 1;
+      }
+    }
+  }
+  if (need > static_cast<int64_t>(a->free_stack.size())) return PA_ERR_OUT_OF_BLOCKS;
+  int np = 0;
+  for (int i = 0; i < n; ++i) {
+    int32_t src, dst;
+    append_one(a, *rows[i], &slot_mapping[i], &src, &dst);
+    if (src >= 0) {
+      cow_pairs[2 * np] = src;
+      cow_pairs[2 * np + 1] = dst;
+      ++np;
+    }
+  }
+  *n_pairs = np;
+  return PA_OK;
+}
+
+pa_status pa_alloc_free_seq(pa_allocator* a, int64_t seq_id) {
+  if (!a) return PA_ERR_INVALID_ARG;
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
+  for (int32_t b : it->second.table) {
+    if (--a->ref[b] == 0) a->free_stack.push_back(b);
+  }
+  a->seqs.erase(it);
+  return PA_OK;
+}
+
+pa_status pa_alloc_block_table(const pa_allocator* a, int64_t seq_id, int32_t* out, int cap,
+                               int* n, int* num_tokens) {
+  if (!a || !n || !num_tokens || cap < 0 || (cap > 0 && !out)) return PA_ERR_INVALID_ARG;
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
+  const Seq& s = it->second;
+  int len = static_cast<int>(s.table.size());
+  int m = std::min(len, cap);
+  if (m > 0) std::memcpy(out, s.table.data(), sizeof(int32_t) * m);
+  *n = len;
+  *num_tokens = static_cast<int>(s.ntok);
+  return PA_OK;
+}
+
+pa_status pa_alloc_block_tables(const pa_allocator* a, const int64_t* seq_ids, int n,
+                                int32_t* block_tables, int max_blocks, int32_t* seq_lens) {
+  if (!a || n < 0 || max_blocks <= 0 ||
+      (n > 0 && (!seq_ids || !block_tables || !seq_lens)))
+    return PA_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    auto it = a->seqs.find(seq_ids[i]);
+    if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
+    if (static_cast<int>(it->second.table.size()) > max_blocks) return PA_ERR_INVALID_ARG;
+  }
+  for (int i = 0; i < n; ++i) {
+    const Seq& s = a->seqs.find(seq_ids[i])->second;
+    int32_t* row = block_tables + static_cast<int64_t>(i) * max_blocks;
+    int len = static_cast<int>(s.table.size());
+    if (len) std::memcpy(row, s.table.data(), sizeof(int32_t) * len);
+    for (int j = len; j < max_blocks; ++j) row[j] = -1;
+    seq_lens[i] = static_cast<int32_t>(s.ntok);
+  }
+  return PA_OK;
+}
+
+int pa_alloc_refcount(const pa_allocator* a, int32_t block) {
+  if (!a || block < 0 || block >= a->num_blocks) return -1;
+  return a->ref[block];
+}
+
+int pa_alloc_num_free(const pa_allocator* a) {
+  return a ? static_cast<int>(a->free_stack.size()) : -1;
+}
+
+int64_t pa_alloc_internal_waste_slots(const pa_allocator* a) {
+  if (!a) return -1;
+  int64_t w = 0;
+  for (const auto& kv : a->seqs)
+    w += static_cast<int64_t>(kv.second.table.size()) * a->block_size - kv.second.ntok;
+  return w;
+}
+
+int pa_alloc_free_list(const pa_allocator* a, int32_t* out, int cap) {
+  if (!a) return -1;
+  int len = static_cast<int>(a->free_stack.size());
+  int m = std::min(len, cap);
+  if (m > 0 && out) std::memcpy(out, a->free_stack.data(), sizeof(int32_t) * m);
+  return len;
+}
+
+}  // extern "C"

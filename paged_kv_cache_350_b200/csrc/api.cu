@@ -1,0 +1,241 @@
+// C ABI of libpagedattn: argument validation, path selection, workspace carving.
+// Every check happens on the host before anything is queued; a failing call queues
+// nothing.  See include/pa.h for the contract of each entry point.
+
+#include <cmath>
+#include <cstdint>
+
+#include "pa.h"
+#include "pa_internal.h"
+
+namespace {
+
+// Smallest context partition the automatic policy ever picks; pa_decode_workspace_size
+// with partition_tokens == 0 sizes the workspace for it, which bounds every automatic
+// choice.
+constexpr int kAutoMinPartition = 512;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool block_size_ok(int bs) { return bs == 4 || bs == 8 || bs == 16 || bs == 32; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+// Automatic partition size: 512 tokens, grown for very long contexts so that a
+// sequence splits into at most ~64 partitions (bounding the reduce traffic).
+int auto_partition(int64_t max_seq, int tile) {
+  if (max_seq <= kAutoMinPartition) return static_cast<int>(round_up(max_seq > 0 ? max_seq : 1, tile));
+  int64_t p = round_up(ceil_div(max_seq, 64), kAutoMinPartition);
+  if (p < kAutoMinPartition) p = kAutoMinPartition;
+  return static_cast<int>(round_up(p, tile));
+}
+
+size_t workspace_bytes_for(int64_t B, int64_t Hq, int64_t D, int64_t parts) {
+  if (parts <= 1) return 0;
+  const int64_t ml = round_up(B * Hq * parts * 2 * 4, 256);
+  const int64_t acc = B * Hq * parts * D * 4;
+  return static_cast<size_t>(ml + acc);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pa_status_string(pa_status s) {
+  switch (s) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID_ARG: return "invalid argument";
+    case PA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case PA_ERR_OUT_OF_BLOCKS: return "no free block left in the pool";
+    case PA_ERR_BAD_BLOCK_ID: return "block id outside [0, num_blocks)";
+    case PA_ERR_CUDA: return "CUDA runtime error";
+    case PA_ERR_NOT_FOUND: return "unknown sequence id";
+    case PA_ERR_EXISTS: return "sequence id already exists";
+    case PA_ERR_BAD_SEQ_LEN: return "sequence length outside [0, max_blocks*block_size]";
+    case PA_ERR_BAD_SLOT: return "slot outside the pool";
+    case PA_ERR_TIMEOUT: return "a bounded device wait expired";
+  }
+  return "unknown status";
+}
+
+pa_status pa_status_from_device_flag(int32_t flag) {
+  if (flag == 0) return PA_OK;
+  if (flag & PA_DEVERR_BAD_BLOCK_ID) return PA_ERR_BAD_BLOCK_ID;
+  if (flag & PA_DEVERR_BAD_SEQ_LEN) return PA_ERR_BAD_SEQ_LEN;
+  if (flag & PA_DEVERR_BAD_SLOT) return PA_ERR_BAD_SLOT;
+  if (flag & PA_DEVERR_TIMEOUT) return PA_ERR_TIMEOUT;
+  return PA_ERR_INVALID_ARG;
+}
+
+const char* pa_version(void) { return "0.1.0"; }
+
+size_t pa_decode_workspace_size(int B, int Hq, int D, int max_seq_len, int block_size,
+                                int partition_tokens) {
+  if (B < 0 || Hq <= 0 || D <= 0 || max_seq_len < 0 || !block_size_ok(block_size) ||
+      partition_tokens < 0 || (partition_tokens > 0 && partition_tokens % block_size != 0))
+    return static_cast<size_t>(-1);
+  const int64_t P = partition_tokens > 0 ? partition_tokens : kAutoMinPartition;
+  return workspace_bytes_for(B, Hq, D, ceil_div(max_seq_len, P));
+}
+
+// Shape/dtype checks and the launch plan shared by pa_decode_plan and pa_decode_ex.
+static pa_status plan_decode(int B, int Hq, int Hkv, int D, int block_size, int max_blocks,
+                             int num_blocks, float scale, pa_dtype dtype, bool have_ws,
+                             size_t workspace_bytes, const pa_decode_opts* opts,
+                             pa_decode_plan_info* info) {
+  const int partition = opts ? opts->partition_tokens : 0;
+  const int path = opts ? opts->path : PA_PATH_AUTO;
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || max_blocks <= 0 || num_blocks <= 0 ||
+      block_size <= 0 || !std::isfinite(scale) || partition < 0 ||
+      (path != PA_PATH_AUTO && path != PA_PATH_GENERIC && path != PA_PATH_TENSOR) ||
+      (dtype != PA_F32 && dtype != PA_BF16))
+    return PA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return PA_ERR_UNSUPPORTED;
+  if (!block_size_ok(block_size)) return PA_ERR_UNSUPPORTED;
+  if (partition > 0 && partition % block_size != 0) return PA_ERR_INVALID_ARG;
+  const int64_t max_seq = static_cast<int64_t>(max_blocks) * block_size;
+  if (max_seq > 0x7fffffffLL) return PA_ERR_INVALID_ARG;
+
+  const int G = Hq / Hkv;
+  bool use_tc = false;
+  if (path != PA_PATH_GENERIC && pa::tc_eligible(G, D, block_size, dtype)) {
+    const int tile = block_size > 16 ? block_size : 16;
+    if (partition == 0 || partition % tile == 0) use_tc = true;
+  }
+  if (path == PA_PATH_TENSOR && !use_tc) {
+    if (!pa::tc_eligible(G, D, block_size, dtype)) return PA_ERR_UNSUPPORTED;
+    return PA_ERR_INVALID_ARG;  // partition not a multiple of the 16-token tile
+  }
+  const int tile = use_tc ? (block_size > 16 ? block_size : 16) : block_size;
+  int P = partition > 0 ? partition : auto_partition(max_seq, tile);
+  int64_t parts = ceil_div(max_seq, P);
+  if (parts > 1) {
+    const size_t need = workspace_bytes_for(B, Hq, D, parts);
+    if (!have_ws || workspace_bytes < need) {
+      if (partition > 0) return PA_ERR_INVALID_ARG;
+      P = static_cast<int>(round_up(max_seq, tile));  // single pass, no workspace
+      parts = 1;
+    }
+  }
+  info->path = use_tc ? PA_PATH_TENSOR : PA_PATH_GENERIC;
+  info->partition_tokens = P;
+  info->max_parts = static_cast<int>(parts);
+  info->launches = B == 0 ? 0 : (parts > 1 ? 2 : 1);
+  return PA_OK;
+}
+
+pa_status pa_decode_plan(int B, int Hq, int Hkv, int D, int block_size, int max_blocks,
+                         pa_dtype dtype, size_t workspace_bytes, const pa_decode_opts* opts,
+                         pa_decode_plan_info* info) {
+  if (!info) return PA_ERR_INVALID_ARG;
+  return plan_decode(B, Hq, Hkv, D, block_size, max_blocks, 1, 1.0f, dtype, true,
+                     workspace_bytes, opts, info);
+}
+
+pa_status pa_decode_ex(void* out, const void* q, const void* k_pool, const void* v_pool,
+                       const int32_t* block_tables, const int32_t* seq_lens, int B, int Hq,
+                       int Hkv, int D, int block_size, int max_blocks, int num_blocks,
+                       float scale, pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                       int32_t* dev_err_flag, pa_stream_t stream, const pa_decode_opts* opts) {
+  pa_decode_plan_info plan;
+  const bool have_ws = workspace != nullptr && aligned(workspace, 256);
+  pa_status st = plan_decode(B, Hq, Hkv, D, block_size, max_blocks, num_blocks, scale, dtype,
+                             have_ws, workspace_bytes, opts, &plan);
+  if (st != PA_OK) return st;
+  if (B == 0) return PA_OK;
+  if (!out || !q || !k_pool || !v_pool || !block_tables || !seq_lens) return PA_ERR_INVALID_ARG;
+  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) ||
+      !aligned(block_tables, 4) || !aligned(seq_lens, 4) ||
+      (dev_err_flag && !aligned(dev_err_flag, 4)))
+    return PA_ERR_INVALID_ARG;
+
+  const int parts = plan.max_parts;
+  pa::DecodeParams p{};
+  p.out = out;
+  p.q = q;
+  p.k_pool = k_pool;
+  p.v_pool = v_pool;
+  p.block_tables = block_tables;
+  p.seq_lens = seq_lens;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.D = D;
+  p.block_size = block_size;
+  p.max_blocks = max_blocks;
+  p.num_blocks = num_blocks;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.partition_tokens = plan.partition_tokens;
+  p.max_parts = parts;
+  if (parts > 1) {
+    char* ws = static_cast<char*>(workspace);
+    p.ws_ml = reinterpret_cast<float*>(ws);
+    p.ws_acc = reinterpret_cast<float*>(
+        ws + round_up(static_cast<int64_t>(B) * Hq * parts * 2 * 4, 256));
+  }
+  p.err = dev_err_flag;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = plan.path == PA_PATH_TENSOR ? pa::launch_decode_tc(p, s)
+                                              : pa::launch_decode_generic(p, dtype, s);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_decode(void* out, const void* q, const void* k_pool, const void* v_pool,
+                    const int32_t* block_tables, const int32_t* seq_lens, int B, int Hq,
+                    int Hkv, int D, int block_size, int max_blocks, int num_blocks,
+                    float scale, pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                    int32_t* dev_err_flag, pa_stream_t stream) {
+  return pa_decode_ex(out, q, k_pool, v_pool, block_tables, seq_lens, B, Hq, Hkv, D, block_size,
+                      max_blocks, num_blocks, scale, dtype, workspace, workspace_bytes,
+                      dev_err_flag, stream, nullptr);
+}
+
+pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_pool, void* v_pool,
+                               const int64_t* slot_mapping, int T, int Hkv, int D,
+                               int block_size, int num_blocks, pa_dtype dtype,
+                               int32_t* dev_err_flag, pa_stream_t stream) {
+  if (T < 0 || Hkv <= 0 || num_blocks <= 0 || block_size <= 0 ||
+      (dtype != PA_F32 && dtype != PA_BF16))
+    return PA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return PA_ERR_UNSUPPORTED;
+  if (!block_size_ok(block_size)) return PA_ERR_UNSUPPORTED;
+  if (T == 0) return PA_OK;
+  if (!key || !value || !k_pool || !v_pool || !slot_mapping) return PA_ERR_INVALID_ARG;
+  if (!aligned(key, 16) || !aligned(value, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) ||
+      !aligned(slot_mapping, 8) || (dev_err_flag && !aligned(dev_err_flag, 4)))
+    return PA_ERR_INVALID_ARG;
+  const int esize = dtype == PA_BF16 ? 2 : 4;
+  const int64_t row_bytes = static_cast<int64_t>(Hkv) * D * esize;
+  if (row_bytes > 0x7fffffffLL) return PA_ERR_INVALID_ARG;
+  const int64_t num_slots = static_cast<int64_t>(num_blocks) * block_size;
+  cudaError_t e = pa::launch_reshape_and_cache(
+      key, value, k_pool, v_pool, slot_mapping, T, Hkv, static_cast<int>(row_bytes), num_slots,
+      dev_err_flag, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_copy_blocks(void* k_pool, void* v_pool, const int32_t* pairs, int n,
+                         int block_size, int Hkv, int D, int num_blocks, pa_dtype dtype,
+                         int32_t* dev_err_flag, pa_stream_t stream) {
+  if (n < 0 || Hkv <= 0 || num_blocks <= 0 || block_size <= 0 ||
+      (dtype != PA_F32 && dtype != PA_BF16))
+    return PA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return PA_ERR_UNSUPPORTED;
+  if (!block_size_ok(block_size)) return PA_ERR_UNSUPPORTED;
+  if (n == 0) return PA_OK;
+  if (!k_pool || !v_pool || !pairs) return PA_ERR_INVALID_ARG;
+  if (!aligned(k_pool, 16) || !aligned(v_pool, 16) || !aligned(pairs, 4) ||
+      (dev_err_flag && !aligned(dev_err_flag, 4)))
+    return PA_ERR_INVALID_ARG;
+  const int esize = dtype == PA_BF16 ? 2 : 4;
+  const int64_t block_bytes = static_cast<int64_t>(block_size) * Hkv * D * esize;
+  cudaError_t e = pa::launch_copy_blocks(k_pool, v_pool, pairs, n, block_bytes, num_blocks,
+                                         dev_err_flag, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -9,3 +9,9 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200) and the built library")
     config.addinivalue_line("markers", "slow: full-size workloads")
+
+
+def pytest_sessionstart(session):
+    # The library is a build artefact (not committed): compile it if missing or stale.
+    from paged_kv_cache_350_b200.build import build
+    build()

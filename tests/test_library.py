@@ -1,0 +1,92 @@
+"""CPU: the C-ABI library loads, exports every symbol include/pa.h declares, and
+rejects bad arguments on the host before touching a GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "pa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    from paged_kv_cache_350_b200 import binding
+    syms = declared_symbols()
+    assert len(syms) >= 20
+    for s in syms:
+        assert hasattr(binding.lib, s), s
+    assert sorted(binding.EXPORTED) == syms
+
+
+def test_status_strings_and_flag_mapping():
+    from paged_kv_cache_350_b200 import binding as b
+    for s in range(11):
+        assert b.lib.pa_status_string(s)
+    assert b.lib.pa_status_from_device_flag(0) == b.PA_OK
+    assert b.lib.pa_status_from_device_flag(b.PA_DEVERR_BAD_BLOCK_ID | 8) == b.PA_ERR_BAD_BLOCK_ID
+    assert b.lib.pa_status_from_device_flag(b.PA_DEVERR_TIMEOUT) == b.PA_ERR_TIMEOUT
+
+
+def test_workspace_size_bounds_every_partition():
+    from paged_kv_cache_350_b200 import binding as b
+    assert b.pa_decode_workspace_size(8, 64, 128, 512, 16, 0) == 0       # no split possible
+    n0 = b.pa_decode_workspace_size(256, 32, 128, 4096, 16, 0)
+    parts = 4096 // 512
+    assert n0 >= 256 * 32 * parts * (128 + 2) * 4
+    assert b.pa_decode_workspace_size(2, 4, 64, 64, 4, 4) >= 2 * 4 * 16 * 66 * 4
+    with pytest.raises(b.PAError):
+        b.pa_decode_workspace_size(2, 4, 64, 64, 4, 6)   # not a multiple of block_size
+
+
+def _call_decode(**kw):
+    from paged_kv_cache_350_b200 import binding as b
+    a = dict(out=16, q=16, k=16, v=16, t=16, l=16, B=2, Hq=8, Hkv=2, D=128, bs=16, MB=4, NB=8,
+             scale=0.1, dtype=b.PA_BF16, ws=0, wsb=0, err=0, stream=0, part=0, path=0)
+    a.update(kw)
+    opts = b.pa_decode_opts(a["part"], a["path"])
+    vp = ctypes.c_void_p
+    return b.lib.pa_decode_ex(vp(a["out"]), vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["t"]),
+                              vp(a["l"]), a["B"], a["Hq"], a["Hkv"], a["D"], a["bs"], a["MB"],
+                              a["NB"], a["scale"], a["dtype"], vp(a["ws"]), a["wsb"], vp(a["err"]),
+                              vp(a["stream"]), ctypes.byref(opts))
+
+
+def test_decode_argument_errors_are_reported_before_any_launch():
+    from paged_kv_cache_350_b200 import binding as b
+    assert _call_decode(B=0) == b.PA_OK                       # empty batch: nothing to do
+    assert _call_decode(Hq=6, Hkv=4) == b.PA_ERR_INVALID_ARG  # Hq % Hkv
+    assert _call_decode(D=96) == b.PA_ERR_UNSUPPORTED
+    assert _call_decode(bs=12) == b.PA_ERR_UNSUPPORTED
+    assert _call_decode(q=8) == b.PA_ERR_INVALID_ARG          # misaligned pointer
+    assert _call_decode(q=0) == b.PA_ERR_INVALID_ARG          # NULL
+    assert _call_decode(scale=float("nan")) == b.PA_ERR_INVALID_ARG
+    assert _call_decode(part=24) == b.PA_ERR_INVALID_ARG      # not a multiple of block_size
+    assert _call_decode(dtype=b.PA_F32, path=b.PA_PATH_TENSOR) == b.PA_ERR_UNSUPPORTED
+    assert _call_decode(bs=4, path=b.PA_PATH_TENSOR) == b.PA_ERR_UNSUPPORTED
+    assert _call_decode(part=32, MB=8, wsb=0) == b.PA_ERR_INVALID_ARG   # explicit split, no workspace
+    assert _call_decode(path=7) == b.PA_ERR_INVALID_ARG
+
+
+def test_cache_op_argument_errors():
+    from paged_kv_cache_350_b200 import binding as b
+    vp = ctypes.c_void_p
+    L = b.lib
+    assert L.pa_reshape_and_cache(vp(16), vp(16), vp(16), vp(16), vp(16), 0, 8, 128, 16, 4,
+                                  b.PA_BF16, vp(0), vp(0)) == b.PA_OK
+    assert L.pa_reshape_and_cache(vp(16), vp(16), vp(16), vp(16), vp(12), 3, 8, 128, 16, 4,
+                                  b.PA_BF16, vp(0), vp(0)) == b.PA_ERR_INVALID_ARG
+    assert L.pa_reshape_and_cache(vp(16), vp(16), vp(16), vp(16), vp(16), 3, 8, 80, 16, 4,
+                                  b.PA_BF16, vp(0), vp(0)) == b.PA_ERR_UNSUPPORTED
+    assert L.pa_copy_blocks(vp(16), vp(16), vp(16), 0, 16, 8, 128, 4, b.PA_BF16, vp(0),
+                            vp(0)) == b.PA_OK
+    assert L.pa_copy_blocks(vp(16), vp(16), vp(0), 2, 16, 8, 128, 4, b.PA_BF16, vp(0),
+                            vp(0)) == b.PA_ERR_INVALID_ARG
+    assert L.pa_copy_blocks(vp(16), vp(16), vp(16), -1, 16, 8, 128, 4, b.PA_BF16, vp(0),
+                            vp(0)) == b.PA_ERR_INVALID_ARG

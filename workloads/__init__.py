@@ -181,6 +181,12 @@ def _independent(name, seed, dtype, B, Hq, Hkv, D, bs, lens_after, max_blocks=No
     )
 
 
+def independent(lens_after, seed=2000, Hq=8, Hkv=2, D=128, bs=16, dtype="bf16", max_blocks=None,
+                name="explicit"):
+    """Independent sequences with the given decode lengths (each >= 1)."""
+    return _independent(name, seed, dtype, len(lens_after), Hq, Hkv, D, bs, lens_after, max_blocks)
+
+
 def mha(seed=1001, B=64, lo=128, hi=2048, Hq=32, D=128, bs=16, dtype="bf16"):
     """Llama-7B-shaped MHA decode: lengths uniform in [lo, hi]."""
     rng = np.random.default_rng(seed)
