@@ -99,7 +99,7 @@ def measured_peak():
 
 def decode_kernel_hash():
     h = hashlib.sha256()
-    for f in ("decode_tc.cu", "pa_device.cuh"):
+    for f in ("decode_stream.cu", "decode_tc.cu", "tc_tile.cuh", "pa_device.cuh"):
         with open(os.path.join(ROOT, "paged_kv_cache_350_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -340,7 +340,7 @@ def run_ours(args):
     lens_d = torch.from_numpy(lens).to(device)
     out = torch.empty_like(q)
     err = torch.zeros(1, dtype=torch.int32, device=device)
-    nws = pa.pa_decode_workspace_size(w.B, w.Hq, w.D, MB * w.block_size, w.block_size, 0)
+    nws = pa.pa_decode_workspace_size(w.B, w.Hq, w.Hkv, w.D, MB * w.block_size, w.block_size, 0)
     ws = torch.empty(max(nws, 1), dtype=torch.uint8, device=device)
     plan = pa.pa_decode_plan(w.B, w.Hq, w.Hkv, w.D, w.block_size, MB, dtype_pa, nws)
     npairs = int(pairs.shape[0])

@@ -109,21 +109,33 @@ typedef enum pa_decode_path {
                            PA_ERR_UNSUPPORTED if not eligible */
 } pa_decode_path;
 
+/* Kernels a decode call can run (reported by pa_decode_plan). */
+typedef enum pa_decode_kernel {
+  PA_KERNEL_NONE = 0,          /* empty batch */
+  PA_KERNEL_GENERIC = 1,       /* CUDA cores, one CTA per (sequence, KV head, heads, partition) */
+  PA_KERNEL_TC_PARTITION = 2,  /* tensor cores, one CTA per (sequence, KV head, partition) */
+  PA_KERNEL_TC_STREAM = 3      /* tensor cores, one persistent wave; every consumer warp owns
+                                  an equal range of the batch's 16-token tiles */
+} pa_decode_kernel;
+
 typedef struct pa_decode_opts {
   /* Tokens per context partition.  0 = automatic.  Otherwise a positive multiple of
-   * block_size (and of 16 on the tensor-core path).  A sequence longer than one
-   * partition is split; each partition writes a partial (max, sum, unnormalised
-   * output) to the workspace and a reduce kernel merges them by log-sum-exp. */
+   * block_size (and of 16 on the tensor-core path), and the partition kernels are used:
+   * a sequence longer than one partition is split; each partition writes a partial
+   * (max, sum, unnormalised output) to the workspace and a reduce kernel merges them by
+   * log-sum-exp. */
   int partition_tokens;
   int path;             /* pa_decode_path */
+  /* Upper bound on the CTAs of the balanced tensor-core kernel (0 = one full wave).
+   * Changes only the schedule, not the result's definition. */
+  int max_ctas;
 } pa_decode_opts;
 
-/* Bytes of workspace pa_decode needs for a batch of B sequences of at most
- * max_seq_len tokens.  partition_tokens as in pa_decode_opts (0 = the automatic
- * choice; its bound holds for every automatic choice).  Returns 0 when no split is
- * possible and (size_t)-1 for invalid arguments. */
-size_t pa_decode_workspace_size(int B, int Hq, int D, int max_seq_len, int block_size,
-                                int partition_tokens);
+/* Bytes of workspace pa_decode needs on the current device for B sequences of at most
+ * max_seq_len tokens, for every kernel the call could choose (partition_tokens as in
+ * pa_decode_opts; 0 = automatic).  Returns (size_t)-1 for invalid arguments. */
+size_t pa_decode_workspace_size(int B, int Hq, int Hkv, int D, int max_seq_len,
+                                int block_size, int partition_tokens);
 
 /* out[b][h][:] = sum_t softmax_t(scale * q[b][h].k_t) v_t over t < seq_lens[b], with
  * k_t = k_pool[block_tables[b][t / block_size]][t % block_size][h / (Hq/Hkv)][:]
@@ -136,14 +148,14 @@ pa_status pa_decode(void* out, const void* q, const void* k_pool, const void* v_
                     float scale, pa_dtype dtype, void* workspace, size_t workspace_bytes,
                     int32_t* dev_err_flag, pa_stream_t stream);
 
-/* What pa_decode_ex would launch for these arguments (host only, queues nothing):
- * the path taken, the partition size, the partitions of the longest possible
- * sequence, and the number of kernel launches (1, or 2 with the reduce). */
+/* What pa_decode_ex would launch for these arguments on the current device (host
+ * only, queues nothing). */
 typedef struct pa_decode_plan_info {
-  int path;              /* PA_PATH_GENERIC or PA_PATH_TENSOR */
-  int partition_tokens;
-  int max_parts;
-  int launches;
+  int kernel;            /* pa_decode_kernel */
+  int partition_tokens;  /* partition kernels: tokens per partition */
+  int max_parts;         /* partition kernels: partitions of the longest possible sequence */
+  int grid;              /* CTAs of the main kernel (stream kernel: one wave) */
+  int launches;          /* kernel launches: 0, 1, or 2 with a reduce */
 } pa_decode_plan_info;
 
 pa_status pa_decode_plan(int B, int Hq, int Hkv, int D, int block_size, int max_blocks,

@@ -52,13 +52,21 @@ class PAError(RuntimeError):
         super().__init__(f"{where}: {msg} (status {status})" if where else msg)
 
 
+# pa_decode_kernel
+PA_KERNEL_NONE = 0
+PA_KERNEL_GENERIC = 1
+PA_KERNEL_TC_PARTITION = 2
+PA_KERNEL_TC_STREAM = 3
+
+
 class pa_decode_opts(ctypes.Structure):
-    _fields_ = [("partition_tokens", ctypes.c_int), ("path", ctypes.c_int)]
+    _fields_ = [("partition_tokens", ctypes.c_int), ("path", ctypes.c_int),
+                ("max_ctas", ctypes.c_int)]
 
 
 class pa_decode_plan_info(ctypes.Structure):
-    _fields_ = [("path", ctypes.c_int), ("partition_tokens", ctypes.c_int),
-                ("max_parts", ctypes.c_int), ("launches", ctypes.c_int)]
+    _fields_ = [("kernel", ctypes.c_int), ("partition_tokens", ctypes.c_int),
+                ("max_parts", ctypes.c_int), ("grid", ctypes.c_int), ("launches", ctypes.c_int)]
 
 
 def _load():
@@ -75,7 +83,7 @@ def _load():
         "pa_status_string": (ctypes.c_char_p, [i32]),
         "pa_status_from_device_flag": (i32, [ctypes.c_int32]),
         "pa_version": (ctypes.c_char_p, []),
-        "pa_decode_workspace_size": (sz, [i32, i32, i32, i32, i32, i32]),
+        "pa_decode_workspace_size": (sz, [i32, i32, i32, i32, i32, i32, i32]),
         "pa_decode": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32, i32,
                             vp, sz, vp, vp]),
         "pa_decode_ex": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32,
@@ -154,26 +162,26 @@ def _need(cond, msg):
 # decode
 # ---------------------------------------------------------------------------
 
-def pa_decode_workspace_size(B, Hq, D, max_seq_len, block_size, partition_tokens=0):
-    n = lib.pa_decode_workspace_size(B, Hq, D, max_seq_len, block_size, partition_tokens)
+def pa_decode_workspace_size(B, Hq, Hkv, D, max_seq_len, block_size, partition_tokens=0):
+    n = lib.pa_decode_workspace_size(B, Hq, Hkv, D, max_seq_len, block_size, partition_tokens)
     if n == ctypes.c_size_t(-1).value:
         raise PAError(PA_ERR_INVALID_ARG, "pa_decode_workspace_size")
     return n
 
 
 def pa_decode_plan(B, Hq, Hkv, D, block_size, max_blocks, dtype, workspace_bytes=0,
-                   partition_tokens=0, path=PA_PATH_AUTO):
-    """dict(path, partition_tokens, max_parts, launches) that pa_decode would use."""
+                   partition_tokens=0, path=PA_PATH_AUTO, max_ctas=0):
+    """dict(kernel, partition_tokens, max_parts, grid, launches) pa_decode would use."""
     info = pa_decode_plan_info()
-    opts = pa_decode_opts(partition_tokens, path)
+    opts = pa_decode_opts(partition_tokens, path, max_ctas)
     _check(lib.pa_decode_plan(B, Hq, Hkv, D, block_size, max_blocks, dtype, workspace_bytes,
                               ctypes.byref(opts), ctypes.byref(info)), "pa_decode_plan")
-    return {"path": info.path, "partition_tokens": info.partition_tokens,
-            "max_parts": info.max_parts, "launches": info.launches}
+    return {"kernel": info.kernel, "partition_tokens": info.partition_tokens,
+            "max_parts": info.max_parts, "grid": info.grid, "launches": info.launches}
 
 
 def pa_decode(out, q, k_pool, v_pool, block_tables, seq_lens, scale, workspace=None,
-              err_flag=None, stream=None, partition_tokens=0, path=PA_PATH_AUTO):
+              err_flag=None, stream=None, partition_tokens=0, path=PA_PATH_AUTO, max_ctas=0):
     """out[B,Hq,D] = paged decode attention of q[B,Hq,D] over the pools (see include/pa.h)."""
     import torch
     _need(q.dim() == 3 and out.shape == q.shape, "q/out must be [B, Hq, D]")
@@ -188,7 +196,7 @@ def pa_decode(out, q, k_pool, v_pool, block_tables, seq_lens, scale, workspace=N
     _need(D2 == D, "head dim mismatch")
     _need(block_tables.shape[0] == B, "block_tables rows != B")
     wbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    opts = pa_decode_opts(partition_tokens, path)
+    opts = pa_decode_opts(partition_tokens, path, max_ctas)
     st = lib.pa_decode_ex(_ptr(out), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables),
                           _ptr(seq_lens), B, Hq, Hkv, D, bs, block_tables.shape[1], NB,
                           float(scale), _dtype_of(q), _ptr(workspace), wbytes, _ptr(err_flag),

@@ -55,7 +55,7 @@ class PagedKVCache:
         return t
 
     def workspace(self, B, Hq, max_blocks):
-        n = _b.pa_decode_workspace_size(B, Hq, self.D, max_blocks * self.block_size,
+        n = _b.pa_decode_workspace_size(B, Hq, self.Hkv, self.D, max_blocks * self.block_size,
                                         self.block_size, 0)
         if n and (self._ws is None or self._ws.numel() < n):
             self._ws = torch.empty(n, dtype=torch.uint8, device=self.device)

@@ -2,6 +2,7 @@
 // Every check happens on the host before anything is queued; a failing call queues
 // nothing.  See include/pa.h for the contract of each entry point.
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 
@@ -14,6 +15,10 @@ namespace {
 // with partition_tokens == 0 sizes the workspace for it, which bounds every automatic
 // choice.
 constexpr int kAutoMinPartition = 512;
+// Largest batch the balanced stream kernel takes (its prefix sums live in shared memory).
+constexpr int kStreamMaxB = 8192;
+// Stream-kernel CTAs assumed when no device can be asked.
+constexpr int kStreamGridBound = 1024;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -71,13 +76,23 @@ pa_status pa_status_from_device_flag(int32_t flag) {
 
 const char* pa_version(void) { return "0.1.0"; }
 
-size_t pa_decode_workspace_size(int B, int Hq, int D, int max_seq_len, int block_size,
-                                int partition_tokens) {
-  if (B < 0 || Hq <= 0 || D <= 0 || max_seq_len < 0 || !block_size_ok(block_size) ||
-      partition_tokens < 0 || (partition_tokens > 0 && partition_tokens % block_size != 0))
+size_t pa_decode_workspace_size(int B, int Hq, int Hkv, int D, int max_seq_len,
+                                int block_size, int partition_tokens) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || D <= 0 || max_seq_len < 0 ||
+      !block_size_ok(block_size) || partition_tokens < 0 ||
+      (partition_tokens > 0 && partition_tokens % block_size != 0))
     return static_cast<size_t>(-1);
   const int64_t P = partition_tokens > 0 ? partition_tokens : kAutoMinPartition;
-  return workspace_bytes_for(B, Hq, D, ceil_div(max_seq_len, P));
+  size_t need = workspace_bytes_for(B, Hq, D, ceil_div(max_seq_len, P));
+  const int G = Hq / Hkv;
+  if (partition_tokens == 0 && B > 0 && B <= kStreamMaxB &&
+      pa::tc_eligible(G, D, block_size, PA_BF16)) {
+    int grid = pa::stream_grid(D, block_size, G, B);
+    if (grid <= 0) grid = kStreamGridBound;  // no device to ask: an upper bound
+    const size_t s = pa::stream_workspace_bytes(grid * 4, G, D);
+    if (s > need) need = s;
+  }
+  return need;
 }
 
 // Shape/dtype checks and the launch plan shared by pa_decode_plan and pa_decode_ex.
@@ -87,8 +102,9 @@ static pa_status plan_decode(int B, int Hq, int Hkv, int D, int block_size, int 
                              pa_decode_plan_info* info) {
   const int partition = opts ? opts->partition_tokens : 0;
   const int path = opts ? opts->path : PA_PATH_AUTO;
+  const int max_ctas = opts ? opts->max_ctas : 0;
   if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || max_blocks <= 0 || num_blocks <= 0 ||
-      block_size <= 0 || !std::isfinite(scale) || partition < 0 ||
+      block_size <= 0 || !std::isfinite(scale) || partition < 0 || max_ctas < 0 ||
       (path != PA_PATH_AUTO && path != PA_PATH_GENERIC && path != PA_PATH_TENSOR) ||
       (dtype != PA_F32 && dtype != PA_BF16))
     return PA_ERR_INVALID_ARG;
@@ -99,16 +115,33 @@ static pa_status plan_decode(int B, int Hq, int Hkv, int D, int block_size, int 
   if (max_seq > 0x7fffffffLL) return PA_ERR_INVALID_ARG;
 
   const int G = Hq / Hkv;
-  bool use_tc = false;
-  if (path != PA_PATH_GENERIC && pa::tc_eligible(G, D, block_size, dtype)) {
-    const int tile = block_size > 16 ? block_size : 16;
-    if (partition == 0 || partition % tile == 0) use_tc = true;
-  }
-  if (path == PA_PATH_TENSOR && !use_tc) {
-    if (!pa::tc_eligible(G, D, block_size, dtype)) return PA_ERR_UNSUPPORTED;
+  const bool tc_ok = path != PA_PATH_GENERIC && pa::tc_eligible(G, D, block_size, dtype);
+  const int tc_tile = block_size > 16 ? block_size : 16;
+  if (path == PA_PATH_TENSOR && !tc_ok) return PA_ERR_UNSUPPORTED;
+  if (path == PA_PATH_TENSOR && partition > 0 && partition % tc_tile != 0)
     return PA_ERR_INVALID_ARG;  // partition not a multiple of the 16-token tile
+  info->kernel = PA_KERNEL_NONE;
+  info->partition_tokens = 0;
+  info->max_parts = 0;
+  info->grid = 0;
+  info->launches = 0;
+  if (B == 0) return PA_OK;
+
+  // Balanced persistent tensor-core kernel: the default for bf16 batches.
+  if (tc_ok && partition == 0 && B <= kStreamMaxB) {
+    int grid = pa::stream_grid(D, block_size, G, B);
+    if (max_ctas > 0 && grid > max_ctas) grid = max_ctas;
+    if (grid > 0 && have_ws && workspace_bytes >= pa::stream_workspace_bytes(grid * 4, G, D)) {
+      info->kernel = PA_KERNEL_TC_STREAM;
+      info->grid = grid;
+      info->max_parts = 1;
+      info->launches = 2;
+      return PA_OK;
+    }
   }
-  const int tile = use_tc ? (block_size > 16 ? block_size : 16) : block_size;
+
+  const bool use_tc = tc_ok && (partition == 0 || partition % tc_tile == 0);
+  const int tile = use_tc ? tc_tile : block_size;
   int P = partition > 0 ? partition : auto_partition(max_seq, tile);
   int64_t parts = ceil_div(max_seq, P);
   if (parts > 1) {
@@ -119,10 +152,12 @@ static pa_status plan_decode(int B, int Hq, int Hkv, int D, int block_size, int 
       parts = 1;
     }
   }
-  info->path = use_tc ? PA_PATH_TENSOR : PA_PATH_GENERIC;
+  info->kernel = use_tc ? PA_KERNEL_TC_PARTITION : PA_KERNEL_GENERIC;
   info->partition_tokens = P;
   info->max_parts = static_cast<int>(parts);
-  info->launches = B == 0 ? 0 : (parts > 1 ? 2 : 1);
+  const int64_t units = static_cast<int64_t>(B) * Hkv * (use_tc ? 1 : (G + 3) / 4);
+  info->grid = static_cast<int>(std::min<int64_t>(units * parts, 0x7fffffff));
+  info->launches = parts > 1 ? 2 : 1;
   return PA_OK;
 }
 
@@ -151,7 +186,6 @@ pa_status pa_decode_ex(void* out, const void* q, const void* k_pool, const void*
       (dev_err_flag && !aligned(dev_err_flag, 4)))
     return PA_ERR_INVALID_ARG;
 
-  const int parts = plan.max_parts;
   pa::DecodeParams p{};
   p.out = out;
   p.q = q;
@@ -169,18 +203,27 @@ pa_status pa_decode_ex(void* out, const void* q, const void* k_pool, const void*
   p.num_blocks = num_blocks;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.partition_tokens = plan.partition_tokens;
-  p.max_parts = parts;
-  if (parts > 1) {
-    char* ws = static_cast<char*>(workspace);
-    p.ws_ml = reinterpret_cast<float*>(ws);
-    p.ws_acc = reinterpret_cast<float*>(
-        ws + round_up(static_cast<int64_t>(B) * Hq * parts * 2 * 4, 256));
-  }
+  p.max_parts = plan.max_parts;
   p.err = dev_err_flag;
-
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = plan.path == PA_PATH_TENSOR ? pa::launch_decode_tc(p, s)
-                                              : pa::launch_decode_generic(p, dtype, s);
+  cudaError_t e;
+  if (plan.kernel == PA_KERNEL_TC_STREAM) {
+    pa::StreamParams sp{};
+    sp.d = p;
+    sp.streams = plan.grid * 4;
+    pa::stream_carve(&sp, workspace);
+    e = pa::launch_decode_stream(sp, plan.grid, s);
+  } else {
+    const int parts = plan.max_parts;
+    if (parts > 1) {
+      char* ws = static_cast<char*>(workspace);
+      p.ws_ml = reinterpret_cast<float*>(ws);
+      p.ws_acc = reinterpret_cast<float*>(
+          ws + round_up(static_cast<int64_t>(B) * Hq * parts * 2 * 4, 256));
+    }
+    e = plan.kernel == PA_KERNEL_TC_PARTITION ? pa::launch_decode_tc(p, s)
+                                               : pa::launch_decode_generic(p, dtype, s);
+  }
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

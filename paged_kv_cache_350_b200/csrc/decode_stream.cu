@@ -1,0 +1,449 @@
+// Paged decode attention, bf16 tensor-core path with a balanced persistent schedule
+// (sm_100a).  Same result as decode_tc.cu — softmax(scale * q.K^T) V per (sequence,
+// query head), K/V read through the block table ("PagedAttention" concept card,
+// 实现要点) — scheduled for a whole batch of ragged lengths.
+//
+// Schedule ("streams"):
+//   * Every (sequence b, KV head) is a unit of nt(b) = ceil(L_b / TILE_T) tiles; units
+//     are laid end to end in (b, KV head) order, T = Hkv * sum_b nt(b) tiles in all.
+//   * The grid is one wave of persistent CTAs (SM count x occupancy).  Each CTA has 4
+//     consumer warps and every consumer warp is one stream: stream s owns the global
+//     tiles [s*per, (s+1)*per), per = ceil(T / streams).  Work is balanced to one tile.
+//   * Each CTA first computes the prefix sums of nt(b) in shared memory; a global tile
+//     index maps to (b, KV head, tile) by binary search.
+//   * Warp 4 produces for all four streams: it resolves the block ids of the next 32
+//     tiles with one coalesced table read per lane, and issues 4-D TMA loads into
+//     per-stream rings of SPW stages (mbarrier expect-tx), across unit boundaries, so
+//     the HBM stream never drains between units.
+//   * A consumer warp runs the tile math of tc_tile.cuh over its range.  A unit that
+//     lies wholly inside the range is finished in place: normalised bf16 output.  A unit
+//     cut by a range boundary leaves a partial (max, sum, unnormalised O) in one of the
+//     stream's two slots; the reduce kernel merges the pieces of each cut unit by
+//     log-sum-exp.  Each stream records which units its slots hold every launch.
+
+#include <cudaTypedefs.h>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+#include "tc_tile.cuh"
+
+namespace pa {
+
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kNCW = 4;                      // consumer warps (= streams) per CTA
+constexpr int kThreads = (kNCW + 1) * 32;
+
+template <int D_, int BS_, bool ROWS16_, int SPW_>
+struct StreamCfg : TileCfg<D_, BS_, ROWS16_> {
+  static constexpr int SPW = SPW_;                 // ring stages per stream
+  static constexpr int NST = kNCW * SPW;
+  static constexpr int RING_BYTES = NST * StreamCfg::STAGE_BYTES;
+};
+
+template <class C>
+size_t stream_smem_bytes(int B) {
+  return C::RING_BYTES + 1024 + static_cast<size_t>(B + 1) * 4;
+}
+
+__device__ __forceinline__ int clamp_len(const DecodeParams& p, int b, bool flag) {
+  int L = __ldg(p.seq_lens + b);
+  const int Lmax = p.max_blocks * p.block_size;
+  if (L < 0 || L > Lmax) {
+    if (flag) flag_error(p.err, PA_DEVERR_BAD_SEQ_LEN);
+    L = L < 0 ? 0 : Lmax;
+  }
+  return L;
+}
+
+// First index in P[0..n) with P[idx] > v.
+__device__ __forceinline__ int upper_bound(const int* P, int n, int v) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (P[mid] > v) hi = mid; else lo = mid + 1;
+  }
+  return lo;
+}
+
+struct TilePos {
+  int b, kvh, j, nt;
+};
+
+// Global tile index -> (sequence, KV head, tile within the unit).
+__device__ __forceinline__ TilePos locate(const int* P, int B, int Hkv, long long g) {
+  TilePos t;
+  const int v = static_cast<int>(g / Hkv);
+  t.b = upper_bound(P, B + 1, v) - 1;
+  t.nt = P[t.b + 1] - P[t.b];
+  const int off = static_cast<int>(g - static_cast<long long>(Hkv) * P[t.b]);
+  t.kvh = off / t.nt;
+  t.j = off - t.kvh * t.nt;
+  return t;
+}
+
+template <class C>
+__global__ void __launch_bounds__(kThreads)
+    decode_stream_kernel(const __grid_constant__ CUtensorMap tmk,
+                         const __grid_constant__ CUtensorMap tmv, const StreamParams sp) {
+  constexpr int D = C::D, BS = C::BS, TILE_T = C::TILE_T, SPW = C::SPW, NST = C::NST;
+  const DecodeParams& p = sp.d;
+  const int B = p.B, Hkv = p.Hkv, G = p.G;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  int* P = reinterpret_cast<int*>(smem + C::RING_BYTES);  // [B + 1] tiles before sequence b
+  __shared__ __align__(8) uint64_t full_bar[NST];
+  __shared__ __align__(8) uint64_t empty_bar[NST];
+  __shared__ int warp_sum[kThreads / 32];
+
+  // ---- prefix sums of per-sequence tile counts (every CTA, identical) --------------
+  {
+    const int chunk = (B + kThreads - 1) / kThreads;
+    const int lo = min(B, static_cast<int>(threadIdx.x) * chunk);
+    const int hi = min(B, lo + chunk);
+    int sum = 0;
+    for (int b = lo; b < hi; ++b) sum += (clamp_len(p, b, blockIdx.x == 0) + TILE_T - 1) / TILE_T;
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(kFull, incl, off);
+      if (lane >= off) incl += v;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < warp; ++w) base += warp_sum[w];
+    int run = base + incl - sum;
+    for (int b = lo; b < hi; ++b) {
+      P[b] = run;
+      run += (clamp_len(p, b, false) + TILE_T - 1) / TILE_T;
+    }
+    if (threadIdx.x == 0) {
+      int total = 0;
+      for (int w = 0; w < kThreads / 32; ++w) total += warp_sum[w];
+      P[B] = total;
+    }
+  }
+  // Empty sequences have no tiles: their output rows are zero (written by one CTA each).
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+  for (int b = blockIdx.x; b < B; b += gridDim.x) {
+    if (clamp_len(p, b, false) == 0) {
+      uint32_t* row = reinterpret_cast<uint32_t*>(out + static_cast<size_t>(b) * p.Hq * D);
+      for (int i = threadIdx.x; i < p.Hq * D / 2; i += kThreads) row[i] = 0u;
+    }
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(smem_addr(&full_bar[s]), 1);
+      mbar_init(smem_addr(&empty_bar[s]), 1);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    fence_proxy_async_smem();
+  }
+  __syncthreads();
+
+  const long long T = static_cast<long long>(Hkv) * P[B];
+  const long long S = static_cast<long long>(gridDim.x) * kNCW;
+  const long long per = (T + S - 1) / S;
+
+  if (warp == kNCW) {
+    // ---------------- producer warp: feeds the 4 streams of this CTA ----------------
+    if (lane == 0) {
+      prefetch_tensormap(&tmk);
+      prefetch_tensormap(&tmv);
+    }
+    const uint64_t policy = l2_policy_evict_first();
+    const int my_w = lane & 3;
+    const long long my_s = static_cast<long long>(blockIdx.x) * kNCW + my_w;
+    const long long my_beg = min(T, my_s * per);
+    const int my_cnt = static_cast<int>(min(T, my_beg + per) - my_beg);
+    int rounds = my_cnt;
+    rounds = max(rounds, __shfl_xor_sync(kFull, rounds, 1));
+    rounds = max(rounds, __shfl_xor_sync(kFull, rounds, 2));
+    bool ok = true;
+    for (int r0 = 0; r0 < rounds && ok; r0 += 8) {
+      // lane l resolves round r0 + l/4 of stream l%4
+      const int rr = r0 + (lane >> 2);
+      const bool v = rr < my_cnt;
+      int kvh = 0, id0 = 0, id1 = 0, nb = 0;
+      if (v) {
+        const TilePos t = locate(P, B, Hkv, my_beg + rr);
+        kvh = t.kvh;
+        const int L = clamp_len(p, t.b, false);
+        const int nblk = (L + BS - 1) / BS;
+        const int blk = t.j * C::BPS;
+        nb = min(C::BPS, nblk - blk);
+        const int32_t* tab = p.block_tables + static_cast<size_t>(t.b) * p.max_blocks + blk;
+        id0 = __ldg(tab);
+        if (id0 < 0 || id0 >= p.num_blocks) {
+          flag_error(p.err, PA_DEVERR_BAD_BLOCK_ID);
+          id0 = 0;
+        }
+        if (C::BPS > 1 && nb > 1) {
+          id1 = __ldg(tab + 1);
+          if (id1 < 0 || id1 >= p.num_blocks) {
+            flag_error(p.err, PA_DEVERR_BAD_BLOCK_ID);
+            id1 = 0;
+          }
+        }
+      }
+      const unsigned vmask = __ballot_sync(kFull, v);
+      for (int l = 0; l < 32; ++l) {
+        const int kv = __shfl_sync(kFull, kvh, l);
+        const int i0 = __shfl_sync(kFull, id0, l);
+        const int i1 = __shfl_sync(kFull, id1, l);
+        const int n = __shfl_sync(kFull, nb, l);
+        if (lane == 0 && ok && ((vmask >> l) & 1u)) {
+          const int w = l & 3;
+          const int r = r0 + (l >> 2);
+          const int stage = w * SPW + r % SPW;
+          if (r >= SPW) ok = mbar_wait(smem_addr(&empty_bar[stage]), ((r / SPW) - 1) & 1, p.err);
+          if (ok) {
+            const uint32_t fb = smem_addr(&full_bar[stage]);
+            mbar_arrive_expect_tx(fb, static_cast<uint32_t>(n * BS * D * 2 * 2));
+            const uint32_t kt = smem_addr(smem + stage * C::STAGE_BYTES);
+            const uint32_t vt = kt + C::TILE_BYTES;
+            for (int sub = 0; sub < n; ++sub) {
+              const int phys = sub == 0 ? i0 : i1;
+#pragma unroll
+              for (int c = 0; c < C::DCH; ++c) {
+                tma_load_4d(kt + c * C::CHUNK_BYTES + sub * BS * 128, &tmk, c * 64, kv, 0, phys,
+                            fb, policy);
+                tma_load_4d(vt + c * C::CHUNK_BYTES + sub * BS * 128, &tmv, c * 64, kv, 0, phys,
+                            fb, policy);
+              }
+            }
+          }
+        }
+      }
+      ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
+    }
+    return;
+  }
+
+  // ---------------- consumer warp = one stream ----------------
+  const long long s = static_cast<long long>(blockIdx.x) * kNCW + warp;
+  const long long beg = min(T, s * per);
+  const long long end = min(T, beg + per);
+  const int g = lane >> 2, tig = lane & 3;
+  const float sl2 = p.scale_log2;
+  int unit_a = -1, a_starts = 0, unit_b = -1;
+  int i = 0;  // tiles consumed by this stream (ring position)
+  bool ok = true;
+  WarpAcc<C> acc;
+
+  long long gpos = beg;
+  while (gpos < end && ok) {
+    const TilePos t = locate(P, B, Hkv, gpos);
+    const int L = clamp_len(p, t.b, false);
+    const long long ubeg = static_cast<long long>(Hkv) * P[t.b] + static_cast<long long>(t.kvh) * t.nt;
+    const long long uend = ubeg + t.nt;
+    const long long pend = min(end, uend);
+    const size_t head0 = static_cast<size_t>(t.b) * p.Hq + static_cast<size_t>(t.kvh) * G;
+    acc.load_q(static_cast<const __nv_bfloat16*>(p.q) + head0 * D, G, lane);
+    acc.reset();
+    const int jend = t.j + static_cast<int>(pend - gpos);
+    for (int j = t.j; j < jend; ++j, ++i) {
+      const int stage = warp * SPW + i % SPW;
+      if (!mbar_wait(smem_addr(&full_bar[stage]), (i / SPW) & 1, p.err)) {
+        ok = false;
+        break;
+      }
+      uint8_t* st_ptr = smem + stage * C::STAGE_BYTES;
+      const int valid = min(TILE_T, L - j * TILE_T);
+      if (valid < TILE_T) zero_tail_rows<C>(st_ptr, valid, lane);
+      acc.tile(smem_addr(st_ptr), valid, sl2, lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(&empty_bar[stage]));
+    }
+    if (!ok) break;
+    acc.reduce_l();
+    const bool complete = (gpos == ubeg) && (pend == uend);
+    if (complete) {
+      const float inv_lo = 1.f / acc.l_lo;
+      const float inv_hi = C::ROWS16 ? 1.f / acc.l_hi : 0.f;
+#pragma unroll
+      for (int jn = 0; jn < C::NT; ++jn) {
+        if (g < G)
+          *reinterpret_cast<uint32_t*>(out + (head0 + g) * D + 8 * jn + 2 * tig) =
+              pack_bf16x2(acc.o_lo[jn][0] * inv_lo, acc.o_lo[jn][1] * inv_lo);
+        if (C::ROWS16 && g + 8 < G)
+          *reinterpret_cast<uint32_t*>(out + (head0 + g + 8) * D + 8 * jn + 2 * tig) =
+              pack_bf16x2(acc.o_hi[jn][0] * inv_hi, acc.o_hi[jn][1] * inv_hi);
+      }
+    } else {
+      const int slot = gpos == beg ? 0 : 1;  // a cut piece is the stream's first or last
+      const size_t row0 = (static_cast<size_t>(s) * 2 + slot) * G;
+      if (tig == 0) {
+        if (g < G)
+          *reinterpret_cast<float2*>(sp.pml + (row0 + g) * 2) = make_float2(acc.m_lo, acc.l_lo);
+        if (C::ROWS16 && g + 8 < G)
+          *reinterpret_cast<float2*>(sp.pml + (row0 + g + 8) * 2) = make_float2(acc.m_hi, acc.l_hi);
+      }
+#pragma unroll
+      for (int jn = 0; jn < C::NT; ++jn) {
+        if (g < G)
+          *reinterpret_cast<float2*>(sp.pacc + (row0 + g) * D + 8 * jn + 2 * tig) =
+              make_float2(acc.o_lo[jn][0], acc.o_lo[jn][1]);
+        if (C::ROWS16 && g + 8 < G)
+          *reinterpret_cast<float2*>(sp.pacc + (row0 + g + 8) * D + 8 * jn + 2 * tig) =
+              make_float2(acc.o_hi[jn][0], acc.o_hi[jn][1]);
+      }
+      const int u = t.b * Hkv + t.kvh;
+      if (slot == 0) {
+        unit_a = u;
+        a_starts = gpos == ubeg ? 1 : 0;
+      } else {
+        unit_b = u;
+      }
+    }
+    gpos = pend;
+  }
+  if (lane == 0) {
+    int4 m = make_int4(ok ? unit_a : -1, ok ? a_starts : 0, ok ? unit_b : -1, 0);
+    *reinterpret_cast<int4*>(sp.meta + s * 4) = m;
+  }
+}
+
+// Merge the pieces of every unit cut by a stream boundary.  Block s owns the unit that
+// STARTS in stream s and continues into later streams: its piece is slot 1 of s (or
+// slot 0 when it spans the whole stream from its first tile); the other pieces are
+// slot 0 of the following streams, as long as their first piece is the same unit.
+template <int D>
+__global__ void __launch_bounds__(128) stream_reduce_kernel(const StreamParams sp) {
+  const DecodeParams& p = sp.d;
+  const int s = blockIdx.x;
+  const int4 m = *reinterpret_cast<const int4*>(sp.meta + static_cast<size_t>(s) * 4);
+  int u, slot;
+  if (m.z >= 0) {
+    u = m.z;
+    slot = 1;
+  } else if (m.x >= 0 && m.y) {
+    u = m.x;
+    slot = 0;
+  } else {
+    return;
+  }
+  const int G = p.G;
+  int last = s;  // last stream holding a piece of u
+  while (last + 1 < sp.streams && sp.meta[static_cast<size_t>(last + 1) * 4] == u) ++last;
+  const int b = u / p.Hkv, kvh = u - (u / p.Hkv) * p.Hkv;
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+  const size_t head0 = static_cast<size_t>(b) * p.Hq + static_cast<size_t>(kvh) * G;
+  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+    const int r = idx / D, d = idx - r * D;
+    float M = -INFINITY;
+    for (int q = s; q <= last; ++q) {
+      const size_t row = (static_cast<size_t>(q) * 2 + (q == s ? slot : 0)) * G + r;
+      M = fmaxf(M, sp.pml[row * 2]);
+    }
+    float lsum = 0.f, a = 0.f;
+    for (int q = s; q <= last; ++q) {
+      const size_t row = (static_cast<size_t>(q) * 2 + (q == s ? slot : 0)) * G + r;
+      const float w = exp2f(sp.pml[row * 2] - M);
+      lsum += w * sp.pml[row * 2 + 1];
+      a += w * sp.pacc[row * D + d];
+    }
+    out[(head0 + r) * D + d] = __float2bfloat16_rn(a / lsum);
+  }
+}
+
+template <class C>
+int stream_grid_for(int B, int device_sms) {
+  int occ = 0;
+  const size_t smem = stream_smem_bytes<C>(B);
+  if (cudaFuncSetAttribute(decode_stream_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_stream_kernel<C>, kThreads,
+                                                    smem) != cudaSuccess)
+    return 0;
+  return occ * device_sms;
+}
+
+template <class C>
+cudaError_t launch_stream_cfg(const StreamParams& sp, int grid, cudaStream_t stream) {
+  CUtensorMap tmk, tmv;
+  const DecodeParams& p = sp.d;
+  if (!make_pool_map(&tmk, p.k_pool, p.num_blocks, C::BS, p.Hkv, C::D) ||
+      !make_pool_map(&tmv, p.v_pool, p.num_blocks, C::BS, p.Hkv, C::D))
+    return cudaErrorInvalidValue;
+  const size_t smem = stream_smem_bytes<C>(p.B);
+  cudaError_t e = cudaFuncSetAttribute(decode_stream_kernel<C>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  decode_stream_kernel<C><<<grid, kThreads, smem, stream>>>(tmk, tmv, sp);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  stream_reduce_kernel<C::D><<<sp.streams, 128, 0, stream>>>(sp);
+  return cudaGetLastError();
+}
+
+constexpr int kSPW = 2;
+
+template <int D, int BS>
+int grid_d_bs(bool rows16, int B, int sms) {
+  return rows16 ? stream_grid_for<StreamCfg<D, BS, true, kSPW>>(B, sms)
+                : stream_grid_for<StreamCfg<D, BS, false, kSPW>>(B, sms);
+}
+
+template <int D, int BS>
+cudaError_t launch_d_bs(const StreamParams& sp, int grid, cudaStream_t stream) {
+  if (sp.d.G > 8) return launch_stream_cfg<StreamCfg<D, BS, true, kSPW>>(sp, grid, stream);
+  return launch_stream_cfg<StreamCfg<D, BS, false, kSPW>>(sp, grid, stream);
+}
+
+}  // namespace
+
+int stream_grid(int D, int block_size, int G, int B) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  const bool r16 = G > 8;
+  switch (D * 100 + block_size) {
+    case 6408: return grid_d_bs<64, 8>(r16, B, sms);
+    case 6416: return grid_d_bs<64, 16>(r16, B, sms);
+    case 6432: return grid_d_bs<64, 32>(r16, B, sms);
+    case 12808: return grid_d_bs<128, 8>(r16, B, sms);
+    case 12816: return grid_d_bs<128, 16>(r16, B, sms);
+    case 12832: return grid_d_bs<128, 32>(r16, B, sms);
+    default: return 0;
+  }
+}
+
+size_t stream_workspace_bytes(int streams, int G, int D) {
+  const size_t meta = static_cast<size_t>(streams) * 4 * 4;
+  const size_t pml = static_cast<size_t>(streams) * 2 * G * 2 * 4;
+  const size_t pacc = static_cast<size_t>(streams) * 2 * G * D * 4;
+  return ((meta + 255) / 256) * 256 + ((pml + 255) / 256) * 256 + pacc;
+}
+
+void stream_carve(StreamParams* sp, void* workspace) {
+  char* ws = static_cast<char*>(workspace);
+  const size_t meta = static_cast<size_t>(sp->streams) * 4 * 4;
+  const size_t pml = static_cast<size_t>(sp->streams) * 2 * sp->d.G * 2 * 4;
+  sp->meta = reinterpret_cast<int32_t*>(ws);
+  sp->pml = reinterpret_cast<float*>(ws + ((meta + 255) / 256) * 256);
+  sp->pacc = reinterpret_cast<float*>(ws + ((meta + 255) / 256) * 256 + ((pml + 255) / 256) * 256);
+}
+
+cudaError_t launch_decode_stream(const StreamParams& sp, int grid, cudaStream_t stream) {
+  switch (sp.d.D * 100 + sp.d.block_size) {
+    case 6408: return launch_d_bs<64, 8>(sp, grid, stream);
+    case 6416: return launch_d_bs<64, 16>(sp, grid, stream);
+    case 6432: return launch_d_bs<64, 32>(sp, grid, stream);
+    case 12808: return launch_d_bs<128, 8>(sp, grid, stream);
+    case 12816: return launch_d_bs<128, 16>(sp, grid, stream);
+    case 12832: return launch_d_bs<128, 32>(sp, grid, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace pa

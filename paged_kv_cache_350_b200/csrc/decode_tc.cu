@@ -17,8 +17,9 @@
 //   * Warps 0-3 are consumers; warp w takes stages w, w+4, ...  Per 16-token sub-tile:
 //     S = Q(16 x D, heads padded to 16 rows) . K^T with m16n8k16 bf16 MMAs (K fragments
 //     by ldmatrix from the swizzled tile), an fp32 online softmax in base 2 (the scale
-//     folded with log2 e), P rounded to bf16 in registers and fed straight back as the A
-//     operand of O += P.V (V fragments by ldmatrix.trans).
+//     folded with log2 e), and P fed straight back from registers as the A operand of
+//     O += P.V (V fragments by ldmatrix.trans).  P goes in as two bf16 MMAs, hi and lo
+//     parts, so the only rounding that reaches the output is the final one to bf16.
 //   * Tokens past the sequence end in the last block are masked out of the softmax and
 //     their V rows zeroed in shared memory, so stale or poisoned slots never reach the
 //     output.  Block ids outside [0, num_blocks) raise PA_DEVERR_BAD_BLOCK_ID and read
@@ -33,6 +34,7 @@
 
 #include "pa_device.cuh"
 #include "pa_internal.h"
+#include "tc_tile.cuh"
 
 namespace pa {
 
@@ -41,39 +43,15 @@ namespace {
 constexpr unsigned kFull = 0xffffffffu;
 
 template <int D_, int BS_, bool ROWS16_, int NSTAGE_>
-struct TcCfg {
-  static constexpr int D = D_;
-  static constexpr int BS = BS_;
-  static constexpr bool ROWS16 = ROWS16_;
+struct TcCfg : TileCfg<D_, BS_, ROWS16_> {
   static constexpr int NSTAGE = NSTAGE_;
-  static constexpr int TILE_T = BS > 16 ? BS : 16;   // tokens per pipeline stage
-  static constexpr int BPS = TILE_T / BS;            // blocks per stage
-  static constexpr int SUBT = TILE_T / 16;           // 16-token sub-tiles per stage
-  static constexpr int DCH = D / 64;                 // 128-byte column chunks per row
-  static constexpr int CHUNK_BYTES = TILE_T * 128;
-  static constexpr int TILE_BYTES = DCH * CHUNK_BYTES;  // one K (or V) tile
-  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-  static constexpr int NCW = 4;                         // consumer warps
+  static constexpr int NCW = 4;  // consumer warps
   static constexpr int THREADS = (NCW + 1) * 32;
-  static constexpr int ROWS = ROWS16 ? 16 : 8;          // query-head rows kept
-  static constexpr int KSTEPS = D / 16;
-  static constexpr int NT = D / 8;                      // output n-tiles of 8 columns
-  static constexpr int MERGE_BYTES = NCW * ROWS * D * 4;
-  static constexpr int RING_BYTES = NSTAGE * STAGE_BYTES;
+  static constexpr int MERGE_BYTES = NCW * TcCfg::ROWS * TcCfg::D * 4;
+  static constexpr int RING_BYTES = NSTAGE * TcCfg::STAGE_BYTES;
   static constexpr int BUF_BYTES = RING_BYTES > MERGE_BYTES ? RING_BYTES : MERGE_BYTES;
-  static constexpr int SMEM_BYTES = BUF_BYTES + 1024;   // + alignment slack
-  static_assert(D == 64 || D == 128, "head dim");
-  static_assert(BS == 8 || BS == 16 || BS == 32, "block size");
+  static constexpr int SMEM_BYTES = BUF_BYTES + 1024;  // + alignment slack
 };
-
-// Byte offset of 16-byte column chunk `c16` of row `row` in a 128B-swizzled tile.
-__device__ __forceinline__ uint32_t sw128(int row, int c16) {
-  return static_cast<uint32_t>(row * 128 + ((c16 ^ (row & 7)) << 4));
-}
-
-__device__ __forceinline__ uint32_t ld_u32(const void* p) {
-  return __ldg(reinterpret_cast<const unsigned int*>(p));
-}
 
 template <class C>
 __global__ void __launch_bounds__(C::THREADS)
@@ -187,183 +165,43 @@ __global__ void __launch_bounds__(C::THREADS)
   }
 
   // ---------------- consumer warps ----------------
-  const int g = lane >> 2;   // fragment row (query head within the group)
-  const int tig = lane & 3;  // thread in group
-  const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + head0 * D;
-
-  // Q as the A operand, one fragment per 16-column k-step.  Rows >= G are zero.
-  uint32_t qa[C::KSTEPS][2];
-  uint32_t qh[C::KSTEPS][2];
-#pragma unroll
-  for (int k = 0; k < C::KSTEPS; ++k) {
-    const bool lo_ok = g < G;
-    qa[k][0] = lo_ok ? ld_u32(qrow + g * D + 16 * k + 2 * tig) : 0u;
-    qa[k][1] = lo_ok ? ld_u32(qrow + g * D + 16 * k + 8 + 2 * tig) : 0u;
-    if constexpr (C::ROWS16) {
-      const bool hi_ok = g + 8 < G;
-      qh[k][0] = hi_ok ? ld_u32(qrow + (g + 8) * D + 16 * k + 2 * tig) : 0u;
-      qh[k][1] = hi_ok ? ld_u32(qrow + (g + 8) * D + 16 * k + 8 + 2 * tig) : 0u;
-    } else {
-      qh[k][0] = 0u;
-      qh[k][1] = 0u;
-    }
-  }
-
+  const int g = lane >> 2;
+  const int tig = lane & 3;
+  WarpAcc<C> acc;
+  acc.load_q(static_cast<const __nv_bfloat16*>(p.q) + head0 * D, G, lane);
+  acc.reset();
   const float sl2 = p.scale_log2;
-  float o_lo[C::NT][2];
-  float o_hi[C::NT][2];
-#pragma unroll
-  for (int j = 0; j < C::NT; ++j) {
-    o_lo[j][0] = o_lo[j][1] = 0.f;
-    o_hi[j][0] = o_hi[j][1] = 0.f;
-  }
-  float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
-
-  // Per-lane ldmatrix row/column roles.
-  const int mi = lane >> 3;  // which 8x8 matrix this lane addresses
-  const int mr = lane & 7;   // row within it
 
   for (int tile = warp; tile < ntiles; tile += NCW) {
     const int stage = tile % NSTAGE;
     if (!mbar_wait(smem_addr(&full_bar[stage]), (tile / NSTAGE) & 1, p.err)) break;
-    uint8_t* kt_ptr = smem + stage * C::STAGE_BYTES;
-    const uint32_t kbase = smem_addr(kt_ptr);
-    const uint32_t vbase = kbase + C::TILE_BYTES;
+    uint8_t* st_ptr = smem + stage * C::STAGE_BYTES;
     const int valid = min(TILE_T, tok1 - (tok0 + tile * TILE_T));
-
-    if (valid < TILE_T) {
-      // Zero the V rows past the sequence end: their slots may hold anything.
-      uint8_t* vt_ptr = kt_ptr + C::TILE_BYTES;
-      const int nchunks = (TILE_T - valid) * C::DCH * 8;
-      for (int i = lane; i < nchunks; i += 32) {
-        const int r = valid + i / (C::DCH * 8);
-        const int rem = i % (C::DCH * 8);
-        *reinterpret_cast<uint4*>(vt_ptr + (rem >> 3) * C::CHUNK_BYTES + r * 128 +
-                                  (rem & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-    }
-
-#pragma unroll
-    for (int st = 0; st < C::SUBT; ++st) {
-      const int r0 = st * 16;
-      if (r0 >= valid) break;
-
-      // ---- S = Q . K^T for 16 tokens: n-tile 0 = tokens r0..r0+7, n-tile 1 = +8..+15
-      float s0[4] = {0.f, 0.f, 0.f, 0.f};
-      float s1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int k = 0; k < C::KSTEPS; ++k) {
-        const int row = r0 + (mi >> 1) * 8 + mr;
-        const int d = 16 * k + (mi & 1) * 8;
-        uint32_t b00, b01, b10, b11;
-        ldmatrix_x4(kbase + (d >> 6) * C::CHUNK_BYTES + sw128(row, (d & 63) >> 3), b00, b01,
-                    b10, b11);
-        mma_bf16_16816(s0[0], s0[1], s0[2], s0[3], qa[k][0], qh[k][0], qa[k][1], qh[k][1], b00,
-                       b01, s0[0], s0[1], s0[2], s0[3]);
-        mma_bf16_16816(s1[0], s1[1], s1[2], s1[3], qa[k][0], qh[k][0], qa[k][1], qh[k][1], b10,
-                       b11, s1[0], s1[1], s1[2], s1[3]);
-      }
-
-      // ---- online softmax (base 2), row g (and g+8)
-      const int lim = valid - r0;  // tokens of this sub-tile inside the sequence
-      const bool v0 = 2 * tig < lim, v1 = 2 * tig + 1 < lim;
-      const bool v2 = 8 + 2 * tig < lim, v3 = 9 + 2 * tig < lim;
-      uint32_t pa0, pa1 = 0u, pa2, pa3 = 0u;
-      float alpha_lo, alpha_hi = 1.f;
-      {
-        const float x0 = v0 ? s0[0] * sl2 : -INFINITY;
-        const float x1 = v1 ? s0[1] * sl2 : -INFINITY;
-        const float x2 = v2 ? s1[0] * sl2 : -INFINITY;
-        const float x3 = v3 ? s1[1] * sl2 : -INFINITY;
-        float mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-        const float m_new = fmaxf(m_lo, mx);
-        alpha_lo = exp2f(m_lo - m_new);
-        m_lo = m_new;
-        pa0 = pack_bf16x2(exp2f(x0 - m_new), exp2f(x1 - m_new));
-        pa2 = pack_bf16x2(exp2f(x2 - m_new), exp2f(x3 - m_new));
-        l_lo = l_lo * alpha_lo + ((bf16_lo(pa0) + bf16_hi(pa0)) + (bf16_lo(pa2) + bf16_hi(pa2)));
-      }
-      if constexpr (C::ROWS16) {
-        const float x0 = v0 ? s0[2] * sl2 : -INFINITY;
-        const float x1 = v1 ? s0[3] * sl2 : -INFINITY;
-        const float x2 = v2 ? s1[2] * sl2 : -INFINITY;
-        const float x3 = v3 ? s1[3] * sl2 : -INFINITY;
-        float mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-        const float m_new = fmaxf(m_hi, mx);
-        alpha_hi = exp2f(m_hi - m_new);
-        m_hi = m_new;
-        pa1 = pack_bf16x2(exp2f(x0 - m_new), exp2f(x1 - m_new));
-        pa3 = pack_bf16x2(exp2f(x2 - m_new), exp2f(x3 - m_new));
-        l_hi = l_hi * alpha_hi + ((bf16_lo(pa1) + bf16_hi(pa1)) + (bf16_lo(pa3) + bf16_hi(pa3)));
-      }
-#pragma unroll
-      for (int j = 0; j < C::NT; ++j) {
-        o_lo[j][0] *= alpha_lo;
-        o_lo[j][1] *= alpha_lo;
-        if constexpr (C::ROWS16) {
-          o_hi[j][0] *= alpha_hi;
-          o_hi[j][1] *= alpha_hi;
-        }
-      }
-
-      // ---- O += P . V: B fragments for output columns 16*jp .. 16*jp+15
-#pragma unroll
-      for (int jp = 0; jp < C::NT / 2; ++jp) {
-        const int row = r0 + (mi & 1) * 8 + mr;
-        const int d = 16 * jp + (mi >> 1) * 8;
-        uint32_t w0, w1, w2, w3;
-        ldmatrix_x4_trans(vbase + (d >> 6) * C::CHUNK_BYTES + sw128(row, (d & 63) >> 3), w0, w1,
-                          w2, w3);
-        if constexpr (C::ROWS16) {
-          mma_bf16_16816(o_lo[2 * jp][0], o_lo[2 * jp][1], o_hi[2 * jp][0], o_hi[2 * jp][1], pa0,
-                         pa1, pa2, pa3, w0, w1, o_lo[2 * jp][0], o_lo[2 * jp][1],
-                         o_hi[2 * jp][0], o_hi[2 * jp][1]);
-          mma_bf16_16816(o_lo[2 * jp + 1][0], o_lo[2 * jp + 1][1], o_hi[2 * jp + 1][0],
-                         o_hi[2 * jp + 1][1], pa0, pa1, pa2, pa3, w2, w3, o_lo[2 * jp + 1][0],
-                         o_lo[2 * jp + 1][1], o_hi[2 * jp + 1][0], o_hi[2 * jp + 1][1]);
-        } else {
-          float dead0, dead1;
-          mma_bf16_16816(o_lo[2 * jp][0], o_lo[2 * jp][1], dead0, dead1, pa0, 0u, pa2, 0u, w0,
-                         w1, o_lo[2 * jp][0], o_lo[2 * jp][1], 0.f, 0.f);
-          mma_bf16_16816(o_lo[2 * jp + 1][0], o_lo[2 * jp + 1][1], dead0, dead1, pa0, 0u, pa2,
-                         0u, w2, w3, o_lo[2 * jp + 1][0], o_lo[2 * jp + 1][1], 0.f, 0.f);
-        }
-      }
-    }
+    if (valid < TILE_T) zero_tail_rows<C>(st_ptr, valid, lane);
+    acc.tile(smem_addr(st_ptr), valid, sl2, lane);
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_addr(&empty_bar[stage]));
   }
 
   // ---- merge the consumer warps: (m, l, O) per warp -> shared memory -> combine
-  l_lo += __shfl_xor_sync(kFull, l_lo, 1);
-  l_lo += __shfl_xor_sync(kFull, l_lo, 2);
-  if constexpr (C::ROWS16) {
-    l_hi += __shfl_xor_sync(kFull, l_hi, 1);
-    l_hi += __shfl_xor_sync(kFull, l_hi, 2);
-  }
+  acc.reduce_l();
   named_barrier_sync(1, NCW * 32);  // every consumer is done with the stage ring
   float* mo = reinterpret_cast<float*>(smem);  // [NCW][ROWS][D]
   if (tig == 0) {
-    sm_m[warp][g] = m_lo;
-    sm_l[warp][g] = l_lo;
+    sm_m[warp][g] = acc.m_lo;
+    sm_l[warp][g] = acc.l_lo;
     if constexpr (C::ROWS16) {
-      sm_m[warp][g + 8] = m_hi;
-      sm_l[warp][g + 8] = l_hi;
+      sm_m[warp][g + 8] = acc.m_hi;
+      sm_l[warp][g + 8] = acc.l_hi;
     }
   }
 #pragma unroll
   for (int j = 0; j < C::NT; ++j) {
     *reinterpret_cast<float2*>(mo + (warp * ROWS + g) * D + 8 * j + 2 * tig) =
-        make_float2(o_lo[j][0], o_lo[j][1]);
+        make_float2(acc.o_lo[j][0], acc.o_lo[j][1]);
     if constexpr (C::ROWS16)
       *reinterpret_cast<float2*>(mo + (warp * ROWS + g + 8) * D + 8 * j + 2 * tig) =
-          make_float2(o_hi[j][0], o_hi[j][1]);
+          make_float2(acc.o_hi[j][0], acc.o_hi[j][1]);
   }
   named_barrier_sync(1, NCW * 32);
 
@@ -395,7 +233,11 @@ __global__ void __launch_bounds__(C::THREADS)
   }
 }
 
+}  // namespace
+
 // ---- tensor maps --------------------------------------------------------------
+
+namespace {
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -413,6 +255,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 
 // View a pool [NB][BS][Hkv][D] (bf16) as a 4-D tensor; box = one block's BS rows x 64
 // columns of one KV head, 128-byte swizzled in shared memory.
+}  // namespace
+
 bool make_pool_map(CUtensorMap* map, const void* pool, int NB, int BS, int Hkv, int D) {
   auto encode = get_encode_fn();
   if (!encode) return false;
@@ -430,6 +274,8 @@ bool make_pool_map(CUtensorMap* map, const void* pool, int NB, int BS, int Hkv, 
   return r == CUDA_SUCCESS;
 }
 
+namespace {
+
 template <class C>
 cudaError_t launch_cfg(const DecodeParams& p, cudaStream_t stream) {
   CUtensorMap tmk, tmv;
@@ -437,13 +283,9 @@ cudaError_t launch_cfg(const DecodeParams& p, cudaStream_t stream) {
       !make_pool_map(&tmv, p.v_pool, p.num_blocks, C::BS, p.Hkv, C::D))
     return cudaErrorInvalidValue;
   auto kern = decode_tc_kernel<C>;
-  static bool attr_set = false;  // per instantiation
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
   const long long grid = static_cast<long long>(p.B) * p.Hkv * p.max_parts;
   if (grid <= 0) return cudaSuccess;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;

@@ -2,6 +2,7 @@
 // launchers the C ABI (api.cu) dispatches to.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -25,6 +26,24 @@ struct DecodeParams {
   float* ws_acc;               // [B][Hq][max_parts][D]: unnormalised output
   int32_t* err;                // nullable device error flag
 };
+
+// Parameters of the balanced persistent ("stream") tensor-core kernel.
+struct StreamParams {
+  DecodeParams d;
+  int streams;     // consumer warps in the grid = tile ranges
+  int32_t* meta;   // [streams][4]: unit in slot 0, it starts in this stream, unit in slot 1
+  float* pml;      // [streams][2][G][2]: (max, sum) of cut-unit pieces, base 2
+  float* pacc;     // [streams][2][G][D]: unnormalised outputs of those pieces
+};
+
+// One wave of the stream kernel for this shape on the current device (0 if unknown).
+int stream_grid(int D, int block_size, int G, int B);
+size_t stream_workspace_bytes(int streams, int G, int D);
+void stream_carve(StreamParams* sp, void* workspace);
+cudaError_t launch_decode_stream(const StreamParams& sp, int grid, cudaStream_t stream);
+
+// 4-D TMA view of a bf16 pool [NB][BS][Hkv][D]: box = BS rows x 64 columns of one head.
+bool make_pool_map(CUtensorMap* map, const void* pool, int NB, int BS, int Hkv, int D);
 
 // Launch the bf16 tensor-core decode kernel (+ reduce when max_parts > 1).
 cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t stream);

@@ -1,0 +1,204 @@
+// Per-warp tensor-core math of the bf16 decode kernels: one 16-token sub-tile of one KV
+// head against the G query heads of its group.
+//
+// S = Q . K^T with m16n8k16 bf16 MMAs (query heads as the 16 rows, padded), an fp32
+// online softmax in base 2, and O += P . V with P fed back from registers as the A
+// operand, split into bf16 hi + lo parts so that P keeps ~16 significant bits.  K and V
+// come from a shared-memory tile written by TMA with 128-byte swizzle: row r's 16-byte
+// column chunk c sits at r*128 + ((c ^ (r & 7)) << 4) inside each 64-column chunk.
+#pragma once
+
+#include "pa_device.cuh"
+
+namespace pa {
+
+template <int D_, int BS_, bool ROWS16_>
+struct TileCfg {
+  static constexpr int D = D_;
+  static constexpr int BS = BS_;
+  static constexpr bool ROWS16 = ROWS16_;
+  static constexpr int TILE_T = BS > 16 ? BS : 16;   // tokens per pipeline stage
+  static constexpr int BPS = TILE_T / BS;            // blocks per stage
+  static constexpr int SUBT = TILE_T / 16;           // 16-token sub-tiles per stage
+  static constexpr int DCH = D / 64;                 // 128-byte column chunks per row
+  static constexpr int CHUNK_BYTES = TILE_T * 128;
+  static constexpr int TILE_BYTES = DCH * CHUNK_BYTES;  // one K (or V) tile
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  static constexpr int ROWS = ROWS16 ? 16 : 8;          // query-head rows kept
+  static constexpr int KSTEPS = D / 16;
+  static constexpr int NT = D / 8;                      // output n-tiles of 8 columns
+  static_assert(D == 64 || D == 128, "head dim");
+  static_assert(BS == 8 || BS == 16 || BS == 32, "block size");
+};
+
+__device__ __forceinline__ uint32_t sw128(int row, int c16) {
+  return static_cast<uint32_t>(row * 128 + ((c16 ^ (row & 7)) << 4));
+}
+
+// Online-softmax state and output accumulator of one warp for one (sequence, KV head).
+// Lane (g = lane/4, tig = lane%4) owns rows g (and g+8 with ROWS16) and output columns
+// 8j + 2tig, 8j + 2tig + 1 of every n-tile j.
+template <class C>
+struct WarpAcc {
+  float o_lo[C::NT][2];
+  float o_hi[C::NT][2];
+  float m_lo, m_hi, l_lo, l_hi;
+  uint32_t qa[C::KSTEPS][2];  // Q rows g as A fragments (k-step columns 2tig.., 8+2tig..)
+  uint32_t qh[C::KSTEPS][2];  // Q rows g+8
+
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int j = 0; j < C::NT; ++j) {
+      o_lo[j][0] = o_lo[j][1] = 0.f;
+      o_hi[j][0] = o_hi[j][1] = 0.f;
+    }
+    m_lo = m_hi = -INFINITY;
+    l_lo = l_hi = 0.f;
+  }
+
+  // Q rows of one group (G heads, row-major [G][D] bf16); rows >= G are zero.
+  __device__ __forceinline__ void load_q(const __nv_bfloat16* qrow, int G, int lane) {
+    const int g = lane >> 2, tig = lane & 3;
+#pragma unroll
+    for (int k = 0; k < C::KSTEPS; ++k) {
+      const bool lo_ok = g < G;
+      qa[k][0] = lo_ok ? __ldg(reinterpret_cast<const unsigned int*>(qrow + g * C::D + 16 * k + 2 * tig)) : 0u;
+      qa[k][1] = lo_ok ? __ldg(reinterpret_cast<const unsigned int*>(qrow + g * C::D + 16 * k + 8 + 2 * tig)) : 0u;
+      if constexpr (C::ROWS16) {
+        const bool hi_ok = g + 8 < G;
+        qh[k][0] = hi_ok ? __ldg(reinterpret_cast<const unsigned int*>(qrow + (g + 8) * C::D + 16 * k + 2 * tig)) : 0u;
+        qh[k][1] = hi_ok ? __ldg(reinterpret_cast<const unsigned int*>(qrow + (g + 8) * C::D + 16 * k + 8 + 2 * tig)) : 0u;
+      } else {
+        qh[k][0] = 0u;
+        qh[k][1] = 0u;
+      }
+    }
+  }
+
+  // One online-softmax row update for scores x0..x3 (tokens 2tig, 2tig+1, 8+2tig, 9+2tig).
+  __device__ __forceinline__ static float row_update(float x0, float x1, float x2, float x3,
+                                                     float& m, float& l, uint32_t& hi0,
+                                                     uint32_t& lo0, uint32_t& hi2,
+                                                     uint32_t& lo2) {
+    constexpr unsigned kFull = 0xffffffffu;
+    float mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+    const float m_new = fmaxf(m, mx);
+    const float alpha = exp2f(m - m_new);
+    m = m_new;
+    const float e0 = exp2f(x0 - m_new), e1 = exp2f(x1 - m_new);
+    const float e2 = exp2f(x2 - m_new), e3 = exp2f(x3 - m_new);
+    split_bf16x2(e0, e1, hi0, lo0);
+    split_bf16x2(e2, e3, hi2, lo2);
+    l = l * alpha + ((e0 + e1) + (e2 + e3));
+    return alpha;
+  }
+
+  // Consume one staged tile (K at kbase, V at kbase + TILE_BYTES, shared addresses) with
+  // `valid` tokens (1..TILE_T) inside the sequence; rows >= valid are masked (their V rows
+  // must already be zero).
+  __device__ __forceinline__ void tile(uint32_t kbase, int valid, float sl2, int lane) {
+    const uint32_t vbase = kbase + C::TILE_BYTES;
+    const int tig = lane & 3;
+    const int mi = lane >> 3, mr = lane & 7;
+#pragma unroll
+    for (int st = 0; st < C::SUBT; ++st) {
+      const int r0 = st * 16;
+      if (r0 >= valid) break;
+      float s0[4] = {0.f, 0.f, 0.f, 0.f};
+      float s1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < C::KSTEPS; ++k) {
+        const int row = r0 + (mi >> 1) * 8 + mr;
+        const int d = 16 * k + (mi & 1) * 8;
+        uint32_t b00, b01, b10, b11;
+        ldmatrix_x4(kbase + (d >> 6) * C::CHUNK_BYTES + sw128(row, (d & 63) >> 3), b00, b01, b10,
+                    b11);
+        mma_bf16_16816(s0[0], s0[1], s0[2], s0[3], qa[k][0], qh[k][0], qa[k][1], qh[k][1], b00,
+                       b01, s0[0], s0[1], s0[2], s0[3]);
+        mma_bf16_16816(s1[0], s1[1], s1[2], s1[3], qa[k][0], qh[k][0], qa[k][1], qh[k][1], b10,
+                       b11, s1[0], s1[1], s1[2], s1[3]);
+      }
+      const int lim = valid - r0;
+      const bool v0 = 2 * tig < lim, v1 = 2 * tig + 1 < lim;
+      const bool v2 = 8 + 2 * tig < lim, v3 = 9 + 2 * tig < lim;
+      uint32_t pa0, pa1 = 0u, pa2, pa3 = 0u;   // P hi parts (A fragment registers)
+      uint32_t pr0, pr1 = 0u, pr2, pr3 = 0u;   // P lo parts
+      const float alpha_lo =
+          row_update(v0 ? s0[0] * sl2 : -INFINITY, v1 ? s0[1] * sl2 : -INFINITY,
+                     v2 ? s1[0] * sl2 : -INFINITY, v3 ? s1[1] * sl2 : -INFINITY, m_lo, l_lo,
+                     pa0, pr0, pa2, pr2);
+      float alpha_hi = 1.f;
+      if constexpr (C::ROWS16)
+        alpha_hi = row_update(v0 ? s0[2] * sl2 : -INFINITY, v1 ? s0[3] * sl2 : -INFINITY,
+                              v2 ? s1[2] * sl2 : -INFINITY, v3 ? s1[3] * sl2 : -INFINITY, m_hi,
+                              l_hi, pa1, pr1, pa3, pr3);
+#pragma unroll
+      for (int j = 0; j < C::NT; ++j) {
+        o_lo[j][0] *= alpha_lo;
+        o_lo[j][1] *= alpha_lo;
+        if constexpr (C::ROWS16) {
+          o_hi[j][0] *= alpha_hi;
+          o_hi[j][1] *= alpha_hi;
+        }
+      }
+#pragma unroll
+      for (int jp = 0; jp < C::NT / 2; ++jp) {
+        const int row = r0 + (mi & 1) * 8 + mr;
+        const int d = 16 * jp + (mi >> 1) * 8;
+        uint32_t w0, w1, w2, w3;
+        ldmatrix_x4_trans(vbase + (d >> 6) * C::CHUNK_BYTES + sw128(row, (d & 63) >> 3), w0, w1,
+                          w2, w3);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const uint32_t a0 = half ? pr0 : pa0, a1 = half ? pr1 : pa1;
+          const uint32_t a2 = half ? pr2 : pa2, a3 = half ? pr3 : pa3;
+          if constexpr (C::ROWS16) {
+            mma_bf16_16816(o_lo[2 * jp][0], o_lo[2 * jp][1], o_hi[2 * jp][0], o_hi[2 * jp][1], a0,
+                           a1, a2, a3, w0, w1, o_lo[2 * jp][0], o_lo[2 * jp][1], o_hi[2 * jp][0],
+                           o_hi[2 * jp][1]);
+            mma_bf16_16816(o_lo[2 * jp + 1][0], o_lo[2 * jp + 1][1], o_hi[2 * jp + 1][0],
+                           o_hi[2 * jp + 1][1], a0, a1, a2, a3, w2, w3, o_lo[2 * jp + 1][0],
+                           o_lo[2 * jp + 1][1], o_hi[2 * jp + 1][0], o_hi[2 * jp + 1][1]);
+          } else {
+            float dead0, dead1;
+            mma_bf16_16816(o_lo[2 * jp][0], o_lo[2 * jp][1], dead0, dead1, a0, 0u, a2, 0u, w0, w1,
+                           o_lo[2 * jp][0], o_lo[2 * jp][1], 0.f, 0.f);
+            mma_bf16_16816(o_lo[2 * jp + 1][0], o_lo[2 * jp + 1][1], dead0, dead1, a0, 0u, a2, 0u,
+                           w2, w3, o_lo[2 * jp + 1][0], o_lo[2 * jp + 1][1], 0.f, 0.f);
+          }
+        }
+      }
+    }
+  }
+
+  // Sum the per-lane partial row sums over the 4 lanes of each row.
+  __device__ __forceinline__ void reduce_l() {
+    constexpr unsigned kFull = 0xffffffffu;
+    l_lo += __shfl_xor_sync(kFull, l_lo, 1);
+    l_lo += __shfl_xor_sync(kFull, l_lo, 2);
+    if constexpr (C::ROWS16) {
+      l_hi += __shfl_xor_sync(kFull, l_hi, 1);
+      l_hi += __shfl_xor_sync(kFull, l_hi, 2);
+    }
+  }
+};
+
+// Zero the V rows [valid, TILE_T) of a staged tile (their slots may hold anything), then
+// order those generic-proxy writes before later TMA writes to the same stage.
+template <class C>
+__device__ __forceinline__ void zero_tail_rows(uint8_t* stage_ptr, int valid, int lane) {
+  uint8_t* vt = stage_ptr + C::TILE_BYTES;
+  const int nchunks = (C::TILE_T - valid) * C::DCH * 8;
+  for (int i = lane; i < nchunks; i += 32) {
+    const int r = valid + i / (C::DCH * 8);
+    const int rem = i % (C::DCH * 8);
+    *reinterpret_cast<uint4*>(vt + (rem >> 3) * C::CHUNK_BYTES + r * 128 + (rem & 7) * 16) =
+        make_uint4(0u, 0u, 0u, 0u);
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+}
+
+}  // namespace pa

@@ -19,8 +19,8 @@ pytestmark = pytest.mark.gpu
 AUTO, GENERIC, TENSOR = 0, 1, 2
 
 
-def check(w, partition_tokens=0, path=AUTO):
-    g = gpu_step(w, partition_tokens=partition_tokens, path=path)
+def check(w, partition_tokens=0, path=AUTO, max_ctas=0):
+    g = gpu_step(w, partition_tokens=partition_tokens, path=path, max_ctas=max_ctas)
     r = oracle_step(w)
     assert g["err"] == 0
     np.testing.assert_array_equal(g["slots"], r["slots"])
@@ -48,10 +48,13 @@ SCALED = {
 
 
 @pytest.mark.parametrize("name", sorted(SCALED))
-@pytest.mark.parametrize("partition,path", [(0, AUTO), (16, TENSOR), (64, TENSOR), (0, GENERIC),
-                                            (32, GENERIC)])
-def test_scaled_workloads(name, partition, path):
-    check(SCALED[name](), partition_tokens=partition, path=path)
+@pytest.mark.parametrize("partition,path,ctas", [(0, AUTO, 0), (0, TENSOR, 1), (0, TENSOR, 3),
+                                                 (0, TENSOR, 37), (16, TENSOR, 0), (64, TENSOR, 0),
+                                                 (0, GENERIC, 0), (32, GENERIC, 0)])
+def test_scaled_workloads(name, partition, path, ctas):
+    """AUTO/TENSOR with partition 0 run the balanced stream kernel (max_ctas varies where
+    the tile ranges cut units); partition > 0 runs the partition kernels."""
+    check(SCALED[name](), partition_tokens=partition, path=path, max_ctas=ctas)
 
 
 # ---- lengths around block and tile boundaries ---------------------------------
@@ -64,6 +67,7 @@ EDGE_LENS = [1, 2, 15, 16, 17, 31, 32, 33, 47, 48, 49, 63, 64, 65, 127, 129]
 def test_edge_lengths_tensor_path(bs, G):
     w = workloads.independent(EDGE_LENS, Hq=2 * G, Hkv=2, bs=bs, seed=3000 + bs + G)
     check(w, path=TENSOR)
+    check(w, path=TENSOR, max_ctas=2)
     check(w, partition_tokens=32, path=TENSOR)
 
 
@@ -79,6 +83,7 @@ def test_edge_lengths_generic_path(D, dtype, bs):
 def test_head_dim_64_tensor_path():
     w = workloads.independent([5, 70, 300, 33], Hq=16, Hkv=2, D=64, bs=16, seed=4100)
     check(w, path=TENSOR)
+    check(w, path=TENSOR, max_ctas=1)
     check(w, partition_tokens=64, path=TENSOR)
 
 
@@ -89,16 +94,16 @@ def test_gqa_group_wider_than_16_uses_cuda_cores():
 
 # ---- direct decode cases (no allocator): empty rows, poisoned slots, logits ----
 
-def _decode_direct(q, kp, vp, tables, lens, scale, path=AUTO, partition=0, dev="cuda"):
+def _decode_direct(q, kp, vp, tables, lens, scale, path=AUTO, partition=0, dev="cuda", max_ctas=0):
     import paged_kv_cache_350_b200 as pa
     out = torch.full_like(q, float("nan"))
     B, Hq, D = q.shape
-    bs = kp.shape[1]
-    n = pa.pa_decode_workspace_size(B, Hq, D, tables.shape[1] * bs, bs, partition)
+    bs, Hkv = kp.shape[1], kp.shape[2]
+    n = pa.pa_decode_workspace_size(B, Hq, Hkv, D, tables.shape[1] * bs, bs, partition)
     ws = torch.empty(max(n, 1), dtype=torch.uint8, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     pa.pa_decode(out, q, kp, vp, tables, lens, scale, workspace=ws, err_flag=err,
-                 partition_tokens=partition, path=path)
+                 partition_tokens=partition, path=path, max_ctas=max_ctas)
     torch.cuda.synchronize()
     return out, int(err.item())
 
@@ -107,8 +112,9 @@ def _bf16_host(t):
     return t.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
 
 
-@pytest.mark.parametrize("path,partition", [(TENSOR, 0), (TENSOR, 16), (GENERIC, 0), (GENERIC, 16)])
-def test_empty_rows_poisoned_tails_and_minus_one_tables(path, partition):
+@pytest.mark.parametrize("path,partition,ctas", [(TENSOR, 0, 0), (TENSOR, 0, 1), (TENSOR, 16, 0),
+                                                 (GENERIC, 0, 0), (GENERIC, 16, 0)])
+def test_empty_rows_poisoned_tails_and_minus_one_tables(path, partition, ctas):
     rng = np.random.default_rng(5)
     B, Hq, Hkv, D, bs, NB = 6, 8, 2, 128, 16, 40
     lens = np.array([0, 1, 17, 0, 33, 50], dtype=np.int32)
@@ -133,15 +139,16 @@ def test_empty_rows_poisoned_tails_and_minus_one_tables(path, partition):
     kp[mask] = float("nan")
     vp[mask] = float("inf")
     out, err = _decode_direct(q.cuda(), kp.cuda(), vp.cuda(), torch.from_numpy(tables).cuda(),
-                              torch.from_numpy(lens).cuda(), 0.088, path=path, partition=partition)
+                              torch.from_numpy(lens).cuda(), 0.088, path=path, partition=partition,
+                              max_ctas=ctas)
     assert err == 0
     w = workloads.independent([1], dtype="bf16")
     assert_close(w, out, ref)
     assert torch.equal(out[0].float().cpu(), torch.zeros(Hq, D))
 
 
-@pytest.mark.parametrize("path", [TENSOR, GENERIC])
-def test_large_logits_and_rising_logits_force_rescaling(path):
+@pytest.mark.parametrize("path,ctas", [(TENSOR, 0), (TENSOR, 1), (GENERIC, 0)])
+def test_large_logits_and_rising_logits_force_rescaling(path, ctas):
     rng = np.random.default_rng(6)
     B, Hq, Hkv, D, bs = 2, 8, 1, 128, 16
     L = 300
@@ -162,7 +169,8 @@ def test_large_logits_and_rising_logits_force_rescaling(path):
     tq, tk, tv = (torch.from_numpy(x).to(torch.bfloat16) for x in (q, kp, vp))
     ref = ref_decode(_bf16_host(tq), _bf16_host(tk), _bf16_host(tv), tables, lens, 1.0)
     out, err = _decode_direct(tq.cuda(), tk.cuda(), tv.cuda(), torch.from_numpy(tables).cuda(),
-                              torch.from_numpy(lens).cuda(), 1.0, path=path, partition=64)
+                              torch.from_numpy(lens).cuda(), 1.0, path=path,
+                              partition=0 if path == TENSOR else 64, max_ctas=ctas)
     assert err == 0 and torch.isfinite(out.float()).all()
     assert_close(workloads.independent([1]), out, ref)
 
@@ -243,11 +251,11 @@ def test_bad_block_id_and_bad_length_set_the_flag():
     vp = torch.randn_like(kp)
     tables = torch.tensor([[0, 99, 1], [2, 3, -7]], dtype=torch.int32, device="cuda")
     lens = torch.tensor([40, 30], dtype=torch.int32, device="cuda")
-    for path in (TENSOR, GENERIC):
-        out, err = _decode_direct(q, kp, vp, tables, lens, 0.1, path=path)
+    for path, part in ((TENSOR, 0), (TENSOR, 16), (GENERIC, 0)):
+        out, err = _decode_direct(q, kp, vp, tables, lens, 0.1, path=path, partition=part)
         assert err & pa.binding.PA_DEVERR_BAD_BLOCK_ID
         assert pa.pa_status_from_device_flag(err) == pa.binding.PA_ERR_BAD_BLOCK_ID
         out, err = _decode_direct(q, kp, vp, tables[:, :1].contiguous(),
                                   torch.tensor([17, -1], dtype=torch.int32, device="cuda"), 0.1,
-                                  path=path)
+                                  path=path, partition=part)
         assert err & pa.binding.PA_DEVERR_BAD_SEQ_LEN

@@ -1,0 +1,40 @@
+"""GPU parity at the full serving sizes, in the launch configuration bench.py times
+(automatic path and partitioning, workspace from pa_decode_workspace_size).
+
+The oracle computes a sample of batch rows one by one; the remaining rows are
+checked for the properties that hold at any size (finite, and each output row
+inside the convex hull bound max|v| of its values)."""
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from _parity import assert_close, gpu_step, oracle_step
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+FULL = {
+    "gqa": (workloads.gqa, [0, 1, 77, 128, 255]),
+    "mha": (workloads.mha, [0, 31, 63]),
+    "long": (workloads.long_context, [0, 5]),
+    "prefix": (workloads.prefix, [0, 9, 255]),
+    "prefix_cow": (workloads.prefix_cow, [0, 7, 8, 250]),
+}
+
+
+@pytest.mark.parametrize("name", sorted(FULL))
+def test_full_size_sampled_rows(name):
+    build, rows = FULL[name]
+    w = build()
+    g = gpu_step(w)
+    assert g["err"] == 0
+    out = g["out"].float()
+    assert torch.isfinite(out).all()
+    # |o| <= max |v| for a convex combination: a property of every row
+    assert float(out.abs().max()) <= 6.0
+    r = oracle_step(w, rows=rows)
+    np.testing.assert_array_equal(g["slots"], r["slots"])
+    np.testing.assert_array_equal(g["pairs"], r["pairs"])
+    np.testing.assert_array_equal(g["tables"], r["tables"])
+    assert_close(w, g["out"][torch.as_tensor(rows)], r["out"])

@@ -36,13 +36,17 @@ def test_status_strings_and_flag_mapping():
 
 def test_workspace_size_bounds_every_partition():
     from paged_kv_cache_350_b200 import binding as b
-    assert b.pa_decode_workspace_size(8, 64, 128, 512, 16, 0) == 0       # no split possible
-    n0 = b.pa_decode_workspace_size(256, 32, 128, 4096, 16, 0)
+    assert b.pa_decode_workspace_size(8, 64, 8, 128, 512, 4, 0) == 0     # CUDA cores, one pass
+    n0 = b.pa_decode_workspace_size(256, 32, 8, 128, 4096, 16, 0)
     parts = 4096 // 512
     assert n0 >= 256 * 32 * parts * (128 + 2) * 4
-    assert b.pa_decode_workspace_size(2, 4, 64, 64, 4, 4) >= 2 * 4 * 16 * 66 * 4
+    assert b.pa_decode_workspace_size(2, 4, 4, 64, 64, 4, 4) >= 2 * 4 * 16 * 66 * 4
+    # the balanced kernel needs room for two partial pieces per stream, whatever B
+    assert b.pa_decode_workspace_size(1, 8, 1, 128, 16, 16, 0) >= 4 * 2 * 8 * 130 * 4
     with pytest.raises(b.PAError):
-        b.pa_decode_workspace_size(2, 4, 64, 64, 4, 6)   # not a multiple of block_size
+        b.pa_decode_workspace_size(2, 4, 4, 64, 64, 4, 6)   # not a multiple of block_size
+    with pytest.raises(b.PAError):
+        b.pa_decode_workspace_size(2, 6, 4, 64, 64, 4, 0)   # Hq % Hkv
 
 
 def _call_decode(**kw):
@@ -50,12 +54,25 @@ def _call_decode(**kw):
     a = dict(out=16, q=16, k=16, v=16, t=16, l=16, B=2, Hq=8, Hkv=2, D=128, bs=16, MB=4, NB=8,
              scale=0.1, dtype=b.PA_BF16, ws=0, wsb=0, err=0, stream=0, part=0, path=0)
     a.update(kw)
-    opts = b.pa_decode_opts(a["part"], a["path"])
+    opts = b.pa_decode_opts(a["part"], a["path"], 0)
     vp = ctypes.c_void_p
     return b.lib.pa_decode_ex(vp(a["out"]), vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["t"]),
                               vp(a["l"]), a["B"], a["Hq"], a["Hkv"], a["D"], a["bs"], a["MB"],
                               a["NB"], a["scale"], a["dtype"], vp(a["ws"]), a["wsb"], vp(a["err"]),
                               vp(a["stream"]), ctypes.byref(opts))
+
+
+def test_plan_on_a_machine_without_gpu_falls_back_to_partitions():
+    from paged_kv_cache_350_b200 import binding as b
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("plan depends on the device here")
+    n = b.pa_decode_workspace_size(256, 32, 8, 128, 4112, 16, 0)
+    plan = b.pa_decode_plan(256, 32, 8, 128, 16, 257, b.PA_BF16, n)
+    assert plan["kernel"] == b.PA_KERNEL_TC_PARTITION and plan["launches"] == 2
+    plan = b.pa_decode_plan(2, 4, 4, 64, 4, 4, b.PA_F32, 0)
+    assert plan["kernel"] == b.PA_KERNEL_GENERIC and plan["launches"] == 1
+    assert b.pa_decode_plan(0, 4, 4, 64, 4, 4, b.PA_F32, 0)["launches"] == 0
 
 
 def test_decode_argument_errors_are_reported_before_any_launch():
