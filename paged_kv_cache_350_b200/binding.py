@@ -14,7 +14,9 @@ import os
 
 import numpy as np
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedattn.so")
+# The in-tree build; PAGEDATTN_LIB may name another build of the same library.
+_LIB_PATH = os.environ.get("PAGEDATTN_LIB") or os.path.join(
+    os.path.dirname(os.path.abspath(__file__)), "libpagedattn.so")
 
 # pa_status
 PA_OK = 0

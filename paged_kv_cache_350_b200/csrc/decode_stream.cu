@@ -31,6 +31,15 @@ namespace pa {
 
 namespace {
 
+// Build-time tunables: ring stages per stream, and the CTAs per SM the register
+// allocation is bounded for (0 = let the compiler choose).
+#ifndef PA_STREAM_SPW
+#define PA_STREAM_SPW 2
+#endif
+#ifndef PA_STREAM_MIN_CTAS
+#define PA_STREAM_MIN_CTAS 3
+#endif
+
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kNCW = 4;                      // consumer warps (= streams) per CTA
 constexpr int kThreads = (kNCW + 1) * 32;
@@ -40,11 +49,13 @@ struct StreamCfg : TileCfg<D_, BS_, ROWS16_> {
   static constexpr int SPW = SPW_;                 // ring stages per stream
   static constexpr int NST = kNCW * SPW;
   static constexpr int RING_BYTES = NST * StreamCfg::STAGE_BYTES;
+  static constexpr int Q_BYTES = WarpAcc<StreamCfg, true>::Q_BYTES;  // per consumer warp
+  static constexpr int FIXED_BYTES = RING_BYTES + kNCW * Q_BYTES;
 };
 
 template <class C>
 size_t stream_smem_bytes(int B) {
-  return C::RING_BYTES + 1024 + static_cast<size_t>(B + 1) * 4;
+  return C::FIXED_BYTES + 1024 + static_cast<size_t>(B + 1) * 4;
 }
 
 __device__ __forceinline__ int clamp_len(const DecodeParams& p, int b, bool flag) {
@@ -71,20 +82,21 @@ struct TilePos {
   int b, kvh, j, nt;
 };
 
-// Global tile index -> (sequence, KV head, tile within the unit).
-__device__ __forceinline__ TilePos locate(const int* P, int B, int Hkv, long long g) {
+// Global tile index -> (sequence, KV head, tile within the unit).  The host keeps the
+// total tile count below 2^31.
+__device__ __forceinline__ TilePos locate(const int* P, int B, int Hkv, int g) {
   TilePos t;
-  const int v = static_cast<int>(g / Hkv);
+  const int v = g / Hkv;
   t.b = upper_bound(P, B + 1, v) - 1;
   t.nt = P[t.b + 1] - P[t.b];
-  const int off = static_cast<int>(g - static_cast<long long>(Hkv) * P[t.b]);
+  const int off = g - Hkv * P[t.b];
   t.kvh = off / t.nt;
   t.j = off - t.kvh * t.nt;
   return t;
 }
 
 template <class C>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, PA_STREAM_MIN_CTAS)
     decode_stream_kernel(const __grid_constant__ CUtensorMap tmk,
                          const __grid_constant__ CUtensorMap tmv, const StreamParams sp) {
   constexpr int D = C::D, BS = C::BS, TILE_T = C::TILE_T, SPW = C::SPW, NST = C::NST;
@@ -96,7 +108,8 @@ __global__ void __launch_bounds__(kThreads)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  int* P = reinterpret_cast<int*>(smem + C::RING_BYTES);  // [B + 1] tiles before sequence b
+  uint8_t* qtiles = smem + C::RING_BYTES;                  // [kNCW][Q_BYTES]
+  int* P = reinterpret_cast<int*>(smem + C::FIXED_BYTES);  // [B + 1] tiles before sequence b
   __shared__ __align__(8) uint64_t full_bar[NST];
   __shared__ __align__(8) uint64_t empty_bar[NST];
   __shared__ int warp_sum[kThreads / 32];
@@ -147,9 +160,9 @@ __global__ void __launch_bounds__(kThreads)
   }
   __syncthreads();
 
-  const long long T = static_cast<long long>(Hkv) * P[B];
-  const long long S = static_cast<long long>(gridDim.x) * kNCW;
-  const long long per = (T + S - 1) / S;
+  const int T = Hkv * P[B];
+  const int S = static_cast<int>(gridDim.x) * kNCW;
+  const int per = (T + S - 1) / S;
 
   if (warp == kNCW) {
     // ---------------- producer warp: feeds the 4 streams of this CTA ----------------
@@ -159,9 +172,9 @@ __global__ void __launch_bounds__(kThreads)
     }
     const uint64_t policy = l2_policy_evict_first();
     const int my_w = lane & 3;
-    const long long my_s = static_cast<long long>(blockIdx.x) * kNCW + my_w;
-    const long long my_beg = min(T, my_s * per);
-    const int my_cnt = static_cast<int>(min(T, my_beg + per) - my_beg);
+    const int my_s = static_cast<int>(blockIdx.x) * kNCW + my_w;
+    const int my_beg = min(T, my_s * per);
+    const int my_cnt = min(T, my_beg + per) - my_beg;
     int rounds = my_cnt;
     rounds = max(rounds, __shfl_xor_sync(kFull, rounds, 1));
     rounds = max(rounds, __shfl_xor_sync(kFull, rounds, 2));
@@ -227,27 +240,28 @@ __global__ void __launch_bounds__(kThreads)
   }
 
   // ---------------- consumer warp = one stream ----------------
-  const long long s = static_cast<long long>(blockIdx.x) * kNCW + warp;
-  const long long beg = min(T, s * per);
-  const long long end = min(T, beg + per);
+  const int s = static_cast<int>(blockIdx.x) * kNCW + warp;
+  const int beg = min(T, s * per);
+  const int end = min(T, beg + per);
   const int g = lane >> 2, tig = lane & 3;
   const float sl2 = p.scale_log2;
   int unit_a = -1, a_starts = 0, unit_b = -1;
   int i = 0;  // tiles consumed by this stream (ring position)
   bool ok = true;
-  WarpAcc<C> acc;
+  WarpAcc<C, true> acc;
+  uint8_t* my_q = qtiles + warp * C::Q_BYTES;
 
-  long long gpos = beg;
+  int gpos = beg;
   while (gpos < end && ok) {
     const TilePos t = locate(P, B, Hkv, gpos);
     const int L = clamp_len(p, t.b, false);
-    const long long ubeg = static_cast<long long>(Hkv) * P[t.b] + static_cast<long long>(t.kvh) * t.nt;
-    const long long uend = ubeg + t.nt;
-    const long long pend = min(end, uend);
+    const int ubeg = Hkv * P[t.b] + t.kvh * t.nt;
+    const int uend = ubeg + t.nt;
+    const int pend = min(end, uend);
     const size_t head0 = static_cast<size_t>(t.b) * p.Hq + static_cast<size_t>(t.kvh) * G;
-    acc.load_q(static_cast<const __nv_bfloat16*>(p.q) + head0 * D, G, lane);
+    acc.stage_q(static_cast<const __nv_bfloat16*>(p.q) + head0 * D, G, my_q, lane);
     acc.reset();
-    const int jend = t.j + static_cast<int>(pend - gpos);
+    const int jend = t.j + (pend - gpos);
     for (int j = t.j; j < jend; ++j, ++i) {
       const int stage = warp * SPW + i % SPW;
       if (!mbar_wait(smem_addr(&full_bar[stage]), (i / SPW) & 1, p.err)) {
@@ -385,7 +399,7 @@ cudaError_t launch_stream_cfg(const StreamParams& sp, int grid, cudaStream_t str
   return cudaGetLastError();
 }
 
-constexpr int kSPW = 2;
+constexpr int kSPW = PA_STREAM_SPW;
 
 template <int D, int BS>
 int grid_d_bs(bool rows16, int B, int sms) {

@@ -38,13 +38,64 @@ __device__ __forceinline__ uint32_t sw128(int row, int c16) {
 // Online-softmax state and output accumulator of one warp for one (sequence, KV head).
 // Lane (g = lane/4, tig = lane%4) owns rows g (and g+8 with ROWS16) and output columns
 // 8j + 2tig, 8j + 2tig + 1 of every n-tile j.
-template <class C>
+//
+// Q (the A operand of S = Q.K^T) is kept either in registers (QSMEM = false) or in a
+// per-warp shared-memory tile of ROWS x D bf16 read by ldmatrix at every k-step
+// (QSMEM = true), which frees 16-32 registers per thread.  The shared tile stores row
+// r's 16-byte chunk c at r*(2D) + ((c ^ (r & 7)) << 4), so ldmatrix reads of 8 rows at
+// one chunk hit 8 different bank groups.
+template <class C, bool QSMEM = false>
 struct WarpAcc {
+  static constexpr int QROW_BYTES = C::D * 2;
+  static constexpr int Q_BYTES = C::ROWS * QROW_BYTES;  // shared Q tile per warp
   float o_lo[C::NT][2];
   float o_hi[C::NT][2];
   float m_lo, m_hi, l_lo, l_hi;
-  uint32_t qa[C::KSTEPS][2];  // Q rows g as A fragments (k-step columns 2tig.., 8+2tig..)
-  uint32_t qh[C::KSTEPS][2];  // Q rows g+8
+  uint32_t qa[QSMEM ? 1 : C::KSTEPS][2];  // Q rows g as A fragments (register mode)
+  uint32_t qh[QSMEM ? 1 : C::KSTEPS][2];  // Q rows g+8
+  uint32_t qs = 0;                         // shared address of the Q tile (shared mode)
+
+  __device__ __forceinline__ static uint32_t q_off(int r, int c16) {
+    return static_cast<uint32_t>(r * QROW_BYTES + ((c16 ^ (r & 7)) << 4));
+  }
+
+  // Shared mode: copy the group's Q rows (G heads, [G][D] bf16) into the warp's tile at
+  // shared address `tile` (generic pointer `tile_ptr`); rows >= G are zero.
+  __device__ __forceinline__ void stage_q(const __nv_bfloat16* qrow, int G, uint8_t* tile_ptr,
+                                          int lane) {
+    constexpr int CPR = QROW_BYTES / 16;  // 16-byte chunks per row
+    __syncwarp();  // the previous unit's ldmatrix reads of this tile are done
+    for (int i = lane; i < C::ROWS * CPR; i += 32) {
+      const int r = i / CPR, c = i - r * CPR;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (r < G) v = __ldg(reinterpret_cast<const uint4*>(qrow + r * C::D) + c);
+      *reinterpret_cast<uint4*>(tile_ptr + q_off(r, c)) = v;
+    }
+    qs = smem_addr(tile_ptr);
+    __syncwarp();
+  }
+
+  // A fragments of k-step k: registers, or ldmatrix from the shared tile.
+  __device__ __forceinline__ void q_frag(int k, int lane, uint32_t& a0, uint32_t& a1,
+                                         uint32_t& a2, uint32_t& a3) const {
+    if constexpr (QSMEM) {
+      const int mi = lane >> 3, mr = lane & 7;
+      if constexpr (C::ROWS16) {
+        // matrices: (rows 0-7, chunk 2k), (rows 8-15, 2k), (rows 0-7, 2k+1), (rows 8-15, 2k+1)
+        ldmatrix_x4(qs + q_off((mi & 1) * 8 + mr, 2 * k + (mi >> 1)), a0, a1, a2, a3);
+      } else {
+        // lanes 0-7: rows 0-7 at chunk 2k; lanes 8-15: rows 0-7 at chunk 2k+1
+        ldmatrix_x2(qs + q_off(mr, 2 * k + (mi & 1)), a0, a2);
+        a1 = 0u;
+        a3 = 0u;
+      }
+    } else {
+      a0 = qa[k][0];
+      a1 = qh[k][0];
+      a2 = qa[k][1];
+      a3 = qh[k][1];
+    }
+  }
 
   __device__ __forceinline__ void reset() {
 #pragma unroll
@@ -115,10 +166,12 @@ struct WarpAcc {
         uint32_t b00, b01, b10, b11;
         ldmatrix_x4(kbase + (d >> 6) * C::CHUNK_BYTES + sw128(row, (d & 63) >> 3), b00, b01, b10,
                     b11);
-        mma_bf16_16816(s0[0], s0[1], s0[2], s0[3], qa[k][0], qh[k][0], qa[k][1], qh[k][1], b00,
-                       b01, s0[0], s0[1], s0[2], s0[3]);
-        mma_bf16_16816(s1[0], s1[1], s1[2], s1[3], qa[k][0], qh[k][0], qa[k][1], qh[k][1], b10,
-                       b11, s1[0], s1[1], s1[2], s1[3]);
+        uint32_t a0, a1, a2, a3;
+        q_frag(k, lane, a0, a1, a2, a3);
+        mma_bf16_16816(s0[0], s0[1], s0[2], s0[3], a0, a1, a2, a3, b00, b01, s0[0], s0[1], s0[2],
+                       s0[3]);
+        mma_bf16_16816(s1[0], s1[1], s1[2], s1[3], a0, a1, a2, a3, b10, b11, s1[0], s1[1], s1[2],
+                       s1[3]);
       }
       const int lim = valid - r0;
       const bool v0 = 2 * tig < lim, v1 = 2 * tig + 1 < lim;
