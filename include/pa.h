@@ -78,7 +78,8 @@ typedef enum pa_status {
   PA_ERR_EXISTS = 7,         /* allocator: sequence id already in use */
   PA_ERR_BAD_SEQ_LEN = 8,    /* device flag: seq_lens[b] outside [0, max_blocks*block_size] */
   PA_ERR_BAD_SLOT = 9,       /* device flag: slot >= num_blocks*block_size */
-  PA_ERR_TIMEOUT = 10        /* device flag: a bounded pipeline wait gave up */
+  PA_ERR_TIMEOUT = 10,       /* device flag: a bounded pipeline wait gave up */
+  PA_ERR_SCRATCH_LIMIT = 11  /* pa_decode_no_alloc: the shape needs more than its static scratch */
 } pa_status;
 
 typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
@@ -168,6 +169,34 @@ pa_status pa_decode_ex(void* out, const void* q, const void* k_pool, const void*
                        int Hkv, int D, int block_size, int max_blocks, int num_blocks,
                        float scale, pa_dtype dtype, void* workspace, size_t workspace_bytes,
                        int32_t* dev_err_flag, pa_stream_t stream, const pa_decode_opts* opts);
+
+/* Decode without any device allocation.  The source pages have no counterpart: this
+ * entry point exists for callers that cannot allocate device memory, so cannot provide
+ * pa_decode's workspace: e.g. a serving runtime that owns every device buffer through
+ * its own pool and forbids further allocations, or a latency-critical caller that
+ * cannot afford cudaMalloc (which may synchronise the device).
+ *
+ * Same arguments and result as pa_decode, minus the workspace.  Runs the balanced
+ * tensor-core kernel with its scratch in a static device array of the library
+ * (PA_NO_ALLOC_SCRATCH_BYTES per device that loads the library, held until exit); it
+ * calls no cudaMalloc, cudaFree or allocating library routine.
+ *   - The first call on each device looks up the array's address (cudaGetSymbolAddress
+ *     with that device current) and caches it: make that first call before any stream
+ *     capture.
+ *   - All calls on a device share the array, which keeps the last call's contents;
+ *     nothing in it has to start at zero.  Calls whose kernels overlap on the GPU race
+ *     on the array: order them (e.g. one stream).
+ *   - PA_ERR_UNSUPPORTED for shapes the tensor-core path does not take (fp32, block
+ *     size 4, Hq/Hkv > 16, B > 8192); PA_ERR_SCRATCH_LIMIT, before anything is queued,
+ *     if the shape's one-wave schedule on this device needs more than
+ *     PA_NO_ALLOC_SCRATCH_BYTES (2 partial slots x G rows x (D+2) floats per consumer
+ *     warp of the wave). */
+#define PA_NO_ALLOC_SCRATCH_BYTES (32u << 20)
+pa_status pa_decode_no_alloc(void* out, const void* q, const void* k_pool, const void* v_pool,
+                             const int32_t* block_tables, const int32_t* seq_lens, int B, int Hq,
+                             int Hkv, int D, int block_size, int max_blocks, int num_blocks,
+                             float scale, pa_dtype dtype, int32_t* dev_err_flag,
+                             pa_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Cache maintenance

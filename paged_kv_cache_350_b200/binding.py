@@ -30,6 +30,7 @@ PA_ERR_EXISTS = 7
 PA_ERR_BAD_SEQ_LEN = 8
 PA_ERR_BAD_SLOT = 9
 PA_ERR_TIMEOUT = 10
+PA_ERR_SCRATCH_LIMIT = 11
 
 # pa_dtype
 PA_F32 = 0
@@ -92,6 +93,8 @@ def _load():
                                i32, vp, sz, vp, vp, ctypes.POINTER(pa_decode_opts)]),
         "pa_decode_plan": (i32, [i32, i32, i32, i32, i32, i32, i32, sz,
                                  ctypes.POINTER(pa_decode_opts), ctypes.POINTER(pa_decode_plan_info)]),
+        "pa_decode_no_alloc": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                     f32, i32, vp, vp]),
         "pa_reshape_and_cache": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]),
         "pa_copy_blocks": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]),
         "pa_alloc_create": (i32, [i32, i32, ctypes.c_uint64, ctypes.POINTER(vp)]),
@@ -122,7 +125,7 @@ lib = _load()
 #: every symbol include/pa.h declares
 EXPORTED = (
     "pa_status_string", "pa_status_from_device_flag", "pa_version", "pa_decode_workspace_size",
-    "pa_decode", "pa_decode_ex", "pa_decode_plan", "pa_reshape_and_cache", "pa_copy_blocks", "pa_alloc_create",
+    "pa_decode", "pa_decode_ex", "pa_decode_plan", "pa_decode_no_alloc", "pa_reshape_and_cache", "pa_copy_blocks", "pa_alloc_create",
     "pa_alloc_create_ordered", "pa_alloc_destroy", "pa_alloc_add_seq", "pa_alloc_fork",
     "pa_alloc_append_slot", "pa_alloc_append_slots", "pa_alloc_free_seq", "pa_alloc_block_table",
     "pa_alloc_block_tables", "pa_alloc_refcount", "pa_alloc_num_free",
@@ -204,6 +207,31 @@ def pa_decode(out, q, k_pool, v_pool, block_tables, seq_lens, scale, workspace=N
                           float(scale), _dtype_of(q), _ptr(workspace), wbytes, _ptr(err_flag),
                           _stream(stream), ctypes.byref(opts))
     _check(st, "pa_decode")
+    return out
+
+
+def pa_decode_no_alloc(out, q, k_pool, v_pool, block_tables, seq_lens, scale, err_flag=None,
+                       stream=None):
+    """pa_decode without a workspace, for callers that cannot allocate device memory.
+
+    The library's static device scratch (PA_NO_ALLOC_SCRATCH_BYTES per device) stands in
+    for the workspace; calls that overlap on the GPU race on it (see include/pa.h)."""
+    import torch
+    _need(q.dim() == 3 and out.shape == q.shape, "q/out must be [B, Hq, D]")
+    _need(k_pool.dim() == 4 and v_pool.shape == k_pool.shape, "pools must be [NB, bs, Hkv, D]")
+    _need(block_tables.dim() == 2 and block_tables.dtype == torch.int32, "block_tables int32 [B, MB]")
+    _need(seq_lens.dtype == torch.int32 and seq_lens.numel() == q.shape[0], "seq_lens int32 [B]")
+    for t in (out, q, k_pool, v_pool, block_tables, seq_lens):
+        _need(t.is_contiguous(), "tensors must be contiguous")
+    _need(q.dtype == out.dtype == k_pool.dtype == v_pool.dtype, "q, out and pools share a dtype")
+    B, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_pool.shape
+    _need(D2 == D and block_tables.shape[0] == B, "shape mismatch")
+    st = lib.pa_decode_no_alloc(_ptr(out), _ptr(q), _ptr(k_pool), _ptr(v_pool),
+                                _ptr(block_tables), _ptr(seq_lens), B, Hq, Hkv, D, bs,
+                                block_tables.shape[1], NB, float(scale), _dtype_of(q),
+                                _ptr(err_flag), _stream(stream))
+    _check(st, "pa_decode_no_alloc")
     return out
 
 

@@ -61,6 +61,7 @@ const char* pa_status_string(pa_status s) {
     case PA_ERR_BAD_SEQ_LEN: return "sequence length outside [0, max_blocks*block_size]";
     case PA_ERR_BAD_SLOT: return "slot outside the pool";
     case PA_ERR_TIMEOUT: return "a bounded device wait expired";
+    case PA_ERR_SCRATCH_LIMIT: return "shape needs more scratch than the static no-alloc buffer";
   }
   return "unknown status";
 }
