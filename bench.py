@@ -451,7 +451,7 @@ def run_ours(args):
         "kernel_kv_gbs": achieved,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": recorded_traffic(args.config),
-                     "kernel": "pa_decode call (partition kernel + reduce), CUDA events per call",
+                     "kernel": "pa_decode call (main kernel + its reduce), CUDA events per call",
                      "peak_source": f"{peak_src} HBM copy bandwidth (burst)"},
         "cpu_baseline": cpu,
         "e2e": e2e,

@@ -7,15 +7,16 @@
 //   * Every (sequence b, KV head) is a unit of nt(b) = ceil(L_b / TILE_T) tiles; units
 //     are laid end to end in (b, KV head) order, T = Hkv * sum_b nt(b) tiles in all.
 //   * The grid is one wave of persistent CTAs (SM count x occupancy).  Each CTA has 4
-//     consumer warps and every consumer warp is one stream: stream s owns the global
-//     tiles [s*per, (s+1)*per), per = ceil(T / streams).  Work is balanced to one tile.
+//     warps and every warp is one stream: stream s owns the global tiles
+//     [s*per, (s+1)*per), per = ceil(T / streams).  Work is balanced to one tile.
 //   * Each CTA first computes the prefix sums of nt(b) in shared memory; a global tile
 //     index maps to (b, KV head, tile) by binary search.
-//   * Warp 4 produces for all four streams: it resolves the block ids of the next 32
-//     tiles with one coalesced table read per lane, and issues 4-D TMA loads into
-//     per-stream rings of SPW stages (mbarrier expect-tx), across unit boundaries, so
-//     the HBM stream never drains between units.
-//   * A consumer warp runs the tile math of tc_tile.cuh over its range.  A unit that
+//   * Each warp feeds itself: it resolves the block ids of its next 32 tiles with one
+//     table read per lane (the following 32 are read one batch ahead), keeps SPW 4-D
+//     TMA loads in flight in its own ring of stages (mbarrier expect-tx), and refills a
+//     stage as soon as it has consumed it, across unit boundaries, so its HBM stream
+//     never drains between units and no warp waits for another.
+//   * The warp runs the tile math of tc_tile.cuh over its range.  A unit that
 //     lies wholly inside the range is finished in place: normalised bf16 output.  A unit
 //     cut by a range boundary leaves a partial (max, sum, unnormalised O) in one of the
 //     stream's two slots; the reduce kernel merges the pieces of each cut unit by
@@ -39,10 +40,15 @@ namespace {
 #ifndef PA_STREAM_MIN_CTAS
 #define PA_STREAM_MIN_CTAS 3
 #endif
+// Launch the reduce as a programmatic dependent of the main kernel (its launch overlaps
+// the main kernel's tail; it waits for the main grid's completion before reading).
+#ifndef PA_STREAM_PDL
+#define PA_STREAM_PDL 1
+#endif
 
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kNCW = 4;                      // consumer warps (= streams) per CTA
-constexpr int kThreads = (kNCW + 1) * 32;
+constexpr int kNCW = 4;                      // warps (= streams) per CTA
+constexpr int kThreads = kNCW * 32;
 
 template <int D_, int BS_, bool ROWS16_, int SPW_>
 struct StreamCfg : TileCfg<D_, BS_, ROWS16_> {
@@ -95,6 +101,28 @@ __device__ __forceinline__ TilePos locate(const int* P, int B, int Hkv, int g) {
   return t;
 }
 
+// Block ids, KV head and block count of one tile, resolved by one lane.
+struct TileIds {
+  int kvh, id0, id1, nb;
+};
+
+template <class C>
+__device__ __forceinline__ TileIds resolve_tile(const DecodeParams& p, const int* P, int g,
+                                                int end) {
+  TileIds r{0, 0, 0, 0};
+  if (g >= end) return r;
+  const TilePos t = locate(P, p.B, p.Hkv, g);
+  r.kvh = t.kvh;
+  const int L = clamp_len(p, t.b, false);
+  const int nblk = (L + C::BS - 1) / C::BS;
+  const int blk = t.j * C::BPS;
+  r.nb = min(C::BPS, nblk - blk);
+  const int32_t* tab = p.block_tables + static_cast<size_t>(t.b) * p.max_blocks + blk;
+  r.id0 = __ldg(tab);
+  if (C::BPS > 1 && r.nb > 1) r.id1 = __ldg(tab + 1);
+  return r;
+}
+
 template <class C>
 __global__ void __launch_bounds__(kThreads, PA_STREAM_MIN_CTAS)
     decode_stream_kernel(const __grid_constant__ CUtensorMap tmk,
@@ -111,7 +139,6 @@ __global__ void __launch_bounds__(kThreads, PA_STREAM_MIN_CTAS)
   uint8_t* qtiles = smem + C::RING_BYTES;                  // [kNCW][Q_BYTES]
   int* P = reinterpret_cast<int*>(smem + C::FIXED_BYTES);  // [B + 1] tiles before sequence b
   __shared__ __align__(8) uint64_t full_bar[NST];
-  __shared__ __align__(8) uint64_t empty_bar[NST];
   __shared__ int warp_sum[kThreads / 32];
 
   // ---- prefix sums of per-sequence tile counts (every CTA, identical) --------------
@@ -151,10 +178,9 @@ __global__ void __launch_bounds__(kThreads, PA_STREAM_MIN_CTAS)
     }
   }
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NST; ++s) {
-      mbar_init(smem_addr(&full_bar[s]), 1);
-      mbar_init(smem_addr(&empty_bar[s]), 1);
-    }
+    prefetch_tensormap(&tmk);
+    prefetch_tensormap(&tmv);
+    for (int st = 0; st < NST; ++st) mbar_init(smem_addr(&full_bar[st]), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_proxy_async_smem();
   }
@@ -163,86 +189,62 @@ __global__ void __launch_bounds__(kThreads, PA_STREAM_MIN_CTAS)
   const int T = Hkv * P[B];
   const int S = static_cast<int>(gridDim.x) * kNCW;
   const int per = (T + S - 1) / S;
+#if PA_STREAM_PDL
+  // Let the reduce grid be launched now; it waits for this grid to complete.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#endif
 
-  if (warp == kNCW) {
-    // ---------------- producer warp: feeds the 4 streams of this CTA ----------------
-    if (lane == 0) {
-      prefetch_tensormap(&tmk);
-      prefetch_tensormap(&tmv);
-    }
-    const uint64_t policy = l2_policy_evict_first();
-    const int my_w = lane & 3;
-    const int my_s = static_cast<int>(blockIdx.x) * kNCW + my_w;
-    const int my_beg = min(T, my_s * per);
-    const int my_cnt = min(T, my_beg + per) - my_beg;
-    int rounds = my_cnt;
-    rounds = max(rounds, __shfl_xor_sync(kFull, rounds, 1));
-    rounds = max(rounds, __shfl_xor_sync(kFull, rounds, 2));
-    bool ok = true;
-    for (int r0 = 0; r0 < rounds && ok; r0 += 8) {
-      // lane l resolves round r0 + l/4 of stream l%4
-      const int rr = r0 + (lane >> 2);
-      const bool v = rr < my_cnt;
-      int kvh = 0, id0 = 0, id1 = 0, nb = 0;
-      if (v) {
-        const TilePos t = locate(P, B, Hkv, my_beg + rr);
-        kvh = t.kvh;
-        const int L = clamp_len(p, t.b, false);
-        const int nblk = (L + BS - 1) / BS;
-        const int blk = t.j * C::BPS;
-        nb = min(C::BPS, nblk - blk);
-        const int32_t* tab = p.block_tables + static_cast<size_t>(t.b) * p.max_blocks + blk;
-        id0 = __ldg(tab);
-        if (id0 < 0 || id0 >= p.num_blocks) {
-          flag_error(p.err, PA_DEVERR_BAD_BLOCK_ID);
-          id0 = 0;
-        }
-        if (C::BPS > 1 && nb > 1) {
-          id1 = __ldg(tab + 1);
-          if (id1 < 0 || id1 >= p.num_blocks) {
-            flag_error(p.err, PA_DEVERR_BAD_BLOCK_ID);
-            id1 = 0;
-          }
-        }
-      }
-      const unsigned vmask = __ballot_sync(kFull, v);
-      for (int l = 0; l < 32; ++l) {
-        const int kv = __shfl_sync(kFull, kvh, l);
-        const int i0 = __shfl_sync(kFull, id0, l);
-        const int i1 = __shfl_sync(kFull, id1, l);
-        const int n = __shfl_sync(kFull, nb, l);
-        if (lane == 0 && ok && ((vmask >> l) & 1u)) {
-          const int w = l & 3;
-          const int r = r0 + (l >> 2);
-          const int stage = w * SPW + r % SPW;
-          if (r >= SPW) ok = mbar_wait(smem_addr(&empty_bar[stage]), ((r / SPW) - 1) & 1, p.err);
-          if (ok) {
-            const uint32_t fb = smem_addr(&full_bar[stage]);
-            mbar_arrive_expect_tx(fb, static_cast<uint32_t>(n * BS * D * 2 * 2));
-            const uint32_t kt = smem_addr(smem + stage * C::STAGE_BYTES);
-            const uint32_t vt = kt + C::TILE_BYTES;
-            for (int sub = 0; sub < n; ++sub) {
-              const int phys = sub == 0 ? i0 : i1;
-#pragma unroll
-              for (int c = 0; c < C::DCH; ++c) {
-                tma_load_4d(kt + c * C::CHUNK_BYTES + sub * BS * 128, &tmk, c * 64, kv, 0, phys,
-                            fb, policy);
-                tma_load_4d(vt + c * C::CHUNK_BYTES + sub * BS * 128, &tmv, c * 64, kv, 0, phys,
-                            fb, policy);
-              }
-            }
-          }
-        }
-      }
-      ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
-    }
-    return;
-  }
-
-  // ---------------- consumer warp = one stream ----------------
+  // ---------------- every warp is one stream and feeds itself ----------------
   const int s = static_cast<int>(blockIdx.x) * kNCW + warp;
   const int beg = min(T, s * per);
   const int end = min(T, beg + per);
+  const int cnt = end - beg;
+  const uint64_t policy = l2_policy_evict_first();
+
+  // Block ids of this stream's tiles, 32 at a time (lane j holds tile 32*batch + j);
+  // the next batch's table reads are issued one batch ahead.
+  TileIds cur = resolve_tile<C>(p, P, beg + lane, end);
+  TileIds nxt = resolve_tile<C>(p, P, beg + 32 + lane, end);
+  int batch = 0;
+  // Issue the TMA loads of this stream's tile k into its stage (warp-collective).
+  auto issue = [&](int k) {
+    if ((k >> 5) != batch) {
+      cur = nxt;
+      ++batch;
+      nxt = resolve_tile<C>(p, P, beg + 32 * (batch + 1) + lane, end);
+    }
+    const int src = k & 31;
+    const int kv = __shfl_sync(kFull, cur.kvh, src);
+    int i0 = __shfl_sync(kFull, cur.id0, src);
+    int i1 = __shfl_sync(kFull, cur.id1, src);
+    const int n = __shfl_sync(kFull, cur.nb, src);
+    if (lane == 0) {
+      if (i0 < 0 || i0 >= p.num_blocks || (n > 1 && (i1 < 0 || i1 >= p.num_blocks))) {
+        flag_error(p.err, PA_DEVERR_BAD_BLOCK_ID);
+        if (i0 < 0 || i0 >= p.num_blocks) i0 = 0;
+        if (i1 < 0 || i1 >= p.num_blocks) i1 = 0;
+      }
+      const int stage = warp * SPW + k % SPW;
+      const uint32_t fb = smem_addr(&full_bar[stage]);
+      const uint32_t kt = smem_addr(smem + stage * C::STAGE_BYTES);
+      const uint32_t vt = kt + C::TILE_BYTES;
+      fence_proxy_async_smem();  // this stage's earlier generic reads/writes come first
+      mbar_arrive_expect_tx(fb, static_cast<uint32_t>(n * BS * D * 2 * 2));
+      for (int sub = 0; sub < n; ++sub) {
+        const int phys = sub == 0 ? i0 : i1;
+#pragma unroll
+        for (int c = 0; c < C::DCH; ++c) {
+          tma_load_4d(kt + c * C::CHUNK_BYTES + sub * BS * 128, &tmk, c * 64, kv, 0, phys, fb,
+                      policy);
+          tma_load_4d(vt + c * C::CHUNK_BYTES + sub * BS * 128, &tmv, c * 64, kv, 0, phys, fb,
+                      policy);
+        }
+      }
+    }
+    __syncwarp();
+  };
+  for (int k = 0; k < SPW && k < cnt; ++k) issue(k);
+
   const int g = lane >> 2, tig = lane & 3;
   const float sl2 = p.scale_log2;
   int unit_a = -1, a_starts = 0, unit_b = -1;
@@ -273,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, PA_STREAM_MIN_CTAS)
       if (valid < TILE_T) zero_tail_rows<C>(st_ptr, valid, lane);
       acc.tile(smem_addr(st_ptr), valid, sl2, lane);
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_addr(&empty_bar[stage]));
+      if (i + SPW < cnt) issue(i + SPW);  // refill the stage just consumed
     }
     if (!ok) break;
     acc.reduce_l();
@@ -318,6 +320,14 @@ __global__ void __launch_bounds__(kThreads, PA_STREAM_MIN_CTAS)
     }
     gpos = pend;
   }
+  if (!ok) {
+    // A load never arrived: wait (bounded) for this stream's loads still in flight so no
+    // TMA write lands after the CTA has left, then report nothing for this stream.
+    for (int k = i; k < cnt && k < i + SPW; ++k) {
+      const int stage = warp * SPW + k % SPW;
+      mbar_wait(smem_addr(&full_bar[stage]), (k / SPW) & 1, p.err);
+    }
+  }
   if (lane == 0) {
     int4 m = make_int4(ok ? unit_a : -1, ok ? a_starts : 0, ok ? unit_b : -1, 0);
     *reinterpret_cast<int4*>(sp.meta + s * 4) = m;
@@ -328,8 +338,22 @@ __global__ void __launch_bounds__(kThreads, PA_STREAM_MIN_CTAS)
 // STARTS in stream s and continues into later streams: its piece is slot 1 of s (or
 // slot 0 when it spans the whole stream from its first tile); the other pieces are
 // slot 0 of the following streams, as long as their first piece is the same unit.
+//
+// 16 warps; each query-head row gets WPR = 16 / G warps that split its pieces
+// round-robin.  A warp loads its pieces' (max, sum) one per lane, so the weights cost
+// one memory round trip; then it streams the pieces' unnormalised outputs (each lane
+// D/32 consecutive columns, 8 pieces in flight) and leaves (max, sum, O) in shared
+// memory, where the row's warps are merged by log-sum-exp.
+constexpr int kReduceWarps = 16;
+constexpr int kReduceThreads = kReduceWarps * 32;
+
 template <int D>
-__global__ void __launch_bounds__(128) stream_reduce_kernel(const StreamParams sp) {
+__global__ void __launch_bounds__(kReduceThreads) stream_reduce_kernel(const StreamParams sp) {
+  constexpr int VPL = D / 32;  // output columns per lane (4 or 2)
+#if PA_STREAM_PDL
+  // Wait until the main kernel has completed and its writes are visible.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+#endif
   const DecodeParams& p = sp.d;
   const int s = blockIdx.x;
   const int4 m = *reinterpret_cast<const int4*>(sp.meta + static_cast<size_t>(s) * 4);
@@ -343,27 +367,96 @@ __global__ void __launch_bounds__(128) stream_reduce_kernel(const StreamParams s
   } else {
     return;
   }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ int s_n;
+  __shared__ float s_m[kReduceWarps], s_l[kReduceWarps];
+  __shared__ __align__(16) float s_o[kReduceWarps][D];
+  // Pieces are streams s .. s+n-1: find n with a warp-wide scan of the following streams.
+  if (warp == 0) {
+    int n = 1;
+    for (int base = s + 1;; base += 32) {
+      const int q = base + lane;
+      const bool same = q < sp.streams && sp.meta[static_cast<size_t>(q) * 4] == u;
+      const unsigned stop = __ballot_sync(kFull, !same);
+      if (stop) {
+        n += __ffs(stop) - 1;
+        break;
+      }
+      n += 32;
+    }
+    if (lane == 0) s_n = n;
+  }
+  __syncthreads();
+  const int n = s_n;
   const int G = p.G;
-  int last = s;  // last stream holding a piece of u
-  while (last + 1 < sp.streams && sp.meta[static_cast<size_t>(last + 1) * 4] == u) ++last;
-  const int b = u / p.Hkv, kvh = u - (u / p.Hkv) * p.Hkv;
+  const int wpr = kReduceWarps / G;  // warps per row (G <= 16)
+  const int r = warp / wpr, k = warp - r * wpr;
+  auto prow = [&](int i) -> size_t {  // pml/pacc row of piece i, head row r
+    return (static_cast<size_t>(s + i) * 2 + (i == 0 ? slot : 0)) * G + r;
+  };
+  if (r < G) {
+    // this warp's pieces: i = k, k + wpr, ...; count nk
+    const int nk = n > k ? (n - k + wpr - 1) / wpr : 0;
+    float M = -INFINITY;
+    for (int j = lane; j < nk; j += 32) M = fmaxf(M, sp.pml[prow(k + j * wpr) * 2]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
+    float lsum = 0.f;
+    float acc[VPL];
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) acc[v] = 0.f;
+    for (int c0 = 0; c0 < nk; c0 += 32) {
+      float w = 0.f;
+      if (c0 + lane < nk) {
+        const float2 ml = *reinterpret_cast<const float2*>(sp.pml + prow(k + (c0 + lane) * wpr) * 2);
+        w = exp2f(ml.x - M);
+        lsum += w * ml.y;
+      }
+      const int cnt = min(32, nk - c0);
+#pragma unroll 8
+      for (int j = 0; j < cnt; ++j) {
+        const float wj = __shfl_sync(kFull, w, j);
+        const float* src = sp.pacc + prow(k + (c0 + j) * wpr) * D + lane * VPL;
+        if constexpr (VPL == 4) {
+          const float4 a = *reinterpret_cast<const float4*>(src);
+          acc[0] += wj * a.x;
+          acc[1] += wj * a.y;
+          acc[2] += wj * a.z;
+          acc[3] += wj * a.w;
+        } else {
+          const float2 a = *reinterpret_cast<const float2*>(src);
+          acc[0] += wj * a.x;
+          acc[1] += wj * a.y;
+        }
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(kFull, lsum, off);
+    if (lane == 0) {
+      s_m[warp] = M;
+      s_l[warp] = lsum;
+    }
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) s_o[warp][lane * VPL + v] = acc[v];
+  }
+  __syncthreads();
+  const int b = u / p.Hkv, kvh = u - b * p.Hkv;
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
   const size_t head0 = static_cast<size_t>(b) * p.Hq + static_cast<size_t>(kvh) * G;
-  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-    const int r = idx / D, d = idx - r * D;
+  for (int idx = threadIdx.x; idx < G * (D / 2); idx += kReduceThreads) {
+    const int rr = idx / (D / 2), d = (idx - rr * (D / 2)) * 2;
     float M = -INFINITY;
-    for (int q = s; q <= last; ++q) {
-      const size_t row = (static_cast<size_t>(q) * 2 + (q == s ? slot : 0)) * G + r;
-      M = fmaxf(M, sp.pml[row * 2]);
+    for (int kk = 0; kk < wpr; ++kk) M = fmaxf(M, s_m[rr * wpr + kk]);
+    float lsum = 0.f, a0 = 0.f, a1 = 0.f;
+    for (int kk = 0; kk < wpr; ++kk) {
+      const int w = rr * wpr + kk;
+      const float sc = s_l[w] > 0.f ? exp2f(s_m[w] - M) : 0.f;  // warps with no piece
+      lsum += sc * s_l[w];
+      a0 += sc * s_o[w][d];
+      a1 += sc * s_o[w][d + 1];
     }
-    float lsum = 0.f, a = 0.f;
-    for (int q = s; q <= last; ++q) {
-      const size_t row = (static_cast<size_t>(q) * 2 + (q == s ? slot : 0)) * G + r;
-      const float w = exp2f(sp.pml[row * 2] - M);
-      lsum += w * sp.pml[row * 2 + 1];
-      a += w * sp.pacc[row * D + d];
-    }
-    out[(head0 + r) * D + d] = __float2bfloat16_rn(a / lsum);
+    const float inv = 1.f / lsum;
+    *reinterpret_cast<uint32_t*>(out + (head0 + rr) * D + d) = pack_bf16x2(a0 * inv, a1 * inv);
   }
 }
 
@@ -395,8 +488,22 @@ cudaError_t launch_stream_cfg(const StreamParams& sp, int grid, cudaStream_t str
   decode_stream_kernel<C><<<grid, kThreads, smem, stream>>>(tmk, tmv, sp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  stream_reduce_kernel<C::D><<<sp.streams, 128, 0, stream>>>(sp);
+#if PA_STREAM_PDL
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(sp.streams));
+  cfg.blockDim = dim3(kReduceThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, stream_reduce_kernel<C::D>, sp);
+#else
+  stream_reduce_kernel<C::D><<<sp.streams, kReduceThreads, 0, stream>>>(sp);
   return cudaGetLastError();
+#endif
 }
 
 constexpr int kSPW = PA_STREAM_SPW;
