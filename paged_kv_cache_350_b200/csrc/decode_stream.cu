@@ -339,17 +339,12 @@ __global__ void __launch_bounds__(kThreads, PA_STREAM_MIN_CTAS)
 // slot 0 when it spans the whole stream from its first tile); the other pieces are
 // slot 0 of the following streams, as long as their first piece is the same unit.
 //
-// 16 warps; each query-head row gets WPR = 16 / G warps that split its pieces
-// round-robin.  A warp loads its pieces' (max, sum) one per lane, so the weights cost
-// one memory round trip; then it streams the pieces' unnormalised outputs (each lane
-// D/32 consecutive columns, 8 pieces in flight) and leaves (max, sum, O) in shared
-// memory, where the row's warps are merged by log-sum-exp.
-constexpr int kReduceWarps = 16;
-constexpr int kReduceThreads = kReduceWarps * 32;
-
+// One thread per (query-head row, 4 output columns) of the owned unit: G * D/4 threads,
+// rounded up to whole warps.
+// Each thread merges the pieces online (running max, sum, output; base 2) with the
+// piece loop unrolled so their loads overlap; each warp counts the pieces itself.
 template <int D>
-__global__ void __launch_bounds__(kReduceThreads) stream_reduce_kernel(const StreamParams sp) {
-  constexpr int VPL = D / 32;  // output columns per lane (4 or 2)
+__global__ void __launch_bounds__(512) stream_reduce_kernel(const StreamParams sp) {
 #if PA_STREAM_PDL
   // Wait until the main kernel has completed and its writes are visible.
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -367,97 +362,51 @@ __global__ void __launch_bounds__(kReduceThreads) stream_reduce_kernel(const Str
   } else {
     return;
   }
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  __shared__ int s_n;
-  __shared__ float s_m[kReduceWarps], s_l[kReduceWarps];
-  __shared__ __align__(16) float s_o[kReduceWarps][D];
+  const int lane = threadIdx.x & 31;
   // Pieces are streams s .. s+n-1: find n with a warp-wide scan of the following streams.
-  if (warp == 0) {
-    int n = 1;
-    for (int base = s + 1;; base += 32) {
-      const int q = base + lane;
-      const bool same = q < sp.streams && sp.meta[static_cast<size_t>(q) * 4] == u;
-      const unsigned stop = __ballot_sync(kFull, !same);
-      if (stop) {
-        n += __ffs(stop) - 1;
-        break;
-      }
-      n += 32;
+  int n = 1;
+  for (int base = s + 1;; base += 32) {
+    const int q = base + lane;
+    const bool same = q < sp.streams && sp.meta[static_cast<size_t>(q) * 4] == u;
+    const unsigned stop = __ballot_sync(kFull, !same);
+    if (stop) {
+      n += __ffs(stop) - 1;
+      break;
     }
-    if (lane == 0) s_n = n;
+    n += 32;
   }
-  __syncthreads();
-  const int n = s_n;
   const int G = p.G;
-  const int wpr = kReduceWarps / G;  // warps per row (G <= 16)
-  const int r = warp / wpr, k = warp - r * wpr;
-  auto prow = [&](int i) -> size_t {  // pml/pacc row of piece i, head row r
-    return (static_cast<size_t>(s + i) * 2 + (i == 0 ? slot : 0)) * G + r;
-  };
-  if (r < G) {
-    // this warp's pieces: i = k, k + wpr, ...; count nk
-    const int nk = n > k ? (n - k + wpr - 1) / wpr : 0;
-    float M = -INFINITY;
-    for (int j = lane; j < nk; j += 32) M = fmaxf(M, sp.pml[prow(k + j * wpr) * 2]);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
-    float lsum = 0.f;
-    float acc[VPL];
-#pragma unroll
-    for (int v = 0; v < VPL; ++v) acc[v] = 0.f;
-    for (int c0 = 0; c0 < nk; c0 += 32) {
-      float w = 0.f;
-      if (c0 + lane < nk) {
-        const float2 ml = *reinterpret_cast<const float2*>(sp.pml + prow(k + (c0 + lane) * wpr) * 2);
-        w = exp2f(ml.x - M);
-        lsum += w * ml.y;
-      }
-      const int cnt = min(32, nk - c0);
-#pragma unroll 8
-      for (int j = 0; j < cnt; ++j) {
-        const float wj = __shfl_sync(kFull, w, j);
-        const float* src = sp.pacc + prow(k + (c0 + j) * wpr) * D + lane * VPL;
-        if constexpr (VPL == 4) {
-          const float4 a = *reinterpret_cast<const float4*>(src);
-          acc[0] += wj * a.x;
-          acc[1] += wj * a.y;
-          acc[2] += wj * a.z;
-          acc[3] += wj * a.w;
-        } else {
-          const float2 a = *reinterpret_cast<const float2*>(src);
-          acc[0] += wj * a.x;
-          acc[1] += wj * a.y;
-        }
-      }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(kFull, lsum, off);
-    if (lane == 0) {
-      s_m[warp] = M;
-      s_l[warp] = lsum;
-    }
-#pragma unroll
-    for (int v = 0; v < VPL; ++v) s_o[warp][lane * VPL + v] = acc[v];
+  const int r = threadIdx.x / (D / 4);
+  const int c = (threadIdx.x % (D / 4)) * 4;
+  if (r >= G) return;
+  float M = -INFINITY, l = 0.f, a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 4
+  for (int i = 0; i < n; ++i) {
+    const size_t row = (static_cast<size_t>(s + i) * 2 + (i == 0 ? slot : 0)) * G + r;
+    const float2 ml = *reinterpret_cast<const float2*>(sp.pml + row * 2);
+    const float4 a = *reinterpret_cast<const float4*>(sp.pacc + row * D + c);
+    const float Mn = fmaxf(M, ml.x);
+    const float so = exp2f(M - Mn), sn = exp2f(ml.x - Mn);
+    l = l * so + ml.y * sn;
+    a0 = a0 * so + a.x * sn;
+    a1 = a1 * so + a.y * sn;
+    a2 = a2 * so + a.z * sn;
+    a3 = a3 * so + a.w * sn;
+    M = Mn;
   }
-  __syncthreads();
   const int b = u / p.Hkv, kvh = u - b * p.Hkv;
-  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-  const size_t head0 = static_cast<size_t>(b) * p.Hq + static_cast<size_t>(kvh) * G;
-  for (int idx = threadIdx.x; idx < G * (D / 2); idx += kReduceThreads) {
-    const int rr = idx / (D / 2), d = (idx - rr * (D / 2)) * 2;
-    float M = -INFINITY;
-    for (int kk = 0; kk < wpr; ++kk) M = fmaxf(M, s_m[rr * wpr + kk]);
-    float lsum = 0.f, a0 = 0.f, a1 = 0.f;
-    for (int kk = 0; kk < wpr; ++kk) {
-      const int w = rr * wpr + kk;
-      const float sc = s_l[w] > 0.f ? exp2f(s_m[w] - M) : 0.f;  // warps with no piece
-      lsum += sc * s_l[w];
-      a0 += sc * s_o[w][d];
-      a1 += sc * s_o[w][d + 1];
-    }
-    const float inv = 1.f / lsum;
-    *reinterpret_cast<uint32_t*>(out + (head0 + rr) * D + d) = pack_bf16x2(a0 * inv, a1 * inv);
-  }
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) +
+                       (static_cast<size_t>(b) * p.Hq + static_cast<size_t>(kvh) * G + r) * D + c;
+  const float inv = 1.f / l;
+  *reinterpret_cast<uint2*>(out) = make_uint2(pack_bf16x2(a0 * inv, a1 * inv),
+                                              pack_bf16x2(a2 * inv, a3 * inv));
+}
+
+// Threads of a reduce block: G * D/4, rounded up to whole warps (the piece count is
+// found with full-warp ballots).
+template <int D>
+int reduce_threads(int G) {
+  return ((G * D / 4 + 31) / 32) * 32;
 }
 
 template <class C>
@@ -491,7 +440,7 @@ cudaError_t launch_stream_cfg(const StreamParams& sp, int grid, cudaStream_t str
 #if PA_STREAM_PDL
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(sp.streams));
-  cfg.blockDim = dim3(kReduceThreads);
+  cfg.blockDim = dim3(static_cast<unsigned>(reduce_threads<C::D>(sp.d.G)));
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -501,7 +450,7 @@ cudaError_t launch_stream_cfg(const StreamParams& sp, int grid, cudaStream_t str
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, stream_reduce_kernel<C::D>, sp);
 #else
-  stream_reduce_kernel<C::D><<<sp.streams, kReduceThreads, 0, stream>>>(sp);
+  stream_reduce_kernel<C::D><<<sp.streams, reduce_threads<C::D>(sp.d.G), 0, stream>>>(sp);
   return cudaGetLastError();
 #endif
 }
