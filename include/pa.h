@@ -260,6 +260,11 @@ pa_status pa_alloc_block_table(const pa_allocator* a, int64_t seq_id, int32_t* o
 /* Fill block_tables[n][max_blocks] (padded with -1) and seq_lens[n] for n sequences. */
 pa_status pa_alloc_block_tables(const pa_allocator* a, const int64_t* seq_ids, int n,
                                 int32_t* block_tables, int max_blocks, int32_t* seq_lens);
+/* Slots of all tokens of a sequence, token t at
+ * table[t / block_size] * block_size + t % block_size (up to cap); *n = its token count.
+ * Used to write a prompt's K/V (prefill) with pa_reshape_and_cache. */
+pa_status pa_alloc_seq_slots(const pa_allocator* a, int64_t seq_id, int64_t* slots, int cap,
+                             int* n);
 int pa_alloc_refcount(const pa_allocator* a, int32_t block);   /* -1 if out of range */
 int pa_alloc_num_free(const pa_allocator* a);
 /* Sum over live sequences of (blocks * block_size - tokens). */

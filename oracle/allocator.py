@@ -99,6 +99,11 @@ class RefAllocator:
     def block_table(self, seq_id):
         return list(self.tables[seq_id]), self.ntok[seq_id]
 
+    def seq_slots(self, seq_id):
+        """Slot of every token: token t sits in block table[t // bs] at offset t % bs."""
+        table, n = self.tables[seq_id], self.ntok[seq_id]
+        return [table[t // self.block_size] * self.block_size + t % self.block_size for t in range(n)]
+
     def internal_waste_slots(self):
         return sum(len(t) * self.block_size - self.ntok[s] for s, t in self.tables.items())
 

@@ -107,6 +107,7 @@ def _load():
         "pa_alloc_free_seq": (i32, [vp, i64]),
         "pa_alloc_block_table": (i32, [vp, i64, pi32, i32, pint, pint]),
         "pa_alloc_block_tables": (i32, [vp, pi64, i32, pi32, i32, pi32]),
+        "pa_alloc_seq_slots": (i32, [vp, i64, pi64, i32, pint]),
         "pa_alloc_refcount": (i32, [vp, ctypes.c_int32]),
         "pa_alloc_num_free": (i32, [vp]),
         "pa_alloc_internal_waste_slots": (i64, [vp]),
@@ -128,7 +129,7 @@ EXPORTED = (
     "pa_decode", "pa_decode_ex", "pa_decode_plan", "pa_decode_no_alloc", "pa_reshape_and_cache", "pa_copy_blocks", "pa_alloc_create",
     "pa_alloc_create_ordered", "pa_alloc_destroy", "pa_alloc_add_seq", "pa_alloc_fork",
     "pa_alloc_append_slot", "pa_alloc_append_slots", "pa_alloc_free_seq", "pa_alloc_block_table",
-    "pa_alloc_block_tables", "pa_alloc_refcount", "pa_alloc_num_free",
+    "pa_alloc_block_tables", "pa_alloc_seq_slots", "pa_alloc_refcount", "pa_alloc_num_free",
     "pa_alloc_internal_waste_slots", "pa_alloc_free_list",
 )
 
@@ -354,6 +355,15 @@ class Allocator:
         _check(lib.pa_alloc_block_tables(self._h, _i64p(ids), n, _i32p(tables), max_blocks,
                                          _i32p(lens)), "pa_alloc_block_tables")
         return tables, lens
+
+    def seq_slots(self, seq_id):
+        """Slots of all tokens of the sequence (int64 array)."""
+        n = ctypes.c_int()
+        _check(lib.pa_alloc_seq_slots(self._h, seq_id, None, 0, ctypes.byref(n)), "pa_alloc_seq_slots")
+        out = np.empty(max(n.value, 1), dtype=np.int64)
+        _check(lib.pa_alloc_seq_slots(self._h, seq_id, _i64p(out), n.value, ctypes.byref(n)),
+               "pa_alloc_seq_slots")
+        return out[: n.value]
 
     def refcount(self, block):
         return lib.pa_alloc_refcount(self._h, block)

@@ -13,6 +13,11 @@ in host memory:
 5. device→host copy of the output, then a stream synchronise.
 
 Everything between the copies runs in the library's kernels.
+
+``host_inputs`` + ``step_staged`` do the same with one host→device copy: the
+caller writes the step's q / new K / new V straight into the cache's pinned
+input buffer, the allocator writes slots, tables and lengths behind them, and a
+single copy moves the whole step input.
 """
 
 from __future__ import annotations
@@ -106,6 +111,108 @@ class PagedKVCache:
             out_host.copy_(out, non_blocking=True)
         stream.synchronize()
         return h2d, out_host.numel() * out_host.element_size()
+
+    # -- one decode step, single staged copy -----------------------------------------
+    def _layout(self, B, Hq, max_blocks):
+        """Byte offsets of the sections of the step input buffer (256-byte aligned)."""
+        esz = torch.tensor([], dtype=self.dtype).element_size()
+        sizes = [("q", B * Hq * self.D * esz), ("k", B * self.Hkv * self.D * esz),
+                 ("v", B * self.Hkv * self.D * esz), ("slots", B * 8),
+                 ("tables", B * max_blocks * 4), ("lens", B * 4), ("pairs", B * 8)]
+        off, lay = 0, {}
+        for name, n in sizes:
+            lay[name] = (off, n)
+            off += (n + 255) // 256 * 256
+        return lay, off
+
+    def host_inputs(self, B, Hq, max_blocks):
+        """Pinned host views (q [B,Hq,D], k [B,Hkv,D], v [B,Hkv,D]) for step_staged to read.
+
+        The buffers only grow, so a batch that changes size from step to step (sequences
+        admitted and retired) reuses them."""
+        lay, total = self._layout(B, Hq, max_blocks)
+        out_elems = B * Hq * self.D
+        if getattr(self, "_hbuf", None) is None or self._hbuf.numel() < total:
+            self._hbuf = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+            self._dbuf = torch.empty(total, dtype=torch.uint8, device=self.device)
+        if getattr(self, "_out_hbuf", None) is None or self._out_hbuf.numel() < out_elems:
+            self._out_hbuf = torch.empty(out_elems, dtype=self.dtype, pin_memory=True)
+            self._out_dbuf = torch.empty(out_elems, dtype=self.dtype, device=self.device)
+        self._stage_key, self._lay = (B, Hq, max_blocks), lay
+        self._out_h = self._out_hbuf[:out_elems].view(B, Hq, self.D)
+        self._out_d = self._out_dbuf[:out_elems].view(B, Hq, self.D)
+        return (self._view(self._hbuf, "q", (B, Hq, self.D), self.dtype),
+                self._view(self._hbuf, "k", (B, self.Hkv, self.D), self.dtype),
+                self._view(self._hbuf, "v", (B, self.Hkv, self.D), self.dtype))
+
+    def _view(self, buf, name, shape, dtype):
+        off, n = self._lay[name]
+        return buf[off:off + n].view(dtype).view(shape)
+
+    def step_staged(self, seq_ids, scale, max_blocks, stream=None):
+        """One decode step whose q / new K / new V the caller wrote into host_inputs().
+
+        Returns the pinned host output [B, Hq, D] (valid until the next call) and the
+        (h2d_bytes, d2h_bytes) moved.
+        """
+        stream = stream or torch.cuda.current_stream(self.device)
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        B = ids.size
+        Hq = self._stage_key[1]
+        assert self._stage_key == (B, Hq, max_blocks), "call host_inputs() with this shape first"
+        h = self._hbuf
+        slots_h = self._view(h, "slots", (B,), torch.int64).numpy()
+        pairs_h = self._view(h, "pairs", (B, 2), torch.int32).numpy()
+        tables_h = self._view(h, "tables", (B, max_blocks), torch.int32).numpy()
+        lens_h = self._view(h, "lens", (B,), torch.int32).numpy()
+        _, pairs = self.alloc.append_slots(ids, slot_out=slots_h, pairs_out=pairs_h)
+        self.alloc.block_tables(ids, max_blocks, tables_out=tables_h, lens_out=lens_h)
+        npairs = pairs.shape[0]
+        used = self._lay["pairs"][0] + npairs * 8 if npairs else self._lay["lens"][0] + B * 4
+        d = self._dbuf
+        with torch.cuda.stream(stream):
+            d[:used].copy_(h[:used], non_blocking=True)
+            kp, vp = self.k_pool, self.v_pool
+            if npairs:
+                _b.pa_copy_blocks(kp, vp, self._view(d, "pairs", (B, 2), torch.int32)[:npairs],
+                                  err_flag=self.err, stream=stream)
+            _b.pa_reshape_and_cache(self._view(d, "k", (B, self.Hkv, self.D), self.dtype),
+                                    self._view(d, "v", (B, self.Hkv, self.D), self.dtype),
+                                    kp, vp, self._view(d, "slots", (B,), torch.int64),
+                                    err_flag=self.err, stream=stream)
+            _b.pa_decode(self._out_d, self._view(d, "q", (B, Hq, self.D), self.dtype), kp, vp,
+                         self._view(d, "tables", (B, max_blocks), torch.int32),
+                         self._view(d, "lens", (B,), torch.int32), scale,
+                         workspace=self.workspace(B, Hq, max_blocks), err_flag=self.err,
+                         stream=stream)
+            self._out_h.copy_(self._out_d, non_blocking=True)
+        stream.synchronize()
+        return self._out_h, (used, self._out_h.numel() * self._out_h.element_size())
+
+    # -- sequence management ------------------------------------------------------------
+    def admit(self, seq_id, k_host, v_host, stream=None):
+        """Register a sequence and write its prompt's K/V ([n, Hkv, D] host) into its blocks."""
+        stream = stream or torch.cuda.current_stream(self.device)
+        n = k_host.shape[0]
+        self.alloc.add_seq(seq_id, n)
+        if n == 0:
+            return
+        slots = torch.from_numpy(self.alloc.seq_slots(seq_id))
+        with torch.cuda.stream(stream):
+            k = k_host.to(self.device, non_blocking=True)
+            v = v_host.to(self.device, non_blocking=True)
+            sl = slots.to(self.device, non_blocking=True)
+            _b.pa_reshape_and_cache(k, v, self.k_pool, self.v_pool, sl, err_flag=self.err,
+                                    stream=stream)
+        stream.synchronize()  # the host tensors above must outlive the copies
+
+    def fork(self, parent_id, child_id):
+        """The child shares every block of the parent (copy on write at its first append)."""
+        self.alloc.fork(parent_id, child_id)
+
+    def retire(self, seq_id):
+        """Free the sequence; blocks no other sequence holds return to the pool."""
+        self.alloc.free_seq(seq_id)
 
     def check_device_errors(self):
         flag = int(self.err.item())

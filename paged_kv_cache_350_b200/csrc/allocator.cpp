@@ -257,6 +257,21 @@ pa_status pa_alloc_block_tables(const pa_allocator* a, const int64_t* seq_ids, i
   return PA_OK;
 }
 
+pa_status pa_alloc_seq_slots(const pa_allocator* a, int64_t seq_id, int64_t* slots, int cap,
+                             int* n) {
+  if (!a || !n || cap < 0 || (cap > 0 && !slots)) return PA_ERR_INVALID_ARG;
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
+  const Seq& s = it->second;
+  const int bs = a->block_size;
+  const int ntok = static_cast<int>(s.ntok);
+  const int m = std::min(ntok, cap);
+  for (int t = 0; t < m; ++t)
+    slots[t] = static_cast<int64_t>(s.table[t / bs]) * bs + t % bs;
+  *n = ntok;
+  return PA_OK;
+}
+
 int pa_alloc_refcount(const pa_allocator* a, int32_t block) {
   if (!a || block < 0 || block >= a->num_blocks) return -1;
   return a->ref[block];

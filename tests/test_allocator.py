@@ -14,14 +14,14 @@ def _alloc(*a, **k):
 
 
 def state(a, seqs, nb):
-    tables = {s: a.block_table(s) for s in sorted(seqs)}
+    tables = {s: (a.block_table(s), [int(x) for x in a.seq_slots(s)]) for s in sorted(seqs)}
     refs = [a.refcount(b) for b in range(nb)]
     free = a.free_list() if hasattr(a, "free_list") else None
     return tables, refs, free, a.num_free(), a.internal_waste_slots()
 
 
 def ref_state(r, seqs, nb):
-    tables = {s: r.block_table(s) for s in sorted(seqs)}
+    tables = {s: (r.block_table(s), r.seq_slots(s)) for s in sorted(seqs)}
     return tables, [r.refcount(b) for b in range(nb)], list(r.free), r.num_free(), \
         r.internal_waste_slots()
 

@@ -1,0 +1,119 @@
+"""Multi-step decode with continuous batching: admissions (prefill of the prompt K/V),
+forks for parallel sampling (copy on write at the first divergent token), retirements
+(blocks back to the pool at refcount 0), and one decode step per live sequence per step.
+
+The product side runs PagedKVCache (C allocator + kernels); the oracle side replays the
+same trace with RefAllocator and the float64 functions.  Every step's slots, copy pairs,
+tables and lengths must be identical, every step's outputs within tolerance, and the
+pools bit-identical at the end."""
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from _parity import assert_close
+from oracle import RefAllocator, ref_copy_blocks, ref_decode, ref_reshape_and_cache
+
+
+def _oracle_replay(tr):
+    alloc = RefAllocator(tr.num_blocks, tr.block_size, shuffle_seed=tr.alloc_seed)
+    kp, vp = tr.pool("k"), tr.pool("v")
+    live, outs, plans = [], [], []
+    for t, ev in enumerate(tr.events):
+        for e in ev:
+            if e[0] == "admit":
+                alloc.add_seq(e[1], e[2])
+                pk, pv = tr.prompt_kv(e[1], e[2])
+                kp, vp = ref_reshape_and_cache(pk, pv, kp, vp, np.array(alloc.seq_slots(e[1])))
+                live.append(e[1])
+            elif e[0] == "fork":
+                alloc.fork(e[1], e[2])
+                live.append(e[2])
+            else:
+                alloc.free_seq(e[1])
+                live.remove(e[1])
+        ids = sorted(live)
+        q, nk, nv = tr.step_inputs(t, len(ids))
+        slots, pairs = [], []
+        for sid in ids:
+            slot, src, dst = alloc.append_slot(sid)
+            slots.append(slot)
+            if src >= 0:
+                pairs.append((src, dst))
+        kp, vp = ref_copy_blocks(kp, vp, pairs)
+        kp, vp = ref_reshape_and_cache(nk, nv, kp, vp, np.array(slots))
+        tables = np.full((len(ids), tr.max_blocks), -1, dtype=np.int32)
+        lens = np.zeros(len(ids), dtype=np.int32)
+        for i, sid in enumerate(ids):
+            tab, n = alloc.block_table(sid)
+            tables[i, :len(tab)] = tab
+            lens[i] = n
+        outs.append(ref_decode(q, kp, vp, tables, lens, tr.scale))
+        plans.append((np.array(slots), np.array(pairs, dtype=np.int32).reshape(-1, 2), tables, lens))
+    return outs, plans, kp, vp, alloc
+
+
+def test_trace_replay_keeps_allocator_invariants():
+    tr = workloads.serving_trace(seed=3101, steps=30)
+    _, _, _, _, alloc = _oracle_replay(tr)
+    used = {}
+    for sid, tab in alloc.tables.items():
+        for b in tab:
+            used[b] = used.get(b, 0) + 1
+    for b in range(tr.num_blocks):
+        assert alloc.refcount(b) == used.get(b, 0)
+    assert alloc.num_free() + len(used) == tr.num_blocks
+    assert any(e[0] == "fork" for ev in tr.events for e in ev)
+    assert any(e[0] == "retire" for ev in tr.events for e in ev)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("seed,bs,G", [(3201, 16, 8), (3202, 8, 4), (3203, 32, 2)])
+def test_serving_trace_matches_oracle_replay(seed, bs, G):
+    import paged_kv_cache_350_b200 as pa
+    tr = workloads.serving_trace(seed=seed, steps=36, bs=bs, Hq=2 * G, Hkv=2)
+    outs, plans, ref_kp, ref_vp, ref_alloc = _oracle_replay(tr)
+
+    def dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+
+    def host(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+    cache = pa.PagedKVCache(tr.num_blocks, tr.block_size, tr.Hkv, tr.D, shuffle_seed=tr.alloc_seed,
+                            k_pool=dev(tr.pool("k")), v_pool=dev(tr.pool("v")))
+    live = []
+    for t, ev in enumerate(tr.events):
+        for e in ev:
+            if e[0] == "admit":
+                pk, pv = tr.prompt_kv(e[1], e[2])
+                cache.admit(e[1], host(pk), host(pv))
+                live.append(e[1])
+            elif e[0] == "fork":
+                cache.fork(e[1], e[2])
+                live.append(e[2])
+            else:
+                cache.retire(e[1])
+                live.remove(e[1])
+        ids = sorted(live)
+        q, nk, nv = tr.step_inputs(t, len(ids))
+        qh, kh, vh = cache.host_inputs(len(ids), tr.Hq, tr.max_blocks)
+        qh.copy_(host(q))
+        kh.copy_(host(nk))
+        vh.copy_(host(nv))
+        out, _ = cache.step_staged(ids, tr.scale, tr.max_blocks)
+        slots, pairs, tables, lens = plans[t]
+        lay = cache._lay
+        got_slots = cache._view(cache._hbuf, "slots", (len(ids),), torch.int64).numpy()
+        got_tables = cache._view(cache._hbuf, "tables", (len(ids), tr.max_blocks), torch.int32).numpy()
+        got_lens = cache._view(cache._hbuf, "lens", (len(ids),), torch.int32).numpy()
+        assert np.array_equal(got_slots, slots) and np.array_equal(got_tables, tables)
+        assert np.array_equal(got_lens, lens)
+        w = workloads.independent([1], dtype="bf16")
+        assert_close(w, out.clone(), outs[t])
+    cache.check_device_errors()
+    kd = cache.k_pool.view(torch.int16).cpu().numpy().view(np.uint16)
+    vd = cache.v_pool.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(kd, ref_kp) and np.array_equal(vd, ref_vp)
+    assert cache.alloc.free_list() == list(ref_alloc.free)

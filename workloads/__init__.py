@@ -309,3 +309,83 @@ def run_step_allocation(w, alloc):
         tables[i, : len(table)] = table
         lens[i] = ntok
     return slots, np.asarray(pairs, dtype=np.int32).reshape(-1, 2), tables, lens
+
+
+# ---- a multi-step serving trace (continuous batching) -----------------------------
+
+@dataclass
+class ServingTrace:
+    """Per-step events of a serving loop; every live sequence decodes one token per step.
+
+    ``events[t]`` lists ("admit", seq_id, prompt_len), ("fork", parent, child) and
+    ("retire", seq_id) applied before step t's decode.  The prompt K/V of an admission
+    and every step's q / new K / new V are drawn with ``draw_normal`` from ``seed`` and
+    the stream numbers ``prompt_stream`` / ``step_stream`` give.
+    """
+    seed: int
+    dtype: str
+    Hq: int
+    Hkv: int
+    D: int
+    block_size: int
+    num_blocks: int
+    scale: float
+    alloc_seed: int
+    events: list
+    max_blocks: int
+
+    def prompt_kv(self, seq_id, n):
+        shape = (n, self.Hkv, self.D)
+        return (draw_normal(shape, self.seed, 100000 + 2 * seq_id, self.dtype),
+                draw_normal(shape, self.seed, 100001 + 2 * seq_id, self.dtype))
+
+    def step_inputs(self, t, B):
+        return (draw_normal((B, self.Hq, self.D), self.seed, 200000 + 3 * t, self.dtype),
+                draw_normal((B, self.Hkv, self.D), self.seed, 200001 + 3 * t, self.dtype),
+                draw_normal((B, self.Hkv, self.D), self.seed, 200002 + 3 * t, self.dtype))
+
+    def pool(self, which):
+        shape = (self.num_blocks, self.block_size, self.Hkv, self.D)
+        return draw_normal(shape, self.seed, 1 if which == "k" else 2, self.dtype)
+
+
+def serving_trace(seed=3000, steps=40, start=6, max_live=12, prompt_lo=1, prompt_hi=90,
+                  p_admit=0.25, p_retire=0.15, p_fork=0.2, Hq=16, Hkv=2, D=128, bs=16,
+                  dtype="bf16", num_blocks=None):
+    """Random admissions, forks (parallel sampling) and retirements over ``steps`` steps."""
+    rng = np.random.default_rng(seed)
+    live = []
+    next_id = 0
+    events = []
+    max_tokens = 0
+    tokens = {}
+    for t in range(steps):
+        ev = []
+        n_admit = start if t == 0 else int(rng.random() < p_admit)
+        for _ in range(n_admit):
+            if len(live) >= max_live:
+                break
+            n = int(rng.integers(prompt_lo, prompt_hi + 1))
+            ev.append(("admit", next_id, n))
+            live.append(next_id)
+            tokens[next_id] = n
+            next_id += 1
+        if live and len(live) < max_live and rng.random() < p_fork:
+            parent = int(rng.choice(live))
+            ev.append(("fork", parent, next_id))
+            live.append(next_id)
+            tokens[next_id] = tokens[parent]
+            next_id += 1
+        if len(live) > 1 and rng.random() < p_retire:
+            gone = int(rng.choice(live))
+            ev.append(("retire", gone))
+            live.remove(gone)
+        events.append(ev)
+        for sid in live:
+            tokens[sid] += 1
+            max_tokens = max(max_tokens, tokens[sid])
+    mb = _blocks(max_tokens, bs) + 1
+    nb = num_blocks or (max_live + 2) * mb * 2
+    return ServingTrace(seed=seed, dtype=dtype, Hq=Hq, Hkv=Hkv, D=D, block_size=bs,
+                        num_blocks=nb, scale=1.0 / math.sqrt(D), alloc_seed=seed + 1,
+                        events=events, max_blocks=mb)
