@@ -71,6 +71,8 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--block-size", type=int, default=0,
+                    help="override the workload's block size (8, 16 or 32) for a sweep")
     return ap.parse_args(argv)
 
 
@@ -318,7 +320,7 @@ def run_ours(args):
     barrier(dist, device)
     import paged_kv_cache_350_b200 as pa
 
-    w = workloads.build(args.config)
+    w = workloads.build(args.config, **({"bs": args.block_size} if args.block_size else {}))
     esize = 2 if w.dtype == "bf16" else 4
     dtype_pa = pa.PA_BF16 if w.dtype == "bf16" else pa.PA_F32
 
@@ -444,6 +446,7 @@ def run_ours(args):
             "num_blocks": w.num_blocks, "mean_seq_len": float(np.mean(lens)),
             "kv_bytes_per_step": kv_bytes, "alg_bytes_per_step": alg_bytes,
             "copy_pairs_per_step": npairs, "decode_plan": plan,
+            "internal_waste_slots": int(alloc.internal_waste_slots()),
             "l2": "inputs larger than L2 (K/V pools of %.2f GB vs 126 MB L2); not flushed"
                   % (2 * kp.numel() * esize / 1e9),
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",

@@ -253,6 +253,17 @@ pa_status pa_alloc_append_slots(pa_allocator* a, const int64_t* seq_ids, int n,
                                 int64_t* slot_mapping, int32_t* cow_pairs, int* n_pairs);
 /* Drop a sequence; blocks whose refcount reaches 0 return to the free list. */
 pa_status pa_alloc_free_seq(pa_allocator* a, int64_t seq_id);
+/* Keep only the first num_tokens tokens (0 <= num_tokens <= current count), e.g. to roll
+ * back rejected speculative tokens.  Blocks past ceil(num_tokens / block_size) are
+ * released in table order (refcount - 1; free at 0).  A now-partial shared last block is
+ * copied on write at the next append, as usual. */
+pa_status pa_alloc_truncate(pa_allocator* a, int64_t seq_id, int num_tokens);
+/* Beam-search step: beam i (seq_ids[i], n distinct live sequences) continues from beam
+ * parent_idx[i] (0 <= parent_idx[i] < n).  Every new beam first takes a shared reference
+ * to its parent's blocks and token count; then the beams' old tables are released, beam
+ * 0 first, each in table order (refcount - 1; free at 0).  Allocates nothing. */
+pa_status pa_alloc_beam_select(pa_allocator* a, const int64_t* seq_ids, const int32_t* parent_idx,
+                               int n);
 
 /* Copy the sequence's table (up to cap entries) to out; *n = its length, *num_tokens. */
 pa_status pa_alloc_block_table(const pa_allocator* a, int64_t seq_id, int32_t* out, int cap,

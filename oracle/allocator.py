@@ -169,6 +169,44 @@ class RefAllocator:
         self.ntok[seq_id] = pos + 1
         return phys * self.block_size + off, src, dst
 
+    def truncate(self, seq_id, num_tokens):
+        """Keep the first ``num_tokens`` tokens; blocks past ceil(n/bs) are released in
+        table order (speculative rollback, concept card section 已知局限)."""
+        if seq_id not in self.tables:
+            raise KeyError(f"unknown sequence {seq_id}")
+        if not 0 <= num_tokens <= self.ntok[seq_id]:
+            raise ValueError("num_tokens out of range")
+        keep = -(-num_tokens // self.block_size)
+        table = self.tables[seq_id]
+        for b in table[keep:]:
+            self.ref[b] -= 1
+            if self.ref[b] == 0:
+                self.free.append(b)
+        del table[keep:]
+        self.ntok[seq_id] = num_tokens
+
+    def beam_select(self, seq_ids, parent_idx):
+        """Beam i continues from beam parent_idx[i] (beam search shares the blocks before
+        the branch point: concept card section 带来的能力).  New references first, then
+        the old tables are released, beam 0 first, each in table order."""
+        seq_ids = [int(x) for x in seq_ids]
+        if len(set(seq_ids)) != len(seq_ids) or any(s not in self.tables for s in seq_ids):
+            raise KeyError("beam ids must be distinct live sequences")
+        if any(not 0 <= int(p) < len(seq_ids) for p in parent_idx):
+            raise ValueError("parent index out of range")
+        new = [(list(self.tables[seq_ids[int(p)]]), self.ntok[seq_ids[int(p)]]) for p in parent_idx]
+        for table, _ in new:
+            for b in table:
+                self.ref[b] += 1
+        for sid in seq_ids:
+            for b in self.tables[sid]:
+                self.ref[b] -= 1
+                if self.ref[b] == 0:
+                    self.free.append(b)
+        for sid, (table, n) in zip(seq_ids, new):
+            self.tables[sid] = table
+            self.ntok[sid] = n
+
     def free_seq(self, seq_id):
         """Drop the sequence; blocks whose refcount reaches 0 return to the free list."""
         if seq_id not in self.tables:

@@ -105,6 +105,8 @@ def _load():
         "pa_alloc_append_slot": (i32, [vp, i64, pi64, pi32, pi32]),
         "pa_alloc_append_slots": (i32, [vp, pi64, i32, pi64, pi32, pint]),
         "pa_alloc_free_seq": (i32, [vp, i64]),
+        "pa_alloc_truncate": (i32, [vp, i64, i32]),
+        "pa_alloc_beam_select": (i32, [vp, pi64, pi32, i32]),
         "pa_alloc_block_table": (i32, [vp, i64, pi32, i32, pint, pint]),
         "pa_alloc_block_tables": (i32, [vp, pi64, i32, pi32, i32, pi32]),
         "pa_alloc_seq_slots": (i32, [vp, i64, pi64, i32, pint]),
@@ -128,7 +130,8 @@ EXPORTED = (
     "pa_status_string", "pa_status_from_device_flag", "pa_version", "pa_decode_workspace_size",
     "pa_decode", "pa_decode_ex", "pa_decode_plan", "pa_decode_no_alloc", "pa_reshape_and_cache", "pa_copy_blocks", "pa_alloc_create",
     "pa_alloc_create_ordered", "pa_alloc_destroy", "pa_alloc_add_seq", "pa_alloc_fork",
-    "pa_alloc_append_slot", "pa_alloc_append_slots", "pa_alloc_free_seq", "pa_alloc_block_table",
+    "pa_alloc_append_slot", "pa_alloc_append_slots", "pa_alloc_free_seq", "pa_alloc_truncate",
+    "pa_alloc_beam_select", "pa_alloc_block_table",
     "pa_alloc_block_tables", "pa_alloc_seq_slots", "pa_alloc_refcount", "pa_alloc_num_free",
     "pa_alloc_internal_waste_slots", "pa_alloc_free_list",
 )
@@ -336,6 +339,16 @@ class Allocator:
 
     def free_seq(self, seq_id):
         _check(lib.pa_alloc_free_seq(self._h, seq_id), "pa_alloc_free_seq")
+
+    def truncate(self, seq_id, num_tokens):
+        _check(lib.pa_alloc_truncate(self._h, seq_id, num_tokens), "pa_alloc_truncate")
+
+    def beam_select(self, seq_ids, parent_idx):
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        par = np.ascontiguousarray(parent_idx, dtype=np.int32)
+        _need(ids.size == par.size, "one parent index per beam")
+        _check(lib.pa_alloc_beam_select(self._h, _i64p(ids), _i32p(par), ids.size),
+               "pa_alloc_beam_select")
 
     def block_table(self, seq_id):
         n, ntok = ctypes.c_int(), ctypes.c_int()

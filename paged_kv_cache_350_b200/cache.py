@@ -210,6 +210,14 @@ class PagedKVCache:
         """The child shares every block of the parent (copy on write at its first append)."""
         self.alloc.fork(parent_id, child_id)
 
+    def beam_select(self, seq_ids, parent_idx):
+        """Beam search: beam i continues from beam parent_idx[i] (blocks shared, no copy)."""
+        self.alloc.beam_select(seq_ids, parent_idx)
+
+    def truncate(self, seq_id, num_tokens):
+        """Roll a sequence back to its first num_tokens tokens (rejected speculation)."""
+        self.alloc.truncate(seq_id, num_tokens)
+
     def retire(self, seq_id):
         """Free the sequence; blocks no other sequence holds return to the pool."""
         self.alloc.free_seq(seq_id)

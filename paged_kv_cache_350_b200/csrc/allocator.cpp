@@ -222,6 +222,47 @@ pa_status pa_alloc_free_seq(pa_allocator* a, int64_t seq_id) {
   return PA_OK;
 }
 
+pa_status pa_alloc_truncate(pa_allocator* a, int64_t seq_id, int num_tokens) {
+  if (!a || num_tokens < 0) return PA_ERR_INVALID_ARG;
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
+  Seq& s = it->second;
+  if (num_tokens > s.ntok) return PA_ERR_INVALID_ARG;
+  const size_t keep = (static_cast<size_t>(num_tokens) + a->block_size - 1) / a->block_size;
+  for (size_t j = keep; j < s.table.size(); ++j) {
+    const int32_t b = s.table[j];
+    if (--a->ref[b] == 0) a->free_stack.push_back(b);
+  }
+  s.table.resize(keep);
+  s.ntok = num_tokens;
+  return PA_OK;
+}
+
+pa_status pa_alloc_beam_select(pa_allocator* a, const int64_t* seq_ids, const int32_t* parent_idx,
+                               int n) {
+  if (!a || n < 0 || (n > 0 && (!seq_ids || !parent_idx))) return PA_ERR_INVALID_ARG;
+  std::vector<Seq*> rows(n);
+  std::unordered_set<int64_t> seen;
+  for (int i = 0; i < n; ++i) {
+    auto it = a->seqs.find(seq_ids[i]);
+    if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
+    if (!seen.insert(seq_ids[i]).second) return PA_ERR_INVALID_ARG;
+    if (parent_idx[i] < 0 || parent_idx[i] >= n) return PA_ERR_INVALID_ARG;
+    rows[i] = &it->second;
+  }
+  std::vector<Seq> next(n);
+  for (int i = 0; i < n; ++i) {
+    next[i] = *rows[parent_idx[i]];
+    for (int32_t b : next[i].table) a->ref[b] += 1;
+  }
+  for (int i = 0; i < n; ++i) {
+    for (int32_t b : rows[i]->table)
+      if (--a->ref[b] == 0) a->free_stack.push_back(b);
+  }
+  for (int i = 0; i < n; ++i) *rows[i] = std::move(next[i]);
+  return PA_OK;
+}
+
 pa_status pa_alloc_block_table(const pa_allocator* a, int64_t seq_id, int32_t* out, int cap,
                                int* n, int* num_tokens) {
   if (!a || !n || !num_tokens || cap < 0 || (cap > 0 && !out)) return PA_ERR_INVALID_ARG;

@@ -37,7 +37,7 @@ def test_random_op_sequences_bit_exact(seed):
     live = set()
     next_id = 0
     for _ in range(300):
-        op = rng.choice(["add", "fork", "append", "append", "append", "free"])
+        op = rng.choice(["add", "fork", "append", "append", "append", "free", "truncate", "select"])
         c_exc = r_exc = None
         if op == "add" or not live:
             sid, n = next_id, int(rng.integers(0, 3 * bs))
@@ -69,6 +69,16 @@ def test_random_op_sequences_bit_exact(seed):
             except OutOfBlocks:
                 r_exc, rres = 3, None
             assert cres == rres
+        elif op == "truncate":
+            sid = int(rng.choice(sorted(live)))
+            n = int(rng.integers(0, r.ntok[sid] + 1))
+            c.truncate(sid, n)
+            r.truncate(sid, n)
+        elif op == "select":
+            beams = [int(x) for x in rng.choice(sorted(live), size=min(len(live), 4), replace=False)]
+            parents = [int(x) for x in rng.integers(0, len(beams), size=len(beams))]
+            c.beam_select(beams, parents)
+            r.beam_select(beams, parents)
         else:
             sid = int(rng.choice(sorted(live)))
             c.free_seq(sid)
@@ -131,3 +141,17 @@ def test_errors_leave_state_unchanged():
     assert state(c, {0, 1, 2}, 3) == before
     with pytest.raises(PAError):
         _alloc(4, 4, pop_order=[0, 1, 1, 2])
+
+
+def test_truncate_and_beam_select_reject_bad_arguments_without_change():
+    from paged_kv_cache_350_b200 import PAError
+    c = _alloc(16, 4)
+    c.add_seq(0, 6)
+    c.add_seq(1, 3)
+    before = state(c, {0, 1}, 16)
+    for f, args in ((c.truncate, (0, 7)), (c.truncate, (0, -1)), (c.truncate, (9, 0)),
+                    (c.beam_select, ([0, 1], [0, 2])), (c.beam_select, ([0, 0], [0, 0])),
+                    (c.beam_select, ([0, 5], [0, 0]))):
+        with pytest.raises(PAError):
+            f(*args)
+    assert state(c, {0, 1}, 16) == before

@@ -158,6 +158,39 @@ def test_out_of_blocks_leaves_state_unchanged():
     assert before == after
 
 
+def test_truncate_releases_tail_blocks_and_rewrites_shared_partial_block():
+    alloc = RefAllocator(8, 4)
+    alloc.add_seq(0, 10)                 # blocks [0, 1, 2], 2 of 4 used in block 2
+    alloc.fork(0, 1)
+    alloc.truncate(0, 5)                 # keeps blocks [0, 1]; block 2 still held by 1
+    assert alloc.block_table(0) == ([0, 1], 5)
+    assert [alloc.refcount(b) for b in range(3)] == [2, 2, 1]
+    slot, src, dst = alloc.append_slot(0)   # block 1 is shared and partial: copy on write
+    assert src == 1 and slot == dst * 4 + 1
+    alloc.truncate(1, 0)                 # all of sequence 1's blocks released
+    assert alloc.block_table(1) == ([], 0)
+    assert alloc.refcount(2) == 0 and alloc.refcount(0) == 1
+    alloc.truncate(0, 4)                 # exactly one block: the copied block goes back
+    assert alloc.block_table(0) == ([0], 4) and alloc.refcount(dst) == 0
+
+
+def test_beam_select_shares_parent_blocks_and_frees_dropped_beams():
+    alloc = RefAllocator(16, 4)
+    alloc.add_seq(0, 4)                  # prompt in block 0
+    for c in (1, 2, 3):
+        alloc.fork(0, c)
+    for s in range(4):                   # each beam writes its own block 1..4
+        alloc.append_slot(s)
+    private = [alloc.block_table(s)[0][1] for s in range(4)]
+    alloc.beam_select([0, 1, 2, 3], [2, 2, 0, 2])
+    for s, p in zip(range(4), [2, 2, 0, 2]):
+        assert alloc.block_table(s)[0] == [0, private[p]]
+    assert alloc.refcount(0) == 4
+    assert alloc.refcount(private[2]) == 3 and alloc.refcount(private[0]) == 1
+    assert alloc.refcount(private[1]) == 0 and alloc.refcount(private[3]) == 0
+    assert alloc.num_free() == 16 - 3
+
+
 def test_splitmix64_published_vectors():
     # splitmix64 reference implementation (Vigna, prng.di.unimi.it/splitmix64.c), seed 1234567
     g = splitmix64_stream(1234567)

@@ -30,6 +30,10 @@ def _oracle_replay(tr):
             elif e[0] == "fork":
                 alloc.fork(e[1], e[2])
                 live.append(e[2])
+            elif e[0] == "select":
+                alloc.beam_select(e[1], e[2])
+            elif e[0] == "truncate":
+                alloc.truncate(e[1], e[2])
             else:
                 alloc.free_seq(e[1])
                 live.remove(e[1])
@@ -68,11 +72,33 @@ def test_trace_replay_keeps_allocator_invariants():
     assert any(e[0] == "retire" for ev in tr.events for e in ev)
 
 
+TRACES = {
+    "serve_bs16_g8": lambda: workloads.serving_trace(seed=3201, steps=36, bs=16, Hq=16, Hkv=2),
+    "serve_bs8_g4": lambda: workloads.serving_trace(seed=3202, steps=36, bs=8, Hq=8, Hkv=2),
+    "serve_bs32_g2": lambda: workloads.serving_trace(seed=3203, steps=36, bs=32, Hq=4, Hkv=2),
+    "beam_bs16": lambda: workloads.beam_trace(seed=3301, bs=16),
+    "beam_bs8": lambda: workloads.beam_trace(seed=3302, bs=8, Hq=8, Hkv=2, prompt_len=20),
+}
+
+
+def test_beam_trace_replay_keeps_allocator_invariants():
+    tr = workloads.beam_trace(seed=3401)
+    _, _, _, _, alloc = _oracle_replay(tr)
+    used = {}
+    for sid, tab in alloc.tables.items():
+        for b in tab:
+            used[b] = used.get(b, 0) + 1
+    for b in range(tr.num_blocks):
+        assert alloc.refcount(b) == used.get(b, 0)
+    assert any(e[0] == "select" for ev in tr.events for e in ev)
+    assert any(e[0] == "truncate" for ev in tr.events for e in ev)
+
+
 @pytest.mark.gpu
-@pytest.mark.parametrize("seed,bs,G", [(3201, 16, 8), (3202, 8, 4), (3203, 32, 2)])
-def test_serving_trace_matches_oracle_replay(seed, bs, G):
+@pytest.mark.parametrize("name", sorted(TRACES))
+def test_serving_trace_matches_oracle_replay(name):
     import paged_kv_cache_350_b200 as pa
-    tr = workloads.serving_trace(seed=seed, steps=36, bs=bs, Hq=2 * G, Hkv=2)
+    tr = TRACES[name]()
     outs, plans, ref_kp, ref_vp, ref_alloc = _oracle_replay(tr)
 
     def dev(a):
@@ -93,6 +119,10 @@ def test_serving_trace_matches_oracle_replay(seed, bs, G):
             elif e[0] == "fork":
                 cache.fork(e[1], e[2])
                 live.append(e[2])
+            elif e[0] == "select":
+                cache.beam_select(e[1], e[2])
+            elif e[0] == "truncate":
+                cache.truncate(e[1], e[2])
             else:
                 cache.retire(e[1])
                 live.remove(e[1])

@@ -317,8 +317,9 @@ def run_step_allocation(w, alloc):
 class ServingTrace:
     """Per-step events of a serving loop; every live sequence decodes one token per step.
 
-    ``events[t]`` lists ("admit", seq_id, prompt_len), ("fork", parent, child) and
-    ("retire", seq_id) applied before step t's decode.  The prompt K/V of an admission
+    ``events[t]`` lists ("admit", seq_id, prompt_len), ("fork", parent, child),
+    ("retire", seq_id), ("select", beam_ids, parent_indices) and ("truncate", seq_id,
+    num_tokens) applied before step t's decode.  The prompt K/V of an admission
     and every step's q / new K / new V are drawn with ``draw_normal`` from ``seed`` and
     the stream numbers ``prompt_stream`` / ``step_stream`` give.
     """
@@ -386,6 +387,35 @@ def serving_trace(seed=3000, steps=40, start=6, max_live=12, prompt_lo=1, prompt
             max_tokens = max(max_tokens, tokens[sid])
     mb = _blocks(max_tokens, bs) + 1
     nb = num_blocks or (max_live + 2) * mb * 2
+    return ServingTrace(seed=seed, dtype=dtype, Hq=Hq, Hkv=Hkv, D=D, block_size=bs,
+                        num_blocks=nb, scale=1.0 / math.sqrt(D), alloc_seed=seed + 1,
+                        events=events, max_blocks=mb)
+
+
+def beam_trace(seed=3300, beams=4, steps=30, prompt_len=37, p_select=0.6, p_truncate=0.25,
+               Hq=16, Hkv=2, D=128, bs=16, dtype="bf16"):
+    """Beam search with speculative rollback: one prompt forked into ``beams`` beams;
+    before a step the beams may be re-selected from random parents, and one beam may be
+    rolled back by 1-3 tokens (never into the prompt)."""
+    rng = np.random.default_rng(seed)
+    events = [[("admit", 0, prompt_len)] + [("fork", 0, b) for b in range(1, beams)]]
+    ntok = [prompt_len] * beams
+    for t in range(1, steps):
+        ev = []
+        if rng.random() < p_select:
+            parents = [int(x) for x in rng.integers(0, beams, size=beams)]
+            ev.append(("select", tuple(range(beams)), tuple(parents)))
+            ntok = [ntok[p] for p in parents]
+        if rng.random() < p_truncate:
+            b = int(rng.integers(0, beams))
+            n = max(prompt_len, ntok[b] - int(rng.integers(1, 4)))
+            ev.append(("truncate", b, n))
+            ntok[b] = n
+        events.append(ev)
+        ntok = [n + 1 for n in ntok]
+    ntok = [n + 1 for n in ntok]
+    mb = _blocks(prompt_len + steps + 1, bs) + 1
+    nb = beams * mb * 3 + 8
     return ServingTrace(seed=seed, dtype=dtype, Hq=Hq, Hkv=Hkv, D=D, block_size=bs,
                         num_blocks=nb, scale=1.0 / math.sqrt(D), alloc_seed=seed + 1,
                         events=events, max_blocks=mb)
