@@ -4,10 +4,11 @@
 // 实现要点) — scheduled for a whole batch of ragged lengths.
 //
 // Schedule ("streams"):
-//   * Every (sequence b, KV head) is a unit of nt(b) = ceil(L_b / TILE_T) tiles; units
-//     are laid end to end in (b, KV head) order, T = Hkv * sum_b nt(b) tiles in all.
-//   * The grid is one wave of persistent CTAs (SM count x occupancy).  Each CTA has 4
-//     warps and every warp is one stream: stream s owns the global tiles
+//   * Every (sequence b, KV head) is a unit of nt(b) = ceil(L_b / TILE_T) tiles of
+//     TILE_T tokens (32 by default: two blocks of 16); units are laid end to end in
+//     (b, KV head) order, T = Hkv * sum_b nt(b) tiles in all.
+//   * The grid is one wave of persistent CTAs (SM count x occupancy: 3 CTAs of 2 warps
+//     per SM by default).  Every warp is one stream: stream s owns the global tiles
 //     [s*per, (s+1)*per), per = ceil(T / streams).  Work is balanced to one tile.
 //   * Each CTA first computes the prefix sums of nt(b) in shared memory; a global tile
 //     index maps to (b, KV head, tile) by binary search.
@@ -46,12 +47,20 @@ namespace {
 #define PA_STREAM_PDL 1
 #endif
 
+// Warps (= streams) per CTA and tokens per pipeline stage.
+#ifndef PA_STREAM_NCW
+#define PA_STREAM_NCW 2
+#endif
+#ifndef PA_STREAM_TILE
+#define PA_STREAM_TILE 32
+#endif
+
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kNCW = 4;                      // warps (= streams) per CTA
+constexpr int kNCW = PA_STREAM_NCW;          // warps (= streams) per CTA
 constexpr int kThreads = kNCW * 32;
 
 template <int D_, int BS_, bool ROWS16_, int SPW_>
-struct StreamCfg : TileCfg<D_, BS_, ROWS16_> {
+struct StreamCfg : TileCfg<D_, BS_, ROWS16_, PA_STREAM_TILE> {
   static constexpr int SPW = SPW_;                 // ring stages per stream
   static constexpr int NST = kNCW * SPW;
   static constexpr int RING_BYTES = NST * StreamCfg::STAGE_BYTES;
@@ -103,13 +112,14 @@ __device__ __forceinline__ TilePos locate(const int* P, int B, int Hkv, int g) {
 
 // Block ids, KV head and block count of one tile, resolved by one lane.
 struct TileIds {
-  int kvh, id0, id1, nb;
+  int kvh, nb;
+  int id[4];
 };
 
 template <class C>
 __device__ __forceinline__ TileIds resolve_tile(const DecodeParams& p, const int* P, int g,
                                                 int end) {
-  TileIds r{0, 0, 0, 0};
+  TileIds r{0, 0, {0, 0, 0, 0}};
   if (g >= end) return r;
   const TilePos t = locate(P, p.B, p.Hkv, g);
   r.kvh = t.kvh;
@@ -118,8 +128,9 @@ __device__ __forceinline__ TileIds resolve_tile(const DecodeParams& p, const int
   const int blk = t.j * C::BPS;
   r.nb = min(C::BPS, nblk - blk);
   const int32_t* tab = p.block_tables + static_cast<size_t>(t.b) * p.max_blocks + blk;
-  r.id0 = __ldg(tab);
-  if (C::BPS > 1 && r.nb > 1) r.id1 = __ldg(tab + 1);
+#pragma unroll
+  for (int k = 0; k < C::BPS; ++k)
+    if (k < r.nb) r.id[k] = __ldg(tab + k);
   return r;
 }
 
@@ -215,23 +226,25 @@ __global__ void __launch_bounds__(kThreads, PA_STREAM_MIN_CTAS)
     }
     const int src = k & 31;
     const int kv = __shfl_sync(kFull, cur.kvh, src);
-    int i0 = __shfl_sync(kFull, cur.id0, src);
-    int i1 = __shfl_sync(kFull, cur.id1, src);
     const int n = __shfl_sync(kFull, cur.nb, src);
+    int ids[C::BPS];
+#pragma unroll
+    for (int q = 0; q < C::BPS; ++q) ids[q] = __shfl_sync(kFull, cur.id[q], src);
     if (lane == 0) {
-      if (i0 < 0 || i0 >= p.num_blocks || (n > 1 && (i1 < 0 || i1 >= p.num_blocks))) {
-        flag_error(p.err, PA_DEVERR_BAD_BLOCK_ID);
-        if (i0 < 0 || i0 >= p.num_blocks) i0 = 0;
-        if (i1 < 0 || i1 >= p.num_blocks) i1 = 0;
-      }
       const int stage = warp * SPW + k % SPW;
       const uint32_t fb = smem_addr(&full_bar[stage]);
       const uint32_t kt = smem_addr(smem + stage * C::STAGE_BYTES);
       const uint32_t vt = kt + C::TILE_BYTES;
       fence_proxy_async_smem();  // this stage's earlier generic reads/writes come first
       mbar_arrive_expect_tx(fb, static_cast<uint32_t>(n * BS * D * 2 * 2));
-      for (int sub = 0; sub < n; ++sub) {
-        const int phys = sub == 0 ? i0 : i1;
+#pragma unroll
+      for (int sub = 0; sub < C::BPS; ++sub) {
+        if (sub >= n) break;
+        int phys = ids[sub];
+        if (phys < 0 || phys >= p.num_blocks) {
+          flag_error(p.err, PA_DEVERR_BAD_BLOCK_ID);
+          phys = 0;
+        }
 #pragma unroll
         for (int c = 0; c < C::DCH; ++c) {
           tma_load_4d(kt + c * C::CHUNK_BYTES + sub * BS * 128, &tmk, c * 64, kv, 0, phys, fb,
@@ -470,6 +483,8 @@ cudaError_t launch_d_bs(const StreamParams& sp, int grid, cudaStream_t stream) {
 }
 
 }  // namespace
+
+int stream_warps_per_cta() { return kNCW; }
 
 int stream_grid(int D, int block_size, int G, int B) {
   int dev = 0, sms = 0;

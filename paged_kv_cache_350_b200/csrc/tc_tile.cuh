@@ -12,12 +12,13 @@
 
 namespace pa {
 
-template <int D_, int BS_, bool ROWS16_>
+// TT: tokens per pipeline stage when blocks are smaller (a stage holds whole blocks).
+template <int D_, int BS_, bool ROWS16_, int TT_ = 16>
 struct TileCfg {
   static constexpr int D = D_;
   static constexpr int BS = BS_;
   static constexpr bool ROWS16 = ROWS16_;
-  static constexpr int TILE_T = BS > 16 ? BS : 16;   // tokens per pipeline stage
+  static constexpr int TILE_T = BS > TT_ ? BS : TT_;  // tokens per pipeline stage
   static constexpr int BPS = TILE_T / BS;            // blocks per stage
   static constexpr int SUBT = TILE_T / 16;           // 16-token sub-tiles per stage
   static constexpr int DCH = D / 64;                 // 128-byte column chunks per row
@@ -29,6 +30,7 @@ struct TileCfg {
   static constexpr int NT = D / 8;                      // output n-tiles of 8 columns
   static_assert(D == 64 || D == 128, "head dim");
   static_assert(BS == 8 || BS == 16 || BS == 32, "block size");
+  static_assert(TILE_T % 16 == 0 && BPS <= 4, "stage tokens");
 };
 
 __device__ __forceinline__ uint32_t sw128(int row, int c16) {
