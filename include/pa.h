@@ -170,6 +170,33 @@ pa_status pa_decode_ex(void* out, const void* q, const void* k_pool, const void*
                        float scale, pa_dtype dtype, void* workspace, size_t workspace_bytes,
                        int32_t* dev_err_flag, pa_stream_t stream, const pa_decode_opts* opts);
 
+/* Decode for a batch in which groups of sequences share their leading blocks: samples
+ * forked from one prompt, or requests with a common system prompt ("深入解析 PagedAttention",
+ * 多序列共享; "什么是 LLM 中的分页注意力", 跨请求的内存共享).  Same result as pa_decode, but each
+ * group's shared tokens are read from HBM once for the whole group: the members' query heads
+ * are stacked as one tile (members x Hq/Hkv <= 16 rows), and each member's own tokens are
+ * merged with its share by log-sum-exp.
+ *   group_of      [B] device int32: group of batch row b, or -1
+ *   group_prefix  [ngroups] device int32: shared tokens of the group, a multiple of
+ *                 PA_SHARED_PREFIX_ALIGN and <= every member's length; members' tables must
+ *                 hold the same block ids for those tokens
+ *   group_members [ngroups][max_members] device int32: the group's batch rows, -1 padded
+ * pa_alloc_prefix_groups builds these from the allocator.  bf16 tensor-core shapes only
+ * (PA_ERR_UNSUPPORTED otherwise); max_members * (Hq/Hkv) <= 16; B + ngroups <= 8192.
+ * Workspace: pa_decode_shared_prefix_workspace_size (on the current device). */
+#define PA_SHARED_PREFIX_ALIGN 32
+size_t pa_decode_shared_prefix_workspace_size(int B, int Hq, int Hkv, int D, int block_size,
+                                              int ngroups);
+pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_pool,
+                                  const void* v_pool, const int32_t* block_tables,
+                                  const int32_t* seq_lens, int B, int Hq, int Hkv, int D,
+                                  int block_size, int max_blocks, int num_blocks, float scale,
+                                  pa_dtype dtype, const int32_t* group_of,
+                                  const int32_t* group_prefix, const int32_t* group_members,
+                                  int ngroups, int max_members, void* workspace,
+                                  size_t workspace_bytes, int32_t* dev_err_flag,
+                                  pa_stream_t stream);
+
 /* Decode without any device allocation.  The source pages have no counterpart: this
  * entry point exists for callers that cannot allocate device memory, so cannot provide
  * pa_decode's workspace: e.g. a serving runtime that owns every device buffer through
@@ -276,6 +303,15 @@ pa_status pa_alloc_block_tables(const pa_allocator* a, const int64_t* seq_ids, i
  * Used to write a prompt's K/V (prefill) with pa_reshape_and_cache. */
 pa_status pa_alloc_seq_slots(const pa_allocator* a, int64_t seq_id, int64_t* slots, int cap,
                              int* n);
+/* Group a batch for pa_decode_shared_prefix (host arrays).  Batch rows whose tables start
+ * with the same block are taken in batch order, in chunks of max_members; a chunk of >= 2
+ * rows becomes a group whose shared prefix is the leading table entries all its members
+ * hold, capped at the shortest member's length and rounded down to align_tokens; a chunk
+ * whose prefix rounds to 0 is not grouped.  Writes group_of[n], group_prefix[ngroups],
+ * group_members[ngroups][max_members] (-1 padded; room for n groups) and *ngroups. */
+pa_status pa_alloc_prefix_groups(const pa_allocator* a, const int64_t* seq_ids, int n,
+                                 int max_members, int align_tokens, int32_t* group_of,
+                                 int32_t* group_prefix, int32_t* group_members, int* ngroups);
 int pa_alloc_refcount(const pa_allocator* a, int32_t block);   /* -1 if out of range */
 int pa_alloc_num_free(const pa_allocator* a);
 /* Sum over live sequences of (blocks * block_size - tokens). */

@@ -16,6 +16,7 @@ imports without it.
 _BINDING_NAMES = {
     "PA_BF16", "PA_F32", "PA_PATH_AUTO", "PA_PATH_GENERIC", "PA_PATH_TENSOR", "PAError",
     "Allocator", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_size", "pa_decode_plan", "pa_decode_no_alloc",
+    "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_size",
     "pa_reshape_and_cache", "pa_status_from_device_flag", "lib",
 }
 

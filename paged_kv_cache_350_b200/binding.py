@@ -93,6 +93,10 @@ def _load():
                                i32, vp, sz, vp, vp, ctypes.POINTER(pa_decode_opts)]),
         "pa_decode_plan": (i32, [i32, i32, i32, i32, i32, i32, i32, sz,
                                  ctypes.POINTER(pa_decode_opts), ctypes.POINTER(pa_decode_plan_info)]),
+        "pa_decode_shared_prefix_workspace_size": (sz, [i32, i32, i32, i32, i32, i32]),
+        "pa_decode_shared_prefix": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                          i32, f32, i32, vp, vp, vp, i32, i32, vp, sz, vp, vp]),
+        "pa_alloc_prefix_groups": (i32, [vp, pi64, i32, i32, i32, pi32, pi32, pi32, pint]),
         "pa_decode_no_alloc": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                      f32, i32, vp, vp]),
         "pa_reshape_and_cache": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]),
@@ -128,7 +132,9 @@ lib = _load()
 #: every symbol include/pa.h declares
 EXPORTED = (
     "pa_status_string", "pa_status_from_device_flag", "pa_version", "pa_decode_workspace_size",
-    "pa_decode", "pa_decode_ex", "pa_decode_plan", "pa_decode_no_alloc", "pa_reshape_and_cache", "pa_copy_blocks", "pa_alloc_create",
+    "pa_decode", "pa_decode_ex", "pa_decode_plan", "pa_decode_no_alloc",
+    "pa_decode_shared_prefix_workspace_size", "pa_decode_shared_prefix", "pa_alloc_prefix_groups",
+    "pa_reshape_and_cache", "pa_copy_blocks", "pa_alloc_create",
     "pa_alloc_create_ordered", "pa_alloc_destroy", "pa_alloc_add_seq", "pa_alloc_fork",
     "pa_alloc_append_slot", "pa_alloc_append_slots", "pa_alloc_free_seq", "pa_alloc_truncate",
     "pa_alloc_beam_select", "pa_alloc_block_table",
@@ -239,6 +245,42 @@ def pa_decode_no_alloc(out, q, k_pool, v_pool, block_tables, seq_lens, scale, er
     return out
 
 
+PA_SHARED_PREFIX_ALIGN = 32
+
+
+def pa_decode_shared_prefix_workspace_size(B, Hq, Hkv, D, block_size, ngroups):
+    n = lib.pa_decode_shared_prefix_workspace_size(B, Hq, Hkv, D, block_size, ngroups)
+    if n == ctypes.c_size_t(-1).value:
+        raise PAError(PA_ERR_INVALID_ARG, "pa_decode_shared_prefix_workspace_size")
+    return n
+
+
+def pa_decode_shared_prefix(out, q, k_pool, v_pool, block_tables, seq_lens, scale, group_of,
+                            group_prefix, group_members, workspace, err_flag=None, stream=None):
+    """pa_decode reading each group's shared prefix once (device int32 group arrays; see
+    include/pa.h and Allocator.prefix_groups)."""
+    import torch
+    _need(q.dim() == 3 and out.shape == q.shape, "q/out must be [B, Hq, D]")
+    _need(k_pool.dim() == 4 and v_pool.shape == k_pool.shape, "pools must be [NB, bs, Hkv, D]")
+    _need(block_tables.dtype == torch.int32 and seq_lens.dtype == torch.int32, "int32 tables/lens")
+    _need(group_of.dtype == torch.int32 and group_of.numel() == q.shape[0], "group_of int32 [B]")
+    _need(group_members.dim() == 2 and group_members.dtype == torch.int32, "members int32 [ng, m]")
+    for t in (out, q, k_pool, v_pool, block_tables, seq_lens, group_of, group_prefix, group_members):
+        _need(t.is_contiguous(), "tensors must be contiguous")
+    B, Hq, D = q.shape
+    NB, bs, Hkv, _ = k_pool.shape
+    ng, maxm = group_members.shape
+    _need(group_prefix.numel() >= ng, "group_prefix [ngroups]")
+    wbytes = workspace.numel() * workspace.element_size()
+    st = lib.pa_decode_shared_prefix(
+        _ptr(out), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables), _ptr(seq_lens), B, Hq,
+        Hkv, D, bs, block_tables.shape[1], NB, float(scale), _dtype_of(q), _ptr(group_of),
+        _ptr(group_prefix), _ptr(group_members), ng, max(maxm, 1), _ptr(workspace), wbytes,
+        _ptr(err_flag), _stream(stream))
+    _check(st, "pa_decode_shared_prefix")
+    return out
+
+
 def pa_reshape_and_cache(key, value, k_pool, v_pool, slot_mapping, err_flag=None, stream=None):
     """Scatter key/value [T,Hkv,D] into the pools at slot_mapping[T] (int64; < 0 skips)."""
     import torch
@@ -339,6 +381,19 @@ class Allocator:
 
     def free_seq(self, seq_id):
         _check(lib.pa_alloc_free_seq(self._h, seq_id), "pa_alloc_free_seq")
+
+    def prefix_groups(self, seq_ids, max_members, align_tokens=PA_SHARED_PREFIX_ALIGN):
+        """(group_of [n], group_prefix [ng], group_members [ng, max_members]) int32 arrays."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = ids.size
+        gof = np.empty(max(n, 1), np.int32)
+        gpre = np.empty(max(n, 1), np.int32)
+        gmem = np.empty((max(n, 1), max_members), np.int32)
+        ng = ctypes.c_int()
+        _check(lib.pa_alloc_prefix_groups(self._h, _i64p(ids), n, max_members, align_tokens,
+                                          _i32p(gof), _i32p(gpre), _i32p(gmem), ctypes.byref(ng)),
+               "pa_alloc_prefix_groups")
+        return gof[:n], gpre[: ng.value], gmem[: ng.value]
 
     def truncate(self, seq_id, num_tokens):
         _check(lib.pa_alloc_truncate(self._h, seq_id, num_tokens), "pa_alloc_truncate")

@@ -313,6 +313,60 @@ pa_status pa_alloc_seq_slots(const pa_allocator* a, int64_t seq_id, int64_t* slo
   return PA_OK;
 }
 
+pa_status pa_alloc_prefix_groups(const pa_allocator* a, const int64_t* seq_ids, int n,
+                                 int max_members, int align_tokens, int32_t* group_of,
+                                 int32_t* group_prefix, int32_t* group_members, int* ngroups) {
+  if (!a || n < 0 || max_members < 1 || align_tokens < 1 || !ngroups ||
+      (n > 0 && (!seq_ids || !group_of || !group_prefix || !group_members)))
+    return PA_ERR_INVALID_ARG;
+  std::vector<const Seq*> rows(n);
+  for (int i = 0; i < n; ++i) {
+    auto it = a->seqs.find(seq_ids[i]);
+    if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
+    rows[i] = &it->second;
+    group_of[i] = -1;
+  }
+  // rows by first block, in batch order (first-appearance order of the blocks)
+  std::vector<int32_t> firsts;
+  std::unordered_map<int32_t, std::vector<int>> buckets;
+  for (int i = 0; i < n; ++i) {
+    if (rows[i]->table.empty()) continue;
+    const int32_t f = rows[i]->table[0];
+    auto& v = buckets[f];
+    if (v.empty()) firsts.push_back(f);
+    v.push_back(i);
+  }
+  int ng = 0;
+  for (int32_t f : firsts) {
+    const std::vector<int>& v = buckets[f];
+    for (size_t c0 = 0; c0 < v.size(); c0 += max_members) {
+      const size_t c1 = std::min(v.size(), c0 + static_cast<size_t>(max_members));
+      if (c1 - c0 < 2) continue;
+      size_t k = rows[v[c0]]->table.size();
+      int64_t shortest = rows[v[c0]]->ntok;
+      for (size_t m = c0 + 1; m < c1; ++m) {
+        const Seq& s = *rows[v[m]];
+        size_t j = 0;
+        while (j < k && j < s.table.size() && s.table[j] == rows[v[c0]]->table[j]) ++j;
+        k = j;
+        shortest = std::min<int64_t>(shortest, s.ntok);
+      }
+      int64_t prefix = std::min<int64_t>(static_cast<int64_t>(k) * a->block_size, shortest);
+      prefix -= prefix % align_tokens;
+      if (prefix <= 0) continue;
+      group_prefix[ng] = static_cast<int32_t>(prefix);
+      for (int m = 0; m < max_members; ++m) {
+        const size_t idx = c0 + m;
+        group_members[static_cast<size_t>(ng) * max_members + m] = idx < c1 ? v[idx] : -1;
+        if (idx < c1) group_of[v[idx]] = ng;
+      }
+      ++ng;
+    }
+  }
+  *ngroups = ng;
+  return PA_OK;
+}
+
 int pa_alloc_refcount(const pa_allocator* a, int32_t block) {
   if (!a || block < 0 || block >= a->num_blocks) return -1;
   return a->ref[block];

@@ -240,6 +240,79 @@ pa_status pa_decode(void* out, const void* q, const void* k_pool, const void* v_
                       dev_err_flag, stream, nullptr);
 }
 
+size_t pa_decode_shared_prefix_workspace_size(int B, int Hq, int Hkv, int D, int block_size,
+                                              int ngroups) {
+  if (B < 0 || ngroups < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || (D != 64 && D != 128) ||
+      !block_size_ok(block_size))
+    return static_cast<size_t>(-1);
+  int grid = pa::prefix_grid(D, block_size, B + ngroups);
+  if (grid <= 0) grid = kStreamGridBound;  // no device to ask: an upper bound
+  return pa::prefix_workspace_bytes(grid * pa::prefix_warps_per_cta(), (B + ngroups) * Hkv, D);
+}
+
+pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_pool,
+                                  const void* v_pool, const int32_t* block_tables,
+                                  const int32_t* seq_lens, int B, int Hq, int Hkv, int D,
+                                  int block_size, int max_blocks, int num_blocks, float scale,
+                                  pa_dtype dtype, const int32_t* group_of,
+                                  const int32_t* group_prefix, const int32_t* group_members,
+                                  int ngroups, int max_members, void* workspace,
+                                  size_t workspace_bytes, int32_t* dev_err_flag,
+                                  pa_stream_t stream) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || max_blocks <= 0 || num_blocks <= 0 ||
+      block_size <= 0 || !std::isfinite(scale) || ngroups < 0 || max_members < 1 ||
+      (dtype != PA_F32 && dtype != PA_BF16))
+    return PA_ERR_INVALID_ARG;
+  const int G = Hq / Hkv;
+  if (!pa::tc_eligible(G, D, block_size, dtype)) return PA_ERR_UNSUPPORTED;
+  if (G * max_members > 16 || B + ngroups > kStreamMaxB) return PA_ERR_UNSUPPORTED;
+  const int64_t max_seq = static_cast<int64_t>(max_blocks) * block_size;
+  if (max_seq > 0x7fffffffLL) return PA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(B + ngroups) * Hkv * ceil_div(max_seq, PA_SHARED_PREFIX_ALIGN) >=
+      (int64_t(1) << 31))
+    return PA_ERR_UNSUPPORTED;
+  if (B == 0) return PA_OK;
+  if (!out || !q || !k_pool || !v_pool || !block_tables || !seq_lens || !group_of ||
+      (ngroups > 0 && (!group_prefix || !group_members)))
+    return PA_ERR_INVALID_ARG;
+  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) ||
+      !aligned(block_tables, 4) || !aligned(seq_lens, 4) || !aligned(group_of, 4) ||
+      (dev_err_flag && !aligned(dev_err_flag, 4)) || !workspace || !aligned(workspace, 256))
+    return PA_ERR_INVALID_ARG;
+  const int grid = pa::prefix_grid(D, block_size, B + ngroups);
+  if (grid <= 0) return PA_ERR_CUDA;
+  pa::PrefixParams pp{};
+  pp.streams = grid * pa::prefix_warps_per_cta();
+  const int units = (B + ngroups) * Hkv;
+  if (workspace_bytes < pa::prefix_workspace_bytes(pp.streams, units, D)) return PA_ERR_INVALID_ARG;
+  pa::DecodeParams& p = pp.d;
+  p.out = out;
+  p.q = q;
+  p.k_pool = k_pool;
+  p.v_pool = v_pool;
+  p.block_tables = block_tables;
+  p.seq_lens = seq_lens;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = G;
+  p.D = D;
+  p.block_size = block_size;
+  p.max_blocks = max_blocks;
+  p.num_blocks = num_blocks;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.max_parts = 1;
+  p.err = dev_err_flag;
+  pp.group_of = group_of;
+  pp.group_prefix = group_prefix;
+  pp.group_members = group_members;
+  pp.ngroups = ngroups;
+  pp.max_members = max_members;
+  pa::prefix_carve(&pp, workspace, units);
+  const cudaError_t e = pa::launch_decode_prefix(pp, grid, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_pool, void* v_pool,
                                const int64_t* slot_mapping, int T, int Hkv, int D,
                                int block_size, int num_blocks, pa_dtype dtype,

@@ -44,6 +44,26 @@ size_t stream_workspace_bytes(int streams, int G, int D);
 void stream_carve(StreamParams* sp, void* workspace);
 cudaError_t launch_decode_stream(const StreamParams& sp, int grid, cudaStream_t stream);
 
+// Parameters of the shared-prefix decode (decode_prefix.cu).
+struct PrefixParams {
+  DecodeParams d;
+  const int32_t* group_of;       // [B] group of batch row b, or -1
+  const int32_t* group_prefix;   // [ngroups] shared tokens (multiple of PA_SHARED_PREFIX_ALIGN)
+  const int32_t* group_members;  // [ngroups][max_members] batch rows, -1 padded
+  int ngroups, max_members;
+  int streams;
+  int32_t* meta;   // [streams][4] cut-unit slot metadata
+  float* pml;      // [streams][2][16][2]
+  float* pacc;     // [streams][2][16][D]
+  float* fml;      // [units][16][2]: per-unit partials (group units, grouped sequences)
+  float* facc;     // [units][16][D]
+};
+int prefix_grid(int D, int block_size, int R);
+int prefix_warps_per_cta();
+size_t prefix_workspace_bytes(int streams, int units, int D);
+void prefix_carve(PrefixParams* pp, void* workspace, int units);
+cudaError_t launch_decode_prefix(const PrefixParams& pp, int grid, cudaStream_t stream);
+
 // 4-D TMA view of a bf16 pool [NB][BS][Hkv][D]: box = BS rows x 64 columns of one head.
 bool make_pool_map(CUtensorMap* map, const void* pool, int NB, int BS, int Hkv, int D);
 

@@ -32,10 +32,12 @@ def gpu_step(w, partition_tokens=0, path=0, device="cuda", keep=False, max_ctas=
     """The product path: allocator, copy_blocks, reshape_and_cache, decode. Returns dict."""
     import paged_kv_cache_350_b200 as pa
     alloc = pa.Allocator(w.num_blocks, w.block_size, shuffle_seed=w.alloc_seed, pop_order=w.pop_order)
-    assert workloads.run_setup(w, alloc) == []
+    setup_pairs = workloads.run_setup(w, alloc)
     slots, pairs, tables, lens = workloads.run_step_allocation(w, alloc)
     kp = to_device(w.k_pool(), w, device)
     vp = to_device(w.v_pool(), w, device)
+    if setup_pairs:  # copy-on-write during setup (forks appending into a partial prompt block)
+        pa.pa_copy_blocks(kp, vp, torch.tensor(setup_pairs, dtype=torch.int32, device=device))
     q = to_device(w.q(), w, device)
     nk = to_device(w.new_k(), w, device)
     nv = to_device(w.new_v(), w, device)
@@ -61,9 +63,10 @@ def gpu_step(w, partition_tokens=0, path=0, device="cuda", keep=False, max_ctas=
 def oracle_step(w, rows=None):
     """The oracle path; ``rows`` restricts the decode to a subset of batch rows."""
     alloc = RefAllocator(w.num_blocks, w.block_size, shuffle_seed=w.alloc_seed, pop_order=w.pop_order)
-    assert workloads.run_setup(w, alloc) == []
+    setup_pairs = workloads.run_setup(w, alloc)
     slots, pairs, tables, lens = workloads.run_step_allocation(w, alloc)
-    kp, vp = ref_copy_blocks(w.k_pool(), w.v_pool(), [tuple(p) for p in pairs])
+    kp, vp = ref_copy_blocks(w.k_pool(), w.v_pool(), setup_pairs)
+    kp, vp = ref_copy_blocks(kp, vp, [tuple(p) for p in pairs])
     kp, vp = ref_reshape_and_cache(w.new_k(), w.new_v(), kp, vp, slots)
     rows = np.arange(w.B) if rows is None else np.asarray(rows)
     out = ref_decode(w.q()[rows], kp, vp, tables[rows], lens[rows], w.scale)

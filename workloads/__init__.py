@@ -271,7 +271,11 @@ def build(name, **overrides):
 # append_slot and block_table with the same meaning.
 
 def run_setup(w, alloc):
-    """Execute ``w.setup_ops``; returns the copy pairs the setup produced (normally none)."""
+    """Execute ``w.setup_ops``; returns the copy pairs the setup produced, in order.
+
+    They are none unless a fork appends into a partial prompt block during setup
+    (prompt lengths that are not block multiples); each side then applies them to
+    its pools before the step."""
     pairs = []
     for op in w.setup_ops:
         if op[0] == "add":
