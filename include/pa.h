@@ -174,8 +174,8 @@ pa_status pa_decode_ex(void* out, const void* q, const void* k_pool, const void*
  * forked from one prompt, or requests with a common system prompt ("深入解析 PagedAttention",
  * 多序列共享; "什么是 LLM 中的分页注意力", 跨请求的内存共享).  Same result as pa_decode, but each
  * group's shared tokens are read from HBM once for the whole group: the members' query heads
- * are stacked as one tile (members x Hq/Hkv <= 16 rows), and each member's own tokens are
- * merged with its share by log-sum-exp.
+ * are stacked as one tile (members x Hq/Hkv <= 16 rows) that streams the shared tokens and
+ * then each member's own tokens with the other members' rows masked out of the softmax.
  *   group_of      [B] device int32: group of batch row b, or -1
  *   group_prefix  [ngroups] device int32: shared tokens of the group, a multiple of
  *                 PA_SHARED_PREFIX_ALIGN and <= every member's length; members' tables must

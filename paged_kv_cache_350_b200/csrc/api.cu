@@ -247,7 +247,7 @@ size_t pa_decode_shared_prefix_workspace_size(int B, int Hq, int Hkv, int D, int
     return static_cast<size_t>(-1);
   int grid = pa::prefix_grid(D, block_size, B + ngroups);
   if (grid <= 0) grid = kStreamGridBound;  // no device to ask: an upper bound
-  return pa::prefix_workspace_bytes(grid * pa::prefix_warps_per_cta(), (B + ngroups) * Hkv, D);
+  return pa::prefix_workspace_bytes(grid * pa::prefix_warps_per_cta(), B + ngroups, D);
 }
 
 pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_pool,
@@ -283,8 +283,8 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_pool,
   if (grid <= 0) return PA_ERR_CUDA;
   pa::PrefixParams pp{};
   pp.streams = grid * pa::prefix_warps_per_cta();
-  const int units = (B + ngroups) * Hkv;
-  if (workspace_bytes < pa::prefix_workspace_bytes(pp.streams, units, D)) return PA_ERR_INVALID_ARG;
+  const int rows = B + ngroups;
+  if (workspace_bytes < pa::prefix_workspace_bytes(pp.streams, rows, D)) return PA_ERR_INVALID_ARG;
   pa::DecodeParams& p = pp.d;
   p.out = out;
   p.q = q;
@@ -308,7 +308,7 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_pool,
   pp.group_members = group_members;
   pp.ngroups = ngroups;
   pp.max_members = max_members;
-  pa::prefix_carve(&pp, workspace, units);
+  pa::prefix_carve(&pp, workspace, rows);
   const cudaError_t e = pa::launch_decode_prefix(pp, grid, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

@@ -4,18 +4,19 @@
 // point at the same blocks instead of storing two copies).  Plain paged decode still reads
 // those shared blocks once per sequence.  This kernel reads them once per group.
 //
-// The result is exactly plain attention per (sequence, query head): softmax over the
-// shared tokens and over the sequence's own tokens is merged by log-sum-exp.
+// The result is exactly plain attention per (sequence, query head).
 //
 // Units (laid end to end, balanced over warp streams as in decode_stream.cu):
-//   * group row r < ngroups, KV head h: the group's shared tokens [0, prefix_r), read
-//     through the first member's table; the Q rows are the members' query heads of KV
-//     head h stacked (members x G <= 16 rows of the MMA);
-//   * sequence row ngroups + b, KV head h: tokens [prefix of b's group (0 if none), L_b).
-// A finished unit of an ungrouped sequence writes its output in place; group units and
-// grouped sequences' units leave a partial (max, sum, unnormalised O) in a per-unit
-// buffer; units cut by a stream boundary are first merged by the cut-unit reduce; a last
-// kernel merges, for every grouped sequence, its group partial and its own partial.
+//   * group row r < ngroups, KV head h: the Q rows are the members' query heads of KV head
+//     h stacked (members x G <= 16 MMA rows).  Its tiles are first the shared tokens
+//     [0, prefix_r), read once through the first member's table for all rows, then each
+//     member's own tokens [prefix_r, L_m) through that member's table, with every other
+//     member's rows masked out of the online softmax.  The unit ends with each member's
+//     complete softmax, so it writes the members' outputs itself;
+//   * sequence row ngroups + b, KV head h, for an ungrouped sequence b: [0, L_b).
+// Units cut by a stream boundary leave partials that the cut-unit reduce merges by
+// log-sum-exp (a piece may hold no tile of some member's rows: its max is -inf and it is
+// skipped).
 
 #include <cudaTypedefs.h>
 
@@ -76,41 +77,121 @@ __device__ __forceinline__ int group_of(const PrefixParams& pp, int b, bool flag
   return g;
 }
 
-// Token range and table of unit row r.
-struct RowSpan {
-  int table_b;  // batch row whose block table covers the tokens
-  int tok0;     // first token (multiple of the stage size)
-  int tok1;     // one past the last token
-};
-
-__device__ __forceinline__ RowSpan row_span(const PrefixParams& pp, int r, bool flag) {
-  const DecodeParams& p = pp.d;
-  RowSpan s;
-  if (r < pp.ngroups) {
-    s.table_b = __ldg(pp.group_members + static_cast<size_t>(r) * pp.max_members);
-    s.tok0 = 0;
-    s.tok1 = __ldg(pp.group_prefix + r);
-    if (s.table_b < 0 || s.table_b >= p.B) {  // malformed group: no tokens
-      if (flag) flag_error(p.err, PA_DEVERR_BAD_SEQ_LEN);
-      s.table_b = 0;
-      s.tok1 = 0;
-    }
-  } else {
-    const int b = r - pp.ngroups;
-    const int L = clamp_len(p, b, flag);
-    const int g = group_of(pp, b, flag);
-    const int pre = g >= 0 ? __ldg(pp.group_prefix + g) : 0;
-    s.table_b = b;
-    s.tok0 = pre < L ? pre : L;
-    s.tok1 = L;
-  }
-  return s;
+__device__ __forceinline__ int member_of(const PrefixParams& pp, int r, int m) {
+  return __ldg(pp.group_members + static_cast<size_t>(r) * pp.max_members + m);
 }
 
-template <class C>
+// Members of group r (up to max_members batch rows, -1 padded at the end).
+__device__ __forceinline__ int group_size(const PrefixParams& pp, int r) {
+  int n = 0;
+  while (n < pp.max_members && member_of(pp, r, n) >= 0) ++n;
+  return n;
+}
+
+// Shared tokens of group r (0 for a malformed group, flagged).
+__device__ __forceinline__ int group_prefix_tokens(const PrefixParams& pp, int r, bool flag) {
+  const int b0 = member_of(pp, r, 0);
+  const int pre = __ldg(pp.group_prefix + r);
+  if (b0 < 0 || b0 >= pp.d.B || pre < 0 || pre % PA_SHARED_PREFIX_ALIGN != 0) {
+    if (flag) flag_error(pp.d.err, PA_DEVERR_BAD_SEQ_LEN);
+    return 0;
+  }
+  return pre;
+}
+
+// Own tiles of member m of group r (tokens [pre, L_m)); a member shorter than the prefix is
+// flagged and contributes none.
+template <int TT>
+__device__ __forceinline__ int member_tiles(const PrefixParams& pp, int r, int m, int pre,
+                                            bool flag) {
+  const int b = member_of(pp, r, m);
+  if (b < 0 || b >= pp.d.B) return 0;
+  const int L = clamp_len(pp.d, b, flag);
+  if (L < pre) {
+    if (flag) flag_error(pp.d.err, PA_DEVERR_BAD_SEQ_LEN);
+    return 0;
+  }
+  return (L - pre + TT - 1) / TT;
+}
+
+template <int TT>
 __device__ __forceinline__ int row_tiles(const PrefixParams& pp, int r, bool flag) {
-  const RowSpan s = row_span(pp, r, flag);
-  return (s.tok1 - s.tok0 + C::TILE_T - 1) / C::TILE_T;
+  if (r < pp.ngroups) {
+    const int pre = group_prefix_tokens(pp, r, flag);
+    if (pre == 0) return 0;
+    // member ids first (independent loads), then their lengths (independent loads)
+    int ids[kRows];
+#pragma unroll
+    for (int m = 0; m < kRows; ++m) ids[m] = m < pp.max_members ? member_of(pp, r, m) : -1;
+    int n = pre / TT;
+    bool live = true;
+#pragma unroll
+    for (int m = 0; m < kRows; ++m) {
+      live = live && ids[m] >= 0;
+      if (live && ids[m] < pp.d.B) {
+        const int L = clamp_len(pp.d, ids[m], flag);
+        if (L < pre) {
+          if (flag) flag_error(pp.d.err, PA_DEVERR_BAD_SEQ_LEN);
+        } else {
+          n += (L - pre + TT - 1) / TT;
+        }
+      }
+    }
+    return n;
+  }
+  const int b = r - pp.ngroups;
+  if (group_of(pp, b, flag) >= 0) return 0;  // covered by its group's unit
+  return (clamp_len(pp.d, b, flag) + TT - 1) / TT;
+}
+
+// Where tile j of unit row r comes from.
+struct TileSrc {
+  int table_b;         // batch row whose block table holds the tokens
+  int tok0, tok1;      // tile starts at tok0; the run of tokens ends at tok1
+  int row_lo, row_hi;  // MMA rows that take part
+};
+
+template <int TT>
+__device__ __forceinline__ TileSrc tile_src(const PrefixParams& pp, int r, int j) {
+  TileSrc t;
+  if (r >= pp.ngroups) {
+    const int b = r - pp.ngroups;
+    t.table_b = b;
+    t.tok0 = j * TT;
+    t.tok1 = clamp_len(pp.d, b, false);
+    t.row_lo = 0;
+    t.row_hi = 16;
+    return t;
+  }
+  const int pre = group_prefix_tokens(pp, r, false);
+  const int np = pre / TT;
+  if (j < np) {
+    t.table_b = member_of(pp, r, 0);
+    t.tok0 = j * TT;
+    t.tok1 = pre;
+    t.row_lo = 0;
+    t.row_hi = 16;
+    return t;
+  }
+  int k = j - np;
+  const int gs = group_size(pp, r);
+  for (int m = 0; m < gs; ++m) {
+    const int n = member_tiles<TT>(pp, r, m, pre, false);
+    if (k < n) {
+      const int b = member_of(pp, r, m);
+      t.table_b = b;
+      t.tok0 = pre + k * TT;
+      t.tok1 = clamp_len(pp.d, b, false);
+      t.row_lo = m * pp.d.G;
+      t.row_hi = (m + 1) * pp.d.G;
+      return t;
+    }
+    k -= n;
+  }
+  t.table_b = member_of(pp, r, 0);  // not reached for j < row_tiles
+  t.tok0 = t.tok1 = 0;
+  t.row_lo = t.row_hi = 0;
+  return t;
 }
 
 struct TilePos {
@@ -140,8 +221,8 @@ __device__ __forceinline__ TileIds resolve_tile(const PrefixParams& pp, const in
   const DecodeParams& p = pp.d;
   const TilePos t = locate(P, R, p.Hkv, g);
   out.kvh = t.kvh;
-  const RowSpan s = row_span(pp, t.r, false);
-  const int blk = s.tok0 / C::BS + t.j * C::BPS;
+  const TileSrc s = tile_src<C::TILE_T>(pp, t.r, t.j);
+  const int blk = s.tok0 / C::BS;
   const int nblk = (s.tok1 + C::BS - 1) / C::BS;
   out.nb = min(C::BPS, nblk - blk);
   const int32_t* tab = p.block_tables + static_cast<size_t>(s.table_b) * p.max_blocks + blk;
@@ -151,13 +232,53 @@ __device__ __forceinline__ TileIds resolve_tile(const PrefixParams& pp, const in
   return out;
 }
 
-// Members of group r (up to max_members batch rows, -1 padded).
-__device__ __forceinline__ int group_size(const PrefixParams& pp, int r) {
-  int n = 0;
-  while (n < pp.max_members &&
-         __ldg(pp.group_members + static_cast<size_t>(r) * pp.max_members + n) >= 0)
-    ++n;
-  return n;
+// Batch row and query head of MMA row rr of unit row r (rows < nrows).
+__device__ __forceinline__ void row_target(const PrefixParams& pp, int r, int kvh, int rr, int& b,
+                                           int& h) {
+  const int G = pp.d.G;
+  if (r < pp.ngroups) {
+    b = member_of(pp, r, rr / G);
+    h = kvh * G + rr % G;
+  } else {
+    b = r - pp.ngroups;
+    h = kvh * G + rr;
+  }
+}
+
+// Tile counts of every unit row, scanned: P[r] = tiles of rows before r, P[R] = total (in
+// rows of Hkv units).  One block; one row per thread per pass, so the dependent loads of
+// different rows (group -> members -> lengths) overlap.
+constexpr int kPlanThreads = 1024;
+
+template <int TT>
+__global__ void __launch_bounds__(kPlanThreads) prefix_plan_kernel(const PrefixParams pp) {
+  // The main kernel may launch now: it waits for this grid before reading the plan.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int R = pp.ngroups + pp.d.B;
+  __shared__ int carry;
+  __shared__ int warp_tot[kPlanThreads / 32];
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int base = 0; base < R; base += kPlanThreads) {
+    const int r = base + static_cast<int>(threadIdx.x);
+    const int n = r < R ? row_tiles<TT>(pp, r, true) : 0;
+    int incl = n;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(kFull, incl, off);
+      if (lane >= off) incl += v;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int before = carry;
+    for (int w = 0; w < warp; ++w) before += warp_tot[w];
+    if (r < R) pp.plan[r] = before + incl - n;
+    __syncthreads();
+    if (threadIdx.x == kPlanThreads - 1) carry = before + incl;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) pp.plan[R] = carry;
 }
 
 template <class C>
@@ -177,35 +298,17 @@ __global__ void __launch_bounds__(kThreads)
   uint8_t* qtiles = smem + C::RING_BYTES;
   int* P = reinterpret_cast<int*>(smem + C::FIXED_BYTES);  // [R + 1] tiles before row r
   __shared__ __align__(8) uint64_t full_bar[NST];
-  __shared__ int warp_sum[kThreads / 32];
 
-  {
-    const int chunk = (R + kThreads - 1) / kThreads;
-    const int lo = min(R, static_cast<int>(threadIdx.x) * chunk);
-    const int hi = min(R, lo + chunk);
-    int sum = 0;
-    for (int r = lo; r < hi; ++r) sum += row_tiles<C>(pp, r, blockIdx.x == 0);
-    int incl = sum;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int v = __shfl_up_sync(kFull, incl, off);
-      if (lane >= off) incl += v;
-    }
-    if (lane == 31) warp_sum[warp] = incl;
-    __syncthreads();
-    int base = 0;
-    for (int w = 0; w < warp; ++w) base += warp_sum[w];
-    int run = base + incl - sum;
-    for (int r = lo; r < hi; ++r) {
-      P[r] = run;
-      run += row_tiles<C>(pp, r, false);
-    }
-    if (threadIdx.x == 0) {
-      int total = 0;
-      for (int w = 0; w < kThreads / 32; ++w) total += warp_sum[w];
-      P[R] = total;
-    }
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < NST; ++st) mbar_init(smem_addr(&full_bar[st]), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    fence_proxy_async_smem();
   }
+  // Everything below reads what earlier kernels wrote: wait for the plan kernel (which
+  // itself ran after every earlier kernel on the stream) to complete.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  for (int r = threadIdx.x; r <= R; r += kThreads) P[r] = pp.plan[r];
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
   for (int b = blockIdx.x; b < B; b += gridDim.x) {
     if (clamp_len(p, b, false) == 0) {
@@ -216,9 +319,6 @@ __global__ void __launch_bounds__(kThreads)
   if (threadIdx.x == 0) {
     prefetch_tensormap(&tmk);
     prefetch_tensormap(&tmv);
-    for (int st = 0; st < NST; ++st) mbar_init(smem_addr(&full_bar[st]), 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    fence_proxy_async_smem();
   }
   __syncthreads();
 
@@ -286,26 +386,22 @@ __global__ void __launch_bounds__(kThreads)
   int gpos = beg;
   while (gpos < end && ok) {
     const TilePos t = locate(P, R, Hkv, gpos);
-    const RowSpan span = row_span(pp, t.r, false);
     const int ubeg = Hkv * P[t.r] + t.kvh * t.nt;
     const int uend = ubeg + t.nt;
     const int pend = min(end, uend);
     const int u = t.r * Hkv + t.kvh;
     const bool is_group = t.r < NG;
-    int nrows = G;
+    const int nrows = is_group ? group_size(pp, t.r) * G : G;
     // Stage the unit's Q rows: a group's members' heads of this KV head, or the sequence's.
     {
       constexpr int CPR = D * 2 / 16;
-      if (is_group) nrows = group_size(pp, t.r) * G;
       __syncwarp();
       for (int idx = lane; idx < kRows * CPR; idx += 32) {
         const int rr = idx / CPR, c = idx - rr * CPR;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (rr < nrows) {
-          const int b = is_group
-              ? __ldg(pp.group_members + static_cast<size_t>(t.r) * pp.max_members + rr / G)
-              : t.r - NG;
-          const int h = t.kvh * G + (rr % G);
+          int b, h;
+          row_target(pp, t.r, t.kvh, rr, b, h);
           if (b >= 0 && b < B)
             v = __ldg(reinterpret_cast<const uint4*>(qbase + (static_cast<size_t>(b) * p.Hq + h) * D) + c);
         }
@@ -322,63 +418,56 @@ __global__ void __launch_bounds__(kThreads)
         ok = false;
         break;
       }
+      const TileSrc src = tile_src<TILE_T>(pp, t.r, j);
       uint8_t* st_ptr = smem + stage * C::STAGE_BYTES;
-      const int valid = min(TILE_T, span.tok1 - (span.tok0 + j * TILE_T));
+      const int valid = min(TILE_T, src.tok1 - src.tok0);
       if (valid < TILE_T) zero_tail_rows<C>(st_ptr, valid, lane);
-      acc.tile(smem_addr(st_ptr), valid, sl2, lane);
+      if (is_group)
+        acc.template tile<true>(smem_addr(st_ptr), valid, sl2, lane, src.row_lo, src.row_hi);
+      else
+        acc.tile(smem_addr(st_ptr), valid, sl2, lane);
       __syncwarp();
       if (i + SPW < cnt) issue(i + SPW);
     }
     if (!ok) break;
     acc.reduce_l();
     const bool complete = (gpos == ubeg) && (pend == uend);
-    const bool plain = !is_group && group_of(pp, t.r - NG, false) < 0;
-    if (complete && plain) {
-      const size_t head0 = static_cast<size_t>(t.r - NG) * p.Hq + static_cast<size_t>(t.kvh) * G;
+    if (complete) {
       const float inv_lo = 1.f / acc.l_lo, inv_hi = 1.f / acc.l_hi;
+      int b0, h0, b1, h1;
+      row_target(pp, t.r, t.kvh, g, b0, h0);
+      row_target(pp, t.r, t.kvh, g + 8, b1, h1);
 #pragma unroll
       for (int jn = 0; jn < C::NT; ++jn) {
-        if (g < G)
-          *reinterpret_cast<uint32_t*>(out + (head0 + g) * D + 8 * jn + 2 * tig) =
+        if (g < nrows)
+          *reinterpret_cast<uint32_t*>(out + (static_cast<size_t>(b0) * p.Hq + h0) * D + 8 * jn + 2 * tig) =
               pack_bf16x2(acc.o_lo[jn][0] * inv_lo, acc.o_lo[jn][1] * inv_lo);
-        if (g + 8 < G)
-          *reinterpret_cast<uint32_t*>(out + (head0 + g + 8) * D + 8 * jn + 2 * tig) =
+        if (g + 8 < nrows)
+          *reinterpret_cast<uint32_t*>(out + (static_cast<size_t>(b1) * p.Hq + h1) * D + 8 * jn + 2 * tig) =
               pack_bf16x2(acc.o_hi[jn][0] * inv_hi, acc.o_hi[jn][1] * inv_hi);
       }
     } else {
-      // partial: the unit's own buffer when complete, else a stream slot
-      size_t row0;
-      float* ml;
-      float* oacc;
-      if (complete) {
-        row0 = static_cast<size_t>(u) * kRows;
-        ml = pp.fml;
-        oacc = pp.facc;
+      const int slot = gpos == beg ? 0 : 1;  // a cut piece is the stream's first or last
+      const size_t row0 = (static_cast<size_t>(s) * 2 + slot) * kRows;
+      if (slot == 0) {
+        unit_a = u;
+        a_starts = gpos == ubeg ? 1 : 0;
       } else {
-        const int slot = gpos == beg ? 0 : 1;
-        row0 = (static_cast<size_t>(s) * 2 + slot) * kRows;
-        ml = pp.pml;
-        oacc = pp.pacc;
-        if (slot == 0) {
-          unit_a = u;
-          a_starts = gpos == ubeg ? 1 : 0;
-        } else {
-          unit_b = u;
-        }
+        unit_b = u;
       }
       if (tig == 0) {
         if (g < nrows)
-          *reinterpret_cast<float2*>(ml + (row0 + g) * 2) = make_float2(acc.m_lo, acc.l_lo);
+          *reinterpret_cast<float2*>(pp.pml + (row0 + g) * 2) = make_float2(acc.m_lo, acc.l_lo);
         if (g + 8 < nrows)
-          *reinterpret_cast<float2*>(ml + (row0 + g + 8) * 2) = make_float2(acc.m_hi, acc.l_hi);
+          *reinterpret_cast<float2*>(pp.pml + (row0 + g + 8) * 2) = make_float2(acc.m_hi, acc.l_hi);
       }
 #pragma unroll
       for (int jn = 0; jn < C::NT; ++jn) {
         if (g < nrows)
-          *reinterpret_cast<float2*>(oacc + (row0 + g) * D + 8 * jn + 2 * tig) =
+          *reinterpret_cast<float2*>(pp.pacc + (row0 + g) * D + 8 * jn + 2 * tig) =
               make_float2(acc.o_lo[jn][0], acc.o_lo[jn][1]);
         if (g + 8 < nrows)
-          *reinterpret_cast<float2*>(oacc + (row0 + g + 8) * D + 8 * jn + 2 * tig) =
+          *reinterpret_cast<float2*>(pp.pacc + (row0 + g + 8) * D + 8 * jn + 2 * tig) =
               make_float2(acc.o_hi[jn][0], acc.o_hi[jn][1]);
       }
     }
@@ -396,11 +485,12 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
-// Merge the pieces of units cut by a stream boundary (as in decode_stream.cu).  An
-// ungrouped sequence's unit goes straight to the output; a group unit or a grouped
-// sequence's unit becomes that unit's partial in the per-unit buffer.
+// Merge the pieces of units cut by a stream boundary (as in decode_stream.cu) and write
+// the outputs of their rows.  A piece that holds no tile of a row has max -inf and is
+// skipped for that row.
 template <int D>
 __global__ void __launch_bounds__(512) prefix_cut_reduce_kernel(const PrefixParams pp) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const DecodeParams& p = pp.d;
   const int s = blockIdx.x;
   const int4 m = *reinterpret_cast<const int4*>(pp.meta + static_cast<size_t>(s) * 4);
@@ -426,11 +516,8 @@ __global__ void __launch_bounds__(512) prefix_cut_reduce_kernel(const PrefixPara
     }
     n += 32;
   }
-  const int G = p.G;
   const int r = u / p.Hkv, kvh = u - r * p.Hkv;
-  const bool is_group = r < pp.ngroups;
-  const int nrows = is_group ? group_size(pp, r) * G : G;
-  const bool plain = !is_group && group_of(pp, r - pp.ngroups, false) < 0;
+  const int nrows = r < pp.ngroups ? group_size(pp, r) * p.G : p.G;
   const int row = threadIdx.x / (D / 4);
   const int c = (threadIdx.x % (D / 4)) * 4;
   if (row >= nrows) return;
@@ -440,6 +527,7 @@ __global__ void __launch_bounds__(512) prefix_cut_reduce_kernel(const PrefixPara
     const size_t pr = (static_cast<size_t>(s + i) * 2 + (i == 0 ? slot : 0)) * kRows + row;
     const float2 ml = *reinterpret_cast<const float2*>(pp.pml + pr * 2);
     const float4 a = *reinterpret_cast<const float4*>(pp.pacc + pr * D + c);
+    if (ml.x == -INFINITY) continue;
     const float Mn = fmaxf(M, ml.x);
     const float so = exp2f(M - Mn), sn = exp2f(ml.x - Mn);
     l = l * so + ml.y * sn;
@@ -449,60 +537,13 @@ __global__ void __launch_bounds__(512) prefix_cut_reduce_kernel(const PrefixPara
     a3 = a3 * so + a.w * sn;
     M = Mn;
   }
-  if (plain) {
-    const int b = r - pp.ngroups;
-    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) +
-                       (static_cast<size_t>(b) * p.Hq + static_cast<size_t>(kvh) * G + row) * D + c;
-    const float inv = 1.f / l;
-    *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf16x2(a0 * inv, a1 * inv),
-                                              pack_bf16x2(a2 * inv, a3 * inv));
-  } else {
-    const size_t fr = static_cast<size_t>(u) * kRows + row;
-    if (c == 0) *reinterpret_cast<float2*>(pp.fml + fr * 2) = make_float2(M, l);
-    *reinterpret_cast<float4*>(pp.facc + fr * D + c) = make_float4(a0, a1, a2, a3);
-  }
-}
-
-// out[b][h] for every grouped sequence b = merge(group partial, own partial).
-template <int D>
-__global__ void __launch_bounds__(256) prefix_merge_kernel(const PrefixParams pp) {
-  const DecodeParams& p = pp.d;
-  const int b = blockIdx.x;
-  const int grp = group_of(pp, b, false);
-  if (grp < 0) return;
-  const int L = clamp_len(p, b, false);
-  if (L == 0) return;
-  int mpos = 0;
-  for (int m = 0; m < pp.max_members; ++m)
-    if (__ldg(pp.group_members + static_cast<size_t>(grp) * pp.max_members + m) == b) mpos = m;
-  const int pre = __ldg(pp.group_prefix + grp);
-  const bool has_own = L > pre;
-  const int G = p.G;
-  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + static_cast<size_t>(b) * p.Hq * D;
-  for (int idx = threadIdx.x; idx < p.Hq * (D / 4); idx += blockDim.x) {
-    const int h = idx / (D / 4), c = (idx % (D / 4)) * 4;
-    const int kvh = h / G, gh = h - kvh * G;
-    const size_t gr = (static_cast<size_t>(grp) * p.Hkv + kvh) * kRows + mpos * G + gh;
-    const float2 ga = *reinterpret_cast<const float2*>(pp.fml + gr * 2);
-    const float4 gacc = *reinterpret_cast<const float4*>(pp.facc + gr * D + c);
-    float M = ga.x, l = ga.y;
-    float a0 = gacc.x, a1 = gacc.y, a2 = gacc.z, a3 = gacc.w;
-    if (has_own) {
-      const size_t sr = (static_cast<size_t>(pp.ngroups + b) * p.Hkv + kvh) * kRows + gh;
-      const float2 sa = *reinterpret_cast<const float2*>(pp.fml + sr * 2);
-      const float4 sacc = *reinterpret_cast<const float4*>(pp.facc + sr * D + c);
-      const float Mn = fmaxf(M, sa.x);
-      const float so = exp2f(M - Mn), sn = exp2f(sa.x - Mn);
-      l = l * so + sa.y * sn;
-      a0 = a0 * so + sacc.x * sn;
-      a1 = a1 * so + sacc.y * sn;
-      a2 = a2 * so + sacc.z * sn;
-      a3 = a3 * so + sacc.w * sn;
-    }
-    const float inv = 1.f / l;
-    *reinterpret_cast<uint2*>(o + static_cast<size_t>(h) * D + c) =
-        make_uint2(pack_bf16x2(a0 * inv, a1 * inv), pack_bf16x2(a2 * inv, a3 * inv));
-  }
+  int b, h;
+  row_target(pp, r, kvh, row, b, h);
+  if (b < 0 || b >= p.B) return;
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + (static_cast<size_t>(b) * p.Hq + h) * D + c;
+  const float inv = 1.f / l;
+  *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf16x2(a0 * inv, a1 * inv),
+                                            pack_bf16x2(a2 * inv, a3 * inv));
 }
 
 template <class C>
@@ -525,17 +566,29 @@ cudaError_t launch_pref_cfg(PrefixParams pp, int grid, cudaStream_t stream) {
   if (!make_pool_map(&tmk, p.k_pool, p.num_blocks, C::BS, p.Hkv, C::D) ||
       !make_pool_map(&tmv, p.v_pool, p.num_blocks, C::BS, p.Hkv, C::D))
     return cudaErrorInvalidValue;
+  prefix_plan_kernel<C::TILE_T><<<1, kPlanThreads, 0, stream>>>(pp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   const size_t smem = pref_smem_bytes<C>(pp.ngroups + p.B);
-  cudaError_t e = cudaFuncSetAttribute(decode_prefix_kernel<C>,
+  e = cudaFuncSetAttribute(decode_prefix_kernel<C>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  decode_prefix_kernel<C><<<grid, kThreads, smem, stream>>>(tmk, tmv, pp);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  prefix_cut_reduce_kernel<C::D><<<pp.streams, kRows * C::D / 4, 0, stream>>>(pp);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  prefix_merge_kernel<C::D><<<p.B, 256, 0, stream>>>(pp);
-  return cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if ((e = cudaLaunchKernelEx(&cfg, decode_prefix_kernel<C>, tmk, tmv, pp)) != cudaSuccess) return e;
+  cfg.gridDim = dim3(static_cast<unsigned>(pp.streams));
+  cfg.blockDim = dim3(kRows * C::D / 4);
+  cfg.dynamicSmemBytes = 0;
+  return cudaLaunchKernelEx(&cfg, prefix_cut_reduce_kernel<C::D>, pp);
 }
 
 }  // namespace
@@ -558,14 +611,14 @@ int prefix_grid(int D, int block_size, int R) {
 
 int prefix_warps_per_cta() { return kNCW; }
 
-size_t prefix_workspace_bytes(int streams, int units, int D) {
+size_t prefix_workspace_bytes(int streams, int rows, int D) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   return up(static_cast<size_t>(streams) * 16) + up(static_cast<size_t>(streams) * 2 * kRows * 8) +
          up(static_cast<size_t>(streams) * 2 * kRows * D * 4) +
-         up(static_cast<size_t>(units) * kRows * 8) + static_cast<size_t>(units) * kRows * D * 4;
+         static_cast<size_t>(rows + 1) * 4;
 }
 
-void prefix_carve(PrefixParams* pp, void* workspace, int units) {
+void prefix_carve(PrefixParams* pp, void* workspace, int rows) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   char* w = static_cast<char*>(workspace);
   const int D = pp->d.D;
@@ -575,9 +628,8 @@ void prefix_carve(PrefixParams* pp, void* workspace, int units) {
   w += up(static_cast<size_t>(pp->streams) * 2 * kRows * 8);
   pp->pacc = reinterpret_cast<float*>(w);
   w += up(static_cast<size_t>(pp->streams) * 2 * kRows * D * 4);
-  pp->fml = reinterpret_cast<float*>(w);
-  w += up(static_cast<size_t>(units) * kRows * 8);
-  pp->facc = reinterpret_cast<float*>(w);
+  pp->plan = reinterpret_cast<int32_t*>(w);
+  (void)rows;
 }
 
 cudaError_t launch_decode_prefix(const PrefixParams& pp, int grid, cudaStream_t stream) {

@@ -55,13 +55,12 @@ struct PrefixParams {
   int32_t* meta;   // [streams][4] cut-unit slot metadata
   float* pml;      // [streams][2][16][2]
   float* pacc;     // [streams][2][16][D]
-  float* fml;      // [units][16][2]: per-unit partials (group units, grouped sequences)
-  float* facc;     // [units][16][D]
+  int32_t* plan;   // [ngroups + B + 1] scanned tile counts of the unit rows
 };
 int prefix_grid(int D, int block_size, int R);
 int prefix_warps_per_cta();
-size_t prefix_workspace_bytes(int streams, int units, int D);
-void prefix_carve(PrefixParams* pp, void* workspace, int units);
+size_t prefix_workspace_bytes(int streams, int rows, int D);
+void prefix_carve(PrefixParams* pp, void* workspace, int rows);
 cudaError_t launch_decode_prefix(const PrefixParams& pp, int grid, cudaStream_t stream);
 
 // 4-D TMA view of a bf16 pool [NB][BS][Hkv][D]: box = BS rows x 64 columns of one head.

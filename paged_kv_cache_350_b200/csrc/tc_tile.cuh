@@ -129,14 +129,19 @@ struct WarpAcc {
   }
 
   // One online-softmax row update for scores x0..x3 (tokens 2tig, 2tig+1, 8+2tig, 9+2tig).
+  // A masked row takes no part in this tile: its state is kept and its P is zero.
   __device__ __forceinline__ static float row_update(float x0, float x1, float x2, float x3,
                                                      float& m, float& l, uint32_t& hi0,
                                                      uint32_t& lo0, uint32_t& hi2,
-                                                     uint32_t& lo2) {
+                                                     uint32_t& lo2, bool masked = false) {
     constexpr unsigned kFull = 0xffffffffu;
     float mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
     mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+    if (masked) {
+      hi0 = lo0 = hi2 = lo2 = 0u;
+      return 1.f;
+    }
     const float m_new = fmaxf(m, mx);
     const float alpha = exp2f(m - m_new);
     m = m_new;
@@ -150,8 +155,10 @@ struct WarpAcc {
 
   // Consume one staged tile (K at kbase, V at kbase + TILE_BYTES, shared addresses) with
   // `valid` tokens (1..TILE_T) inside the sequence; rows >= valid are masked (their V rows
-  // must already be zero).
-  __device__ __forceinline__ void tile(uint32_t kbase, int valid, float sl2, int lane) {
+  // must already be zero).  With ROWMASK only query rows [row_lo, row_hi) take part.
+  template <bool ROWMASK = false>
+  __device__ __forceinline__ void tile(uint32_t kbase, int valid, float sl2, int lane,
+                                       int row_lo = 0, int row_hi = 16) {
     const uint32_t vbase = kbase + C::TILE_BYTES;
     const int tig = lane & 3;
     const int mi = lane >> 3, mr = lane & 7;
@@ -180,15 +187,18 @@ struct WarpAcc {
       const bool v2 = 8 + 2 * tig < lim, v3 = 9 + 2 * tig < lim;
       uint32_t pa0, pa1 = 0u, pa2, pa3 = 0u;   // P hi parts (A fragment registers)
       uint32_t pr0, pr1 = 0u, pr2, pr3 = 0u;   // P lo parts
+      const int gr = lane >> 2;
+      const bool mask_lo = ROWMASK && (gr < row_lo || gr >= row_hi);
+      const bool mask_hi = ROWMASK && (gr + 8 < row_lo || gr + 8 >= row_hi);
       const float alpha_lo =
           row_update(v0 ? s0[0] * sl2 : -INFINITY, v1 ? s0[1] * sl2 : -INFINITY,
                      v2 ? s1[0] * sl2 : -INFINITY, v3 ? s1[1] * sl2 : -INFINITY, m_lo, l_lo,
-                     pa0, pr0, pa2, pr2);
+                     pa0, pr0, pa2, pr2, mask_lo);
       float alpha_hi = 1.f;
       if constexpr (C::ROWS16)
         alpha_hi = row_update(v0 ? s0[2] * sl2 : -INFINITY, v1 ? s0[3] * sl2 : -INFINITY,
                               v2 ? s1[2] * sl2 : -INFINITY, v3 ? s1[3] * sl2 : -INFINITY, m_hi,
-                              l_hi, pa1, pr1, pa3, pr3);
+                              l_hi, pa1, pr1, pa3, pr3, mask_hi);
 #pragma unroll
       for (int j = 0; j < C::NT; ++j) {
         o_lo[j][0] *= alpha_lo;
