@@ -4,8 +4,10 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config gqa] [--impl ours|reference]
 
 One step = one decode step of the whole hot path over one synthetic batch:
-copy-on-write block copies (when the step has any), reshape_and_cache of the
-step's new K/V, and pa_decode (plus its split-context reduce).  The allocator's
+copy-on-write block copies (when the step has any), then pa_decode_append: the
+step's new K/V written to their slots (reshape_and_cache, fused into the decode
+kernel) and the decode attention (plus its reduce).  ``--unfused`` runs
+pa_reshape_and_cache and pa_decode as two calls instead.  The allocator's
 slot mapping, copy pairs, tables and lengths for the step are computed on the
 host before timing and are resident in HBM; the timed steps repeat the same
 step (the cache writes are idempotent), over pools larger than the 126 MB L2.
@@ -13,9 +15,10 @@ step (the cache writes are idempotent), over pools larger than the 126 MB L2.
 Prints ONE JSON line (rank 0).  ``value`` = algorithmic KV bytes of pa_decode
 per step x steps x ranks / max-over-ranks device time, in GB/s (the whole step
 is in the denominator).  ``e2e`` = the same metric through
-``PagedKVCache.step`` with host buffers: allocator, host->device copies,
-kernels, device->host copy of the output, per step.  ``roofline`` is pa_decode
-alone against the measured HBM copy bandwidth.
+``PagedKVCache.step_staged`` with host buffers: allocator, host->device copy,
+kernels, device->host copy of the output, per step.  ``roofline`` is the decode
+call alone (pa_decode_append, or pa_decode with ``--unfused``) against the
+measured HBM copy bandwidth.
 
 With ``--impl reference`` the float64 CPU oracle is timed instead, on a
 bounded sample of the same workload per step.
@@ -75,6 +78,8 @@ def parse_args(argv=None):
                     help="decode with pa_decode_shared_prefix (fork groups read shared blocks once)")
     ap.add_argument("--block-size", type=int, default=0,
                     help="override the workload's block size (8, 16 or 32) for a sweep")
+    ap.add_argument("--unfused", action="store_true",
+                    help="pa_reshape_and_cache + pa_decode as two calls (default: pa_decode_append)")
     return ap.parse_args(argv)
 
 
@@ -109,15 +114,16 @@ def decode_kernel_hash():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(config):
-    """DRAM bytes per pa_decode launch from a committed ncu summary, if the kernel is unchanged."""
+def recorded_traffic(config, call):
+    """DRAM bytes per call from a committed ncu summary, if it covers this call and the kernel
+    sources are unchanged."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f).get(config)
     except Exception:
         return None
-    if not rec or rec.get("kernel_hash") != decode_kernel_hash():
+    if not rec or rec.get("call") != call or rec.get("kernel_hash") != decode_kernel_hash():
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -349,7 +355,11 @@ def run_ours(args):
     plan = pa.pa_decode_plan(w.B, w.Hq, w.Hkv, w.D, w.block_size, MB, dtype_pa, nws)
     npairs = int(pairs.shape[0])
     stream = torch.cuda.current_stream(device)
-    launches_per_step = plan["launches"] + 1 + (1 if npairs else 0)
+    fused = not (args.unfused or args.shared_prefix)
+    # the fused call adds an append kernel only on the paths whose decode kernel does
+    # not write the token itself
+    append_launch = 1 if (not fused or plan["kernel"] != pa.binding.PA_KERNEL_TC_STREAM) else 0
+    launches_per_step = plan["launches"] + append_launch + (1 if npairs else 0)
     unique_kv = None
     if args.shared_prefix:
         maxm = max(1, 16 // (w.Hq // w.Hkv))
@@ -369,6 +379,14 @@ def run_ours(args):
     def step(ev=None):
         if npairs:
             pa.pa_copy_blocks(kp, vp, pairs_d, err_flag=err, stream=stream)
+        if fused:
+            if ev is not None:
+                ev[0].record(stream)
+            pa.pa_decode_append(out, q, nk, nv, kp, vp, tables_d, lens_d, w.scale, workspace=ws,
+                                err_flag=err, stream=stream)
+            if ev is not None:
+                ev[1].record(stream)
+            return
         pa.pa_reshape_and_cache(nk, nv, kp, vp, slots_d, err_flag=err, stream=stream)
         if ev is not None:
             ev[0].record(stream)
@@ -413,6 +431,10 @@ def run_ours(args):
     peak, peak_src = measured_peak()
     # bytes that must cross HBM: with shared prefixes, each group's shared tokens once
     roof_bytes = alg_bytes if unique_kv is None else alg_bytes - kv_bytes + unique_kv
+    # the fused call also writes each row's new K/V to its slot (its read replaces the
+    # read of that slot, already counted in the decode bytes)
+    append_bytes = 2 * w.B * w.Hkv * w.D * esize if fused else 0
+    roof_bytes += append_bytes
     achieved = roof_bytes / (dec_avg_ms / 1e3) / 1e9
 
     # ---- end to end through PagedKVCache.step with host buffers -------------------
@@ -469,6 +491,9 @@ def run_ours(args):
             "num_blocks": w.num_blocks, "mean_seq_len": float(np.mean(lens)),
             "kv_bytes_per_step": kv_bytes, "alg_bytes_per_step": alg_bytes,
             "copy_pairs_per_step": npairs, "decode_plan": plan,
+            "step_calls": ("pa_copy_blocks + " if npairs else "") + (
+                "pa_decode_append" if fused else "pa_reshape_and_cache + " + (
+                    "pa_decode_shared_prefix" if args.shared_prefix else "pa_decode")),
             "internal_waste_slots": int(alloc.internal_waste_slots()),
             "kv_bytes_unique_per_step": unique_kv,
             "l2": "inputs larger than L2 (K/V pools of %.2f GB vs 126 MB L2); not flushed"
@@ -478,8 +503,13 @@ def run_ours(args):
         "decode_tokens_per_s": tokens_per_s,
         "kernel_kv_gbs": alg_bytes / (dec_avg_ms / 1e3) / 1e9,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": recorded_traffic(args.config),
-                     "kernel": "pa_decode call (main kernel + its reduce), CUDA events per call",
+                     "frac": achieved / peak,
+                     "traffic": recorded_traffic(args.config, "pa_decode_append" if fused
+                                                 else "pa_decode"),
+                     "kernel": ("pa_decode_append call (decode kernel with the fused cache "
+                                "write + its reduce)" if fused else "pa_decode call (main kernel "
+                                "+ its reduce)") + ", CUDA events per call",
+                     "append_bytes_per_call": append_bytes,
                      "peak_source": f"{peak_src} HBM copy bandwidth (burst)"},
         "cpu_baseline": cpu,
         "e2e": e2e,

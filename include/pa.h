@@ -12,6 +12,8 @@
  *                        ("什么是分页注意力", 边界与常见误解): for query head h of
  *                        sequence b, o = softmax(scale * q.K^T) V over the sequence's
  *                        tokens.
+ *   pa_decode_append     pa_reshape_and_cache of the step's tokens and pa_decode in one
+ *                        call; the balanced decode kernel writes the tokens itself.
  *   pa_reshape_and_cache Scatter the step's new K/V rows into their slots (each step
  *                        computes one key and value per token and caches them:
  *                        "什么是 LLM 中的分页注意力", 快速回顾:KV 缓存; slot addressing
@@ -169,6 +171,31 @@ pa_status pa_decode_ex(void* out, const void* q, const void* k_pool, const void*
                        int Hkv, int D, int block_size, int max_blocks, int num_blocks,
                        float scale, pa_dtype dtype, void* workspace, size_t workspace_bytes,
                        int32_t* dev_err_flag, pa_stream_t stream, const pa_decode_opts* opts);
+
+/* One decode step with the cache write fused in.  For every row b with L = seq_lens[b]
+ * >= 1, position L-1 is the step's token: its key and value (k_new[b], v_new[b], each
+ * [B][Hkv][D] in the pools' dtype, 16-byte aligned) are written to slot
+ * block_tables[b][(L-1) / block_size] * block_size + (L-1) % block_size of the pools
+ * (a new token fills the next free slot of the sequence's current block: "什么是 LLM
+ * 中的分页注意力", 使用分页注意力), and out is pa_decode over positions 0 .. L-1 with
+ * that token included.  The result, out and pools, is the same as pa_reshape_and_cache
+ * with those slots followed by pa_decode_ex.  Rows with L = 0 write nothing (zero
+ * output row); a row whose length is out of range or whose table entry is outside
+ * [0, num_blocks) writes nothing and raises its PA_DEVERR_* bit.
+ *   - The block receiving row b's token must not be read by another row of the call
+ *     (the allocator's copy-on-write guarantees this); such a row could see the old or
+ *     the new values.
+ *   - The balanced tensor-core kernel writes the token itself (the step is that
+ *     kernel and its reduce); the other kernels run after a one-launch append kernel,
+ *     so pa_decode_plan's `launches` is one more for them.
+ * Arguments, workspace and options otherwise as pa_decode_ex. */
+pa_status pa_decode_append(void* out, const void* q, const void* k_new, const void* v_new,
+                           void* k_pool, void* v_pool, const int32_t* block_tables,
+                           const int32_t* seq_lens, int B, int Hq, int Hkv, int D,
+                           int block_size, int max_blocks, int num_blocks, float scale,
+                           pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                           int32_t* dev_err_flag, pa_stream_t stream,
+                           const pa_decode_opts* opts);
 
 /* Decode for a batch in which groups of sequences share their leading blocks: samples
  * forked from one prompt, or requests with a common system prompt ("深入解析 PagedAttention",

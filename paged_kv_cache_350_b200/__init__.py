@@ -3,7 +3,8 @@
 The product is the C-ABI library ``libpagedattn.so`` (``include/pa.h``): batched
 single-token decode attention that reads K/V from a block pool through
 per-sequence block tables, the two kernels that keep the pool consistent
-(``reshape_and_cache``, ``copy_blocks``), and a host block allocator with
+(``reshape_and_cache``, ``copy_blocks``; ``pa_decode_append`` fuses the first into
+the decode), and a host block allocator with
 reference counts.  This package is its Python face: ``binding`` marshals torch
 tensors into the C calls (same names), ``cache.PagedKVCache`` chains one decode
 step end to end, and ``build`` compiles the library in-tree.
@@ -16,6 +17,7 @@ imports without it.
 _BINDING_NAMES = {
     "PA_BF16", "PA_F32", "PA_PATH_AUTO", "PA_PATH_GENERIC", "PA_PATH_TENSOR", "PAError",
     "Allocator", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_size", "pa_decode_plan", "pa_decode_no_alloc",
+    "pa_decode_append",
     "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_size",
     "pa_reshape_and_cache", "pa_status_from_device_flag", "lib",
 }

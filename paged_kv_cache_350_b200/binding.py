@@ -91,6 +91,9 @@ def _load():
                             vp, sz, vp, vp]),
         "pa_decode_ex": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, f32,
                                i32, vp, sz, vp, vp, ctypes.POINTER(pa_decode_opts)]),
+        "pa_decode_append": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                   i32, f32, i32, vp, sz, vp, vp,
+                                   ctypes.POINTER(pa_decode_opts)]),
         "pa_decode_plan": (i32, [i32, i32, i32, i32, i32, i32, i32, sz,
                                  ctypes.POINTER(pa_decode_opts), ctypes.POINTER(pa_decode_plan_info)]),
         "pa_decode_shared_prefix_workspace_size": (sz, [i32, i32, i32, i32, i32, i32]),
@@ -132,7 +135,7 @@ lib = _load()
 #: every symbol include/pa.h declares
 EXPORTED = (
     "pa_status_string", "pa_status_from_device_flag", "pa_version", "pa_decode_workspace_size",
-    "pa_decode", "pa_decode_ex", "pa_decode_plan", "pa_decode_no_alloc",
+    "pa_decode", "pa_decode_ex", "pa_decode_append", "pa_decode_plan", "pa_decode_no_alloc",
     "pa_decode_shared_prefix_workspace_size", "pa_decode_shared_prefix", "pa_alloc_prefix_groups",
     "pa_reshape_and_cache", "pa_copy_blocks", "pa_alloc_create",
     "pa_alloc_create_ordered", "pa_alloc_destroy", "pa_alloc_add_seq", "pa_alloc_fork",
@@ -217,6 +220,35 @@ def pa_decode(out, q, k_pool, v_pool, block_tables, seq_lens, scale, workspace=N
                           float(scale), _dtype_of(q), _ptr(workspace), wbytes, _ptr(err_flag),
                           _stream(stream), ctypes.byref(opts))
     _check(st, "pa_decode")
+    return out
+
+
+def pa_decode_append(out, q, k_new, v_new, k_pool, v_pool, block_tables, seq_lens, scale,
+                     workspace=None, err_flag=None, stream=None, partition_tokens=0,
+                     path=PA_PATH_AUTO, max_ctas=0):
+    """One decode step with the cache write fused: k_new/v_new[B,Hkv,D] go to position
+    seq_lens[b]-1 of each row's table, then out = pa_decode (see include/pa.h)."""
+    import torch
+    _need(q.dim() == 3 and out.shape == q.shape, "q/out must be [B, Hq, D]")
+    _need(k_pool.dim() == 4 and v_pool.shape == k_pool.shape, "pools must be [NB, bs, Hkv, D]")
+    _need(block_tables.dim() == 2 and block_tables.dtype == torch.int32, "block_tables int32 [B, MB]")
+    _need(seq_lens.dtype == torch.int32 and seq_lens.numel() == q.shape[0], "seq_lens int32 [B]")
+    B, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_pool.shape
+    _need(D2 == D and block_tables.shape[0] == B, "shape mismatch")
+    _need(k_new.shape == (B, Hkv, D) and v_new.shape == k_new.shape, "k_new/v_new must be [B, Hkv, D]")
+    for t in (out, q, k_new, v_new, k_pool, v_pool, block_tables, seq_lens):
+        _need(t.is_contiguous(), "tensors must be contiguous")
+    _need(q.dtype == out.dtype == k_new.dtype == v_new.dtype == k_pool.dtype == v_pool.dtype,
+          "q, out, new K/V and pools share a dtype")
+    wbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    opts = pa_decode_opts(partition_tokens, path, max_ctas)
+    st = lib.pa_decode_append(_ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool),
+                              _ptr(v_pool), _ptr(block_tables), _ptr(seq_lens), B, Hq, Hkv, D, bs,
+                              block_tables.shape[1], NB, float(scale), _dtype_of(q),
+                              _ptr(workspace), wbytes, _ptr(err_flag), _stream(stream),
+                              ctypes.byref(opts))
+    _check(st, "pa_decode_append")
     return out
 
 

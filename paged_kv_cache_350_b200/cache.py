@@ -9,7 +9,9 @@ in host memory:
    pairs for partial blocks that are still shared;
 2. ``pa_alloc_block_tables`` (C, host): padded tables and lengths;
 3. host→device copies of those and of q / new K / new V (pinned staging);
-4. ``pa_copy_blocks`` → ``pa_reshape_and_cache`` → ``pa_decode`` on the stream;
+4. ``pa_copy_blocks`` (when a shared partial block is appended to), then
+   ``pa_decode_append``: the decode kernel itself writes each sequence's new K/V at
+   its last position (the slot the allocator reserved) and attends;
 5. device→host copy of the output, then a stream synchronise.
 
 Everything between the copies runs in the library's kernels.
@@ -88,13 +90,13 @@ class PagedKVCache:
             q = self._dev(("q",), q_host.shape, self.dtype)
             kn = self._dev(("k",), k_host.shape, self.dtype)
             vn = self._dev(("v",), v_host.shape, self.dtype)
-            slots = self._dev(("slots",), (B,), torch.int64)
             tables = self._dev(("tables",), (B, max_blocks), torch.int32)
             lens = self._dev(("lens",), (B,), torch.int32)
             out = self._dev(("out",), q_host.shape, self.dtype)
             h2d = 0
-            for dst, src in ((q, q_host), (kn, k_host), (vn, v_host), (slots, slots_h),
-                             (tables, tables_h), (lens, lens_h)):
+            # the slots stay on the host: the kernel derives them from tables and lengths
+            for dst, src in ((q, q_host), (kn, k_host), (vn, v_host), (tables, tables_h),
+                             (lens, lens_h)):
                 dst.copy_(src, non_blocking=True)
                 h2d += src.numel() * src.element_size()
             if npairs:
@@ -103,11 +105,9 @@ class PagedKVCache:
                 h2d += npairs * 8
                 _b.pa_copy_blocks(self.k_pool, self.v_pool, pairs_d[:npairs], err_flag=self.err,
                                   stream=stream)
-            _b.pa_reshape_and_cache(kn, vn, self.k_pool, self.v_pool, slots, err_flag=self.err,
-                                    stream=stream)
             ws = self.workspace(B, Hq, max_blocks)
-            _b.pa_decode(out, q, self.k_pool, self.v_pool, tables, lens, scale, workspace=ws,
-                         err_flag=self.err, stream=stream)
+            _b.pa_decode_append(out, q, kn, vn, self.k_pool, self.v_pool, tables, lens, scale,
+                                workspace=ws, err_flag=self.err, stream=stream)
             out_host.copy_(out, non_blocking=True)
         stream.synchronize()
         return h2d, out_host.numel() * out_host.element_size()
@@ -116,9 +116,10 @@ class PagedKVCache:
     def _layout(self, B, Hq, max_blocks):
         """Byte offsets of the sections of the step input buffer (256-byte aligned)."""
         esz = torch.tensor([], dtype=self.dtype).element_size()
+        # slots last: the allocator writes them but the device never reads them
         sizes = [("q", B * Hq * self.D * esz), ("k", B * self.Hkv * self.D * esz),
-                 ("v", B * self.Hkv * self.D * esz), ("slots", B * 8),
-                 ("tables", B * max_blocks * 4), ("lens", B * 4), ("pairs", B * 8)]
+                 ("v", B * self.Hkv * self.D * esz), ("tables", B * max_blocks * 4),
+                 ("lens", B * 4), ("pairs", B * 8), ("slots", B * 8)]
         off, lay = 0, {}
         for name, n in sizes:
             lay[name] = (off, n)
@@ -176,15 +177,13 @@ class PagedKVCache:
             if npairs:
                 _b.pa_copy_blocks(kp, vp, self._view(d, "pairs", (B, 2), torch.int32)[:npairs],
                                   err_flag=self.err, stream=stream)
-            _b.pa_reshape_and_cache(self._view(d, "k", (B, self.Hkv, self.D), self.dtype),
-                                    self._view(d, "v", (B, self.Hkv, self.D), self.dtype),
-                                    kp, vp, self._view(d, "slots", (B,), torch.int64),
-                                    err_flag=self.err, stream=stream)
-            _b.pa_decode(self._out_d, self._view(d, "q", (B, Hq, self.D), self.dtype), kp, vp,
-                         self._view(d, "tables", (B, max_blocks), torch.int32),
-                         self._view(d, "lens", (B,), torch.int32), scale,
-                         workspace=self.workspace(B, Hq, max_blocks), err_flag=self.err,
-                         stream=stream)
+            _b.pa_decode_append(self._out_d, self._view(d, "q", (B, Hq, self.D), self.dtype),
+                                self._view(d, "k", (B, self.Hkv, self.D), self.dtype),
+                                self._view(d, "v", (B, self.Hkv, self.D), self.dtype), kp, vp,
+                                self._view(d, "tables", (B, max_blocks), torch.int32),
+                                self._view(d, "lens", (B,), torch.int32), scale,
+                                workspace=self.workspace(B, Hq, max_blocks), err_flag=self.err,
+                                stream=stream)
             self._out_h.copy_(self._out_d, non_blocking=True)
         stream.synchronize()
         return self._out_h, (used, self._out_h.numel() * self._out_h.element_size())

@@ -172,11 +172,14 @@ pa_status pa_decode_plan(int B, int Hq, int Hkv, int D, int block_size, int max_
                      workspace_bytes, opts, info);
 }
 
-pa_status pa_decode_ex(void* out, const void* q, const void* k_pool, const void* v_pool,
-                       const int32_t* block_tables, const int32_t* seq_lens, int B, int Hq,
-                       int Hkv, int D, int block_size, int max_blocks, int num_blocks,
-                       float scale, pa_dtype dtype, void* workspace, size_t workspace_bytes,
-                       int32_t* dev_err_flag, pa_stream_t stream, const pa_decode_opts* opts) {
+// pa_decode_ex and pa_decode_append: k_new/v_new null = plain decode.
+static pa_status decode_call(void* out, const void* q, const void* k_new, const void* v_new,
+                             const void* k_pool, const void* v_pool, const int32_t* block_tables,
+                             const int32_t* seq_lens, int B, int Hq, int Hkv, int D,
+                             int block_size, int max_blocks, int num_blocks, float scale,
+                             pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                             int32_t* dev_err_flag, pa_stream_t stream,
+                             const pa_decode_opts* opts) {
   pa_decode_plan_info plan;
   const bool have_ws = workspace != nullptr && aligned(workspace, 256);
   pa_status st = plan_decode(B, Hq, Hkv, D, block_size, max_blocks, num_blocks, scale, dtype,
@@ -188,6 +191,8 @@ pa_status pa_decode_ex(void* out, const void* q, const void* k_pool, const void*
       !aligned(block_tables, 4) || !aligned(seq_lens, 4) ||
       (dev_err_flag && !aligned(dev_err_flag, 4)))
     return PA_ERR_INVALID_ARG;
+  const bool append = k_new != nullptr;
+  if (append && (!v_new || !aligned(k_new, 16) || !aligned(v_new, 16))) return PA_ERR_INVALID_ARG;
 
   pa::DecodeParams p{};
   p.out = out;
@@ -215,8 +220,21 @@ pa_status pa_decode_ex(void* out, const void* q, const void* k_pool, const void*
     sp.d = p;
     sp.streams = plan.grid * pa::stream_warps_per_cta();
     pa::stream_carve(&sp, workspace);
+    if (append) {  // the decode kernel writes the step's token itself
+      sp.k_new = k_new;
+      sp.v_new = v_new;
+      sp.k_pool_w = const_cast<void*>(k_pool);
+      sp.v_pool_w = const_cast<void*>(v_pool);
+    }
     e = pa::launch_decode_stream(sp, plan.grid, s);
   } else {
+    if (append) {
+      const int esize = dtype == PA_BF16 ? 2 : 4;
+      e = pa::launch_append_kv(k_new, v_new, const_cast<void*>(k_pool), const_cast<void*>(v_pool),
+                               block_tables, seq_lens, B, max_blocks, block_size, num_blocks,
+                               Hkv * D * esize, dev_err_flag, s);
+      if (e != cudaSuccess) return PA_ERR_CUDA;
+    }
     const int parts = plan.max_parts;
     if (parts > 1) {
       char* ws = static_cast<char*>(workspace);
@@ -228,6 +246,29 @@ pa_status pa_decode_ex(void* out, const void* q, const void* k_pool, const void*
                                                : pa::launch_decode_generic(p, dtype, s);
   }
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_decode_ex(void* out, const void* q, const void* k_pool, const void* v_pool,
+                       const int32_t* block_tables, const int32_t* seq_lens, int B, int Hq,
+                       int Hkv, int D, int block_size, int max_blocks, int num_blocks,
+                       float scale, pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                       int32_t* dev_err_flag, pa_stream_t stream, const pa_decode_opts* opts) {
+  return decode_call(out, q, nullptr, nullptr, k_pool, v_pool, block_tables, seq_lens, B, Hq,
+                     Hkv, D, block_size, max_blocks, num_blocks, scale, dtype, workspace,
+                     workspace_bytes, dev_err_flag, stream, opts);
+}
+
+pa_status pa_decode_append(void* out, const void* q, const void* k_new, const void* v_new,
+                           void* k_pool, void* v_pool, const int32_t* block_tables,
+                           const int32_t* seq_lens, int B, int Hq, int Hkv, int D,
+                           int block_size, int max_blocks, int num_blocks, float scale,
+                           pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                           int32_t* dev_err_flag, pa_stream_t stream,
+                           const pa_decode_opts* opts) {
+  if (B > 0 && (!k_new || !v_new)) return PA_ERR_INVALID_ARG;
+  return decode_call(out, q, k_new, v_new, k_pool, v_pool, block_tables, seq_lens, B, Hq, Hkv,
+                     D, block_size, max_blocks, num_blocks, scale, dtype, workspace,
+                     workspace_bytes, dev_err_flag, stream, opts);
 }
 
 pa_status pa_decode(void* out, const void* q, const void* k_pool, const void* v_pool,

@@ -1,10 +1,14 @@
-// The two kernels that keep the paged KV pool consistent (sm_100a).
+// The kernels that keep the paged KV pool consistent (sm_100a).
 //
 // reshape_and_cache: every decode step computes a key and a value for each new token
 // and caches them for later steps ("什么是 LLM 中的分页注意力", 快速回顾:KV 缓存).  In the
 // paged layout token t goes to slot s = slot_mapping[t]: block s / block_size, offset
 // s % block_size.  Because the pool is [NB][BS][Hkv][D], slot s is simply row s of the
 // pool viewed as [NB*BS][Hkv][D], so the copy is one contiguous Hkv*D row per token.
+//
+// append_kv: the same write for a decode step whose slots are implied by the tables: row
+// b's token is position seq_lens[b]-1 (pa_decode_append on the paths whose decode kernel
+// does not write it itself).
 //
 // copy_blocks: copy on write of shared blocks before a forked sequence writes into one
 // ("PagedAttention" concept card, 实现要点; "深入解析 PagedAttention", 多序列共享): whole
@@ -40,6 +44,35 @@ __global__ void reshape_and_cache_kernel(const uint4* __restrict__ key,
        i += gridDim.x * blockDim.x) {
     k_pool[dst + i] = __ldg(key + src + i);
     v_pool[dst + i] = __ldg(value + src + i);
+  }
+}
+
+// One block per batch row: the step's token is position L-1 of the row (L = seq_lens[b]),
+// so its slot is the table entry of block (L-1) / block_size at offset (L-1) % block_size
+// ("什么是 LLM 中的分页注意力", 使用分页注意力: a new token fills the next free slot of the
+// sequence's current block).  Rows with L = 0 have no token this step.
+__global__ void append_kv_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+                                 uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
+                                 const int32_t* __restrict__ block_tables,
+                                 const int32_t* __restrict__ seq_lens, int max_blocks,
+                                 int block_size, int num_blocks, int vec_per_row, int32_t* err) {
+  const int b = blockIdx.x;
+  const int L = __ldg(seq_lens + b);
+  if (L == 0) return;
+  if (L < 0 || static_cast<int64_t>(L) > static_cast<int64_t>(max_blocks) * block_size) {
+    if (threadIdx.x == 0) flag_error(err, PA_DEVERR_BAD_SEQ_LEN);
+    return;
+  }
+  const int phys = __ldg(block_tables + static_cast<int64_t>(b) * max_blocks + (L - 1) / block_size);
+  if (phys < 0 || phys >= num_blocks) {
+    if (threadIdx.x == 0) flag_error(err, PA_DEVERR_BAD_BLOCK_ID);
+    return;
+  }
+  const int64_t src = static_cast<int64_t>(b) * vec_per_row;
+  const int64_t dst = (static_cast<int64_t>(phys) * block_size + (L - 1) % block_size) * vec_per_row;
+  for (int i = threadIdx.x; i < vec_per_row; i += blockDim.x) {
+    k_pool[dst + i] = __ldg(k_new + src + i);
+    v_pool[dst + i] = __ldg(v_new + src + i);
   }
 }
 
@@ -92,6 +125,20 @@ cudaError_t launch_reshape_and_cache(const void* key, const void* value, void* k
       static_cast<const uint4*>(key), static_cast<const uint4*>(value),
       static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), slot_mapping, vec, num_slots,
       err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append_kv(const void* k_new, const void* v_new, void* k_pool, void* v_pool,
+                             const int32_t* block_tables, const int32_t* seq_lens, int B,
+                             int max_blocks, int block_size, int num_blocks, int row_bytes,
+                             int32_t* err, cudaStream_t stream) {
+  if (B <= 0) return cudaSuccess;
+  const int vec = row_bytes / 16;
+  const int threads = vec < 256 ? ((vec + 31) / 32) * 32 : 256;
+  append_kv_kernel<<<B, threads, 0, stream>>>(
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
+      static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), block_tables, seq_lens,
+      max_blocks, block_size, num_blocks, vec, err);
   return cudaGetLastError();
 }
 

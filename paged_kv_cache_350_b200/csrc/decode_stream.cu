@@ -22,6 +22,8 @@
 //     cut by a range boundary leaves a partial (max, sum, unnormalised O) in one of the
 //     stream's two slots; the reduce kernel merges the pieces of each cut unit by
 //     log-sum-exp.  Each stream records which units its slots hold every launch.
+//   * pa_decode_append fuses the step's cache write: the stream that consumes a unit's
+//     last tile writes the new token's K/V to its slot and into the staged tile.
 
 #include <cudaTypedefs.h>
 
@@ -132,6 +134,28 @@ __device__ __forceinline__ TileIds resolve_tile(const DecodeParams& p, const int
   for (int k = 0; k < C::BPS; ++k)
     if (k < r.nb) r.id[k] = __ldg(tab + k);
   return r;
+}
+
+// Fused cache write of pa_decode_append: put the step's token (K and V, one 16-byte chunk
+// per lane in `v`: lanes [0, D/8) K, [D/8, D/4) V) into row r of the staged tile, and into
+// its slot (block `phys`, offset `off`, KV head `kvh`) of the pools.  The tile was loaded
+// from the pool before the write, so the staged row is replaced here; the proxy fence
+// orders these shared writes before the next TMA write to the stage.
+template <class C>
+__device__ __forceinline__ void put_token(uint8_t* stage_ptr, int r, const uint4& v, int phys,
+                                          int off, int kvh, const StreamParams& sp, int lane) {
+  constexpr int VPR = C::D / 8;  // 16-byte chunks per head row
+  if (lane < 2 * VPR) {
+    const int which = lane / VPR, ch = lane % VPR;
+    *reinterpret_cast<uint4*>(stage_ptr + which * C::TILE_BYTES + (ch >> 3) * C::CHUNK_BYTES +
+                              sw128(r, ch & 7)) = v;
+    fence_proxy_async_smem();
+    if (phys >= 0 && phys < sp.d.num_blocks) {  // a bad id was flagged when the tile was loaded
+      uint4* pool = static_cast<uint4*>(which ? sp.v_pool_w : sp.k_pool_w);
+      pool[((static_cast<size_t>(phys) * C::BS + off) * sp.d.Hkv + kvh) * VPR + ch] = v;
+    }
+  }
+  __syncwarp();
 }
 
 template <class C>
@@ -260,6 +284,8 @@ __global__ void __launch_bounds__(kThreads, PA_STREAM_MIN_CTAS)
 
   const int g = lane >> 2, tig = lane & 3;
   const float sl2 = p.scale_log2;
+  const bool append = sp.k_new != nullptr;
+  constexpr int VPR = D / 8;
   int unit_a = -1, a_starts = 0, unit_b = -1;
   int i = 0;  // tiles consumed by this stream (ring position)
   bool ok = true;
@@ -274,6 +300,19 @@ __global__ void __launch_bounds__(kThreads, PA_STREAM_MIN_CTAS)
     const int uend = ubeg + t.nt;
     const int pend = min(end, uend);
     const size_t head0 = static_cast<size_t>(t.b) * p.Hq + static_cast<size_t>(t.kvh) * G;
+    // pa_decode_append: the step's token is position L-1, in the unit's last tile.  The
+    // stream that owns that tile fetches the token's K/V now and writes them when the
+    // tile has landed (not for a length that was clamped as out of range).
+    bool put = false;
+    uint4 put_kv = make_uint4(0u, 0u, 0u, 0u);
+    int put_phys = -1;
+    if (append && pend == uend && __ldg(p.seq_lens + t.b) == L) {
+      put = true;
+      if (lane < 2 * VPR)
+        put_kv = __ldg(static_cast<const uint4*>(lane < VPR ? sp.k_new : sp.v_new) +
+                       (static_cast<size_t>(t.b) * Hkv + t.kvh) * VPR + lane % VPR);
+      put_phys = __ldg(p.block_tables + static_cast<size_t>(t.b) * p.max_blocks + (L - 1) / BS);
+    }
     acc.stage_q(static_cast<const __nv_bfloat16*>(p.q) + head0 * D, G, my_q, lane);
     acc.reset();
     const int jend = t.j + (pend - gpos);
@@ -286,6 +325,8 @@ __global__ void __launch_bounds__(kThreads, PA_STREAM_MIN_CTAS)
       uint8_t* st_ptr = smem + stage * C::STAGE_BYTES;
       const int valid = min(TILE_T, L - j * TILE_T);
       if (valid < TILE_T) zero_tail_rows<C>(st_ptr, valid, lane);
+      if (put && j == t.nt - 1)
+        put_token<C>(st_ptr, valid - 1, put_kv, put_phys, (L - 1) % BS, t.kvh, sp, lane);
       acc.tile(smem_addr(st_ptr), valid, sl2, lane);
       __syncwarp();
       if (i + SPW < cnt) issue(i + SPW);  // refill the stage just consumed

@@ -34,6 +34,11 @@ struct StreamParams {
   int32_t* meta;   // [streams][4]: unit in slot 0, it starts in this stream, unit in slot 1
   float* pml;      // [streams][2][G][2]: (max, sum) of cut-unit pieces, base 2
   float* pacc;     // [streams][2][G][D]: unnormalised outputs of those pieces
+  // Fused cache write (pa_decode_append); all null for a plain decode.
+  const void* k_new;  // [B][Hkv][D] the step's keys: position seq_lens[b]-1 of row b
+  const void* v_new;
+  void* k_pool_w;     // the pools of `d`, written at that position
+  void* v_pool_w;
 };
 
 // One wave of the stream kernel for this shape on the current device (0 if unknown).
@@ -77,6 +82,11 @@ cudaError_t launch_reshape_and_cache(const void* key, const void* value, void* k
                                      void* v_pool, const int64_t* slot_mapping, int T, int Hkv,
                                      int row_bytes, int64_t num_slots, int32_t* err,
                                      cudaStream_t stream);
+// Write k_new/v_new[b] ([B][Hkv][D]) at position seq_lens[b]-1 of row b's block table.
+cudaError_t launch_append_kv(const void* k_new, const void* v_new, void* k_pool, void* v_pool,
+                             const int32_t* block_tables, const int32_t* seq_lens, int B,
+                             int max_blocks, int block_size, int num_blocks, int row_bytes,
+                             int32_t* err, cudaStream_t stream);
 cudaError_t launch_copy_blocks(void* k_pool, void* v_pool, const int32_t* pairs, int n,
                                int64_t block_bytes, int num_blocks, int32_t* err,
                                cudaStream_t stream);

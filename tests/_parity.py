@@ -28,8 +28,12 @@ def to_device(arr, w, device="cuda"):
     return torch.from_numpy(np.ascontiguousarray(arr)).to(device)
 
 
-def gpu_step(w, partition_tokens=0, path=0, device="cuda", keep=False, max_ctas=0):
-    """The product path: allocator, copy_blocks, reshape_and_cache, decode. Returns dict."""
+def gpu_step(w, partition_tokens=0, path=0, device="cuda", keep=False, max_ctas=0, fused=False):
+    """The product path: allocator, copy_blocks, reshape_and_cache, decode. Returns dict.
+
+    With ``fused`` the cache write and the decode are one pa_decode_append call, which
+    derives each row's slot from its table and length (the allocator's slots are only
+    compared, not passed)."""
     import paged_kv_cache_350_b200 as pa
     alloc = pa.Allocator(w.num_blocks, w.block_size, shuffle_seed=w.alloc_seed, pop_order=w.pop_order)
     setup_pairs = workloads.run_setup(w, alloc)
@@ -43,20 +47,25 @@ def gpu_step(w, partition_tokens=0, path=0, device="cuda", keep=False, max_ctas=
     nv = to_device(w.new_v(), w, device)
     err = torch.zeros(1, dtype=torch.int32, device=device)
     pa.pa_copy_blocks(kp, vp, torch.from_numpy(pairs).to(device), err_flag=err)
-    pa.pa_reshape_and_cache(nk, nv, kp, vp, torch.from_numpy(slots).to(device), err_flag=err)
+    if not fused:
+        pa.pa_reshape_and_cache(nk, nv, kp, vp, torch.from_numpy(slots).to(device), err_flag=err)
     out = torch.empty_like(q)
     nws = pa.pa_decode_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.max_blocks * w.block_size,
                                       w.block_size, partition_tokens)
     ws = torch.empty(max(nws, 1), dtype=torch.uint8, device=device)
     t_d = torch.from_numpy(tables).to(device)
     l_d = torch.from_numpy(lens).to(device)
-    pa.pa_decode(out, q, kp, vp, t_d, l_d, w.scale, workspace=ws, err_flag=err,
-                 partition_tokens=partition_tokens, path=path, max_ctas=max_ctas)
+    if fused:
+        pa.pa_decode_append(out, q, nk, nv, kp, vp, t_d, l_d, w.scale, workspace=ws, err_flag=err,
+                            partition_tokens=partition_tokens, path=path, max_ctas=max_ctas)
+    else:
+        pa.pa_decode(out, q, kp, vp, t_d, l_d, w.scale, workspace=ws, err_flag=err,
+                     partition_tokens=partition_tokens, path=path, max_ctas=max_ctas)
     torch.cuda.synchronize()
     res = {"out": out, "slots": slots, "pairs": pairs, "tables": tables, "lens": lens,
            "err": int(err.item()), "alloc": alloc}
     if keep:
-        res.update(k_pool=kp, v_pool=vp, q=q, ws=ws, t_d=t_d, l_d=l_d)
+        res.update(k_pool=kp, v_pool=vp, q=q, ws=ws, t_d=t_d, l_d=l_d, nk=nk, nv=nv)
     return res
 
 
@@ -72,6 +81,18 @@ def oracle_step(w, rows=None):
     out = ref_decode(w.q()[rows], kp, vp, tables[rows], lens[rows], w.scale)
     return {"out": out, "slots": slots, "pairs": pairs, "tables": tables, "lens": lens,
             "k_pool": kp, "v_pool": vp, "alloc": alloc, "rows": rows}
+
+
+def pool_bits(t):
+    """Device pool -> host array of its raw element bits (int16 for bf16, float32 else)."""
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).cpu().numpy()
+    return t.cpu().numpy()
+
+
+def oracle_bits(a, w):
+    """Oracle pool (uint16 bf16 bits or float32) -> the same form as pool_bits."""
+    return np.asarray(a).view(np.int16) if w.dtype == "bf16" else np.asarray(a, dtype=np.float32)
 
 
 def bf16_ulp(x):

@@ -23,12 +23,20 @@ FULL = {
 }
 
 
+@pytest.mark.parametrize("fused", [True, False])
 @pytest.mark.parametrize("name", sorted(FULL))
-def test_full_size_sampled_rows(name):
+def test_full_size_sampled_rows(name, fused):
+    """fused: pa_decode_append, the call bench.py times; else reshape_and_cache + pa_decode."""
     build, rows = FULL[name]
     w = build()
-    g = gpu_step(w)
+    g = gpu_step(w, fused=fused, keep=fused)
     assert g["err"] == 0
+    if fused:
+        # every row's new K/V sits in the slot the allocator reserved for it
+        slots = torch.from_numpy(g["slots"]).cuda()
+        for pool, new in ((g["k_pool"], g["nk"]), (g["v_pool"], g["nv"])):
+            rows_at = pool.view(-1, w.Hkv, w.D)[slots]
+            assert torch.equal(rows_at, new)
     out = g["out"].float()
     assert torch.isfinite(out).all()
     # |o| <= max |v| for a convex combination: a property of every row

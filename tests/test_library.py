@@ -91,6 +91,28 @@ def test_decode_argument_errors_are_reported_before_any_launch():
     assert _call_decode(path=7) == b.PA_ERR_INVALID_ARG
 
 
+def _call_append(**kw):
+    from paged_kv_cache_350_b200 import binding as b
+    a = dict(out=16, q=16, kn=16, vn=16, k=16, v=16, t=16, l=16, B=2, Hq=8, Hkv=2, D=128, bs=16,
+             MB=4, NB=8, scale=0.1, dtype=b.PA_BF16)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    return b.lib.pa_decode_append(vp(a["out"]), vp(a["q"]), vp(a["kn"]), vp(a["vn"]), vp(a["k"]),
+                                  vp(a["v"]), vp(a["t"]), vp(a["l"]), a["B"], a["Hq"], a["Hkv"],
+                                  a["D"], a["bs"], a["MB"], a["NB"], a["scale"], a["dtype"],
+                                  vp(0), 0, vp(0), vp(0), None)
+
+
+def test_decode_append_argument_errors_are_reported_before_any_launch():
+    from paged_kv_cache_350_b200 import binding as b
+    assert _call_append(B=0, kn=0, vn=0) == b.PA_OK           # empty batch: nothing to do
+    assert _call_append(kn=0) == b.PA_ERR_INVALID_ARG         # no new keys
+    assert _call_append(vn=0) == b.PA_ERR_INVALID_ARG
+    assert _call_append(vn=24) == b.PA_ERR_INVALID_ARG        # misaligned new values
+    assert _call_append(D=96) == b.PA_ERR_UNSUPPORTED
+    assert _call_append(Hq=6, Hkv=4) == b.PA_ERR_INVALID_ARG
+
+
 def test_cache_op_argument_errors():
     from paged_kv_cache_350_b200 import binding as b
     vp = ctypes.c_void_p
