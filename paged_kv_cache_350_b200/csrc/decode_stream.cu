@@ -67,7 +67,11 @@ struct StreamCfg : TileCfg<D_, BS_, ROWS16_, PA_STREAM_TILE> {
   static constexpr int NST = kNCW * SPW;
   static constexpr int RING_BYTES = NST * StreamCfg::STAGE_BYTES;
   static constexpr int Q_BYTES = WarpAcc<StreamCfg, true>::Q_BYTES;  // per consumer warp
-  static constexpr int FIXED_BYTES = RING_BYTES + kNCW * Q_BYTES;
+  // Q tiles per warp: with 8 query rows two, so that the next unit's Q is copied in
+  // while the current unit streams (16 rows would cost the third CTA per SM: one tile,
+  // and the next unit's Q is only prefetched into L2).
+  static constexpr int QBUF = StreamCfg::ROWS16 ? 1 : 2;
+  static constexpr int FIXED_BYTES = RING_BYTES + kNCW * QBUF * Q_BYTES;
 };
 
 template <class C>
@@ -171,18 +175,23 @@ __global__ void __launch_bounds__(kThreads, PA_STREAM_MIN_CTAS)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* qtiles = smem + C::RING_BYTES;                  // [kNCW][Q_BYTES]
+  uint8_t* qtiles = smem + C::RING_BYTES;                  // [kNCW][QBUF][Q_BYTES]
   int* P = reinterpret_cast<int*>(smem + C::FIXED_BYTES);  // [B + 1] tiles before sequence b
   __shared__ __align__(8) uint64_t full_bar[NST];
   __shared__ int warp_sum[kThreads / 32];
 
   // ---- prefix sums of per-sequence tile counts (every CTA, identical) --------------
   {
+    // tile counts first, read with independent coalesced loads, then scanned in place
+#pragma unroll 4
+    for (int b = threadIdx.x; b < B; b += kThreads)
+      P[b] = (clamp_len(p, b, blockIdx.x == 0) + TILE_T - 1) / TILE_T;
+    __syncthreads();
     const int chunk = (B + kThreads - 1) / kThreads;
     const int lo = min(B, static_cast<int>(threadIdx.x) * chunk);
     const int hi = min(B, lo + chunk);
     int sum = 0;
-    for (int b = lo; b < hi; ++b) sum += (clamp_len(p, b, blockIdx.x == 0) + TILE_T - 1) / TILE_T;
+    for (int b = lo; b < hi; ++b) sum += P[b];
     int incl = sum;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -195,8 +204,9 @@ __global__ void __launch_bounds__(kThreads, PA_STREAM_MIN_CTAS)
     for (int w = 0; w < warp; ++w) base += warp_sum[w];
     int run = base + incl - sum;
     for (int b = lo; b < hi; ++b) {
+      const int n = P[b];
       P[b] = run;
-      run += (clamp_len(p, b, false) + TILE_T - 1) / TILE_T;
+      run += n;
     }
     if (threadIdx.x == 0) {
       int total = 0;
@@ -290,11 +300,20 @@ __global__ void __launch_bounds__(kThreads, PA_STREAM_MIN_CTAS)
   int i = 0;  // tiles consumed by this stream (ring position)
   bool ok = true;
   WarpAcc<C, true> acc;
-  uint8_t* my_q = qtiles + warp * C::Q_BYTES;
+  uint8_t* my_q = qtiles + warp * C::QBUF * C::Q_BYTES;
+  const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(p.q);
+  auto q_rows = [&](const TilePos& u) {  // the group's query rows of unit u
+    return qg + (static_cast<size_t>(u.b) * p.Hq + static_cast<size_t>(u.kvh) * G) * D;
+  };
 
   int gpos = beg;
+  int qb = 0;  // Q tile of the current unit (QBUF == 2)
+  TilePos t{};
+  if (gpos < end) {
+    t = locate(P, B, Hkv, gpos);
+    if constexpr (C::QBUF == 2) acc.prefetch_q(q_rows(t), G, my_q, lane);
+  }
   while (gpos < end && ok) {
-    const TilePos t = locate(P, B, Hkv, gpos);
     const int L = clamp_len(p, t.b, false);
     const int ubeg = Hkv * P[t.b] + t.kvh * t.nt;
     const int uend = ubeg + t.nt;
@@ -313,7 +332,19 @@ __global__ void __launch_bounds__(kThreads, PA_STREAM_MIN_CTAS)
                        (static_cast<size_t>(t.b) * Hkv + t.kvh) * VPR + lane % VPR);
       put_phys = __ldg(p.block_tables + static_cast<size_t>(t.b) * p.max_blocks + (L - 1) / BS);
     }
-    acc.stage_q(static_cast<const __nv_bfloat16*>(p.q) + head0 * D, G, my_q, lane);
+    // The next unit of this stream (if any) starts at tile pend: its Q rows are copied
+    // while this unit streams.
+    TilePos tn{};
+    if (pend < end) tn = locate(P, B, Hkv, pend);
+    if constexpr (C::QBUF == 2) {
+      acc.use_q(my_q + qb * C::Q_BYTES);
+      if (pend < end) acc.prefetch_q(q_rows(tn), G, my_q + (qb ^ 1) * C::Q_BYTES, lane);
+      qb ^= 1;
+    } else {
+      if (pend < end && lane < G * D * 2 / 128)
+        prefetch_l2(reinterpret_cast<const uint8_t*>(q_rows(tn)) + lane * 128);
+      acc.stage_q(qg + head0 * D, G, my_q, lane);
+    }
     acc.reset();
     const int jend = t.j + (pend - gpos);
     for (int j = t.j; j < jend; ++j, ++i) {
@@ -373,7 +404,9 @@ __global__ void __launch_bounds__(kThreads, PA_STREAM_MIN_CTAS)
       }
     }
     gpos = pend;
+    t = tn;
   }
+  cp_async_wait_all();  // a Q copy still in flight after an early exit
   if (!ok) {
     // A load never arrived: wait (bounded) for this stream's loads still in flight so no
     // TMA write lands after the CTA has left, then report nothing for this stream.

@@ -88,6 +88,30 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ---- per-thread asynchronous copies global -> shared (cp.async) ------------------
+
+// Copy 16 bytes, of which the first `src_bytes` (0 or 16) come from `src` and the rest
+// are zero.  Completion: cp_async_commit() closes a group, cp_async_wait_all() waits
+// for this thread's groups.
+__device__ __forceinline__ void cp_async_16_zfill(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// Bring the 128-byte line holding `p` into L2 (no register, no completion).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // ---- TMA ---------------------------------------------------------------------
 
 // 4-D tiled bulk tensor load global -> shared, completion counted on `bar` in bytes.

@@ -77,6 +77,30 @@ struct WarpAcc {
     __syncwarp();
   }
 
+  // Shared mode, asynchronous: start copying the group's Q rows into the tile at
+  // `tile_ptr` with cp.async (rows >= G zero-filled), so that the load overlaps other
+  // work; use_q() then waits for the copies and makes that tile the A operand.  The
+  // warp must be done reading the tile (it was last used two units ago, and a
+  // __syncwarp has passed since).
+  __device__ __forceinline__ void prefetch_q(const __nv_bfloat16* qrow, int G,
+                                             uint8_t* tile_ptr, int lane) {
+    constexpr int CPR = QROW_BYTES / 16;
+    for (int i = lane; i < C::ROWS * CPR; i += 32) {
+      const int r = i / CPR, c = i - r * CPR;
+      const bool live = r < G;
+      cp_async_16_zfill(smem_addr(tile_ptr + q_off(r, c)),
+                        reinterpret_cast<const uint4*>(qrow + (live ? r : 0) * C::D) + c,
+                        live ? 16 : 0);
+    }
+    cp_async_commit();
+  }
+
+  __device__ __forceinline__ void use_q(uint8_t* tile_ptr) {
+    cp_async_wait_all();
+    __syncwarp();
+    qs = smem_addr(tile_ptr);
+  }
+
   // A fragments of k-step k: registers, or ldmatrix from the shared tile.
   __device__ __forceinline__ void q_frag(int k, int lane, uint32_t& a0, uint32_t& a1,
                                          uint32_t& a2, uint32_t& a3) const {
