@@ -3,7 +3,9 @@
 //
 // S = Q . K^T with m16n8k16 bf16 MMAs (query heads as the 16 rows, padded), an fp32
 // online softmax in base 2, and O += P . V with P fed back from registers as the A
-// operand, split into bf16 hi + lo parts so that P keeps ~16 significant bits.  K and V
+// operand, split into bf16 hi + lo parts so that P keeps ~16 significant bits (with at
+// most 8 query rows, the lo part rides in the otherwise empty rows 8-15 of the same
+// MMA).  K and V
 // come from a shared-memory tile written by TMA with 128-byte swizzle: row r's 16-byte
 // column chunk c sits at r*128 + ((c ^ (r & 7)) << 4) inside each 64-column chunk.
 #pragma once
@@ -227,10 +229,9 @@ struct WarpAcc {
       for (int j = 0; j < C::NT; ++j) {
         o_lo[j][0] *= alpha_lo;
         o_lo[j][1] *= alpha_lo;
-        if constexpr (C::ROWS16) {
-          o_hi[j][0] *= alpha_hi;
-          o_hi[j][1] *= alpha_hi;
-        }
+        // with 8 rows, o_hi holds the lo-part products of the same rows (see below)
+        o_hi[j][0] *= C::ROWS16 ? alpha_hi : alpha_lo;
+        o_hi[j][1] *= C::ROWS16 ? alpha_hi : alpha_lo;
       }
 #pragma unroll
       for (int jp = 0; jp < C::NT / 2; ++jp) {
@@ -239,32 +240,44 @@ struct WarpAcc {
         uint32_t w0, w1, w2, w3;
         ldmatrix_x4_trans(vbase + (d >> 6) * C::CHUNK_BYTES + sw128(row, (d & 63) >> 3), w0, w1,
                           w2, w3);
+        if constexpr (C::ROWS16) {
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const uint32_t a0 = half ? pr0 : pa0, a1 = half ? pr1 : pa1;
-          const uint32_t a2 = half ? pr2 : pa2, a3 = half ? pr3 : pa3;
-          if constexpr (C::ROWS16) {
+          for (int half = 0; half < 2; ++half) {
+            const uint32_t a0 = half ? pr0 : pa0, a1 = half ? pr1 : pa1;
+            const uint32_t a2 = half ? pr2 : pa2, a3 = half ? pr3 : pa3;
             mma_bf16_16816(o_lo[2 * jp][0], o_lo[2 * jp][1], o_hi[2 * jp][0], o_hi[2 * jp][1], a0,
                            a1, a2, a3, w0, w1, o_lo[2 * jp][0], o_lo[2 * jp][1], o_hi[2 * jp][0],
                            o_hi[2 * jp][1]);
             mma_bf16_16816(o_lo[2 * jp + 1][0], o_lo[2 * jp + 1][1], o_hi[2 * jp + 1][0],
                            o_hi[2 * jp + 1][1], a0, a1, a2, a3, w2, w3, o_lo[2 * jp + 1][0],
                            o_lo[2 * jp + 1][1], o_hi[2 * jp + 1][0], o_hi[2 * jp + 1][1]);
-          } else {
-            float dead0, dead1;
-            mma_bf16_16816(o_lo[2 * jp][0], o_lo[2 * jp][1], dead0, dead1, a0, 0u, a2, 0u, w0, w1,
-                           o_lo[2 * jp][0], o_lo[2 * jp][1], 0.f, 0.f);
-            mma_bf16_16816(o_lo[2 * jp + 1][0], o_lo[2 * jp + 1][1], dead0, dead1, a0, 0u, a2, 0u,
-                           w2, w3, o_lo[2 * jp + 1][0], o_lo[2 * jp + 1][1], 0.f, 0.f);
           }
+        } else {
+          // 8 query rows: A rows 0-7 carry P's hi part and rows 8-15 (otherwise unused)
+          // its lo part, so one MMA accumulates hi.V into o_lo and lo.V into o_hi;
+          // reduce_l() adds the two.
+          mma_bf16_16816(o_lo[2 * jp][0], o_lo[2 * jp][1], o_hi[2 * jp][0], o_hi[2 * jp][1], pa0,
+                         pr0, pa2, pr2, w0, w1, o_lo[2 * jp][0], o_lo[2 * jp][1], o_hi[2 * jp][0],
+                         o_hi[2 * jp][1]);
+          mma_bf16_16816(o_lo[2 * jp + 1][0], o_lo[2 * jp + 1][1], o_hi[2 * jp + 1][0],
+                         o_hi[2 * jp + 1][1], pa0, pr0, pa2, pr2, w2, w3, o_lo[2 * jp + 1][0],
+                         o_lo[2 * jp + 1][1], o_hi[2 * jp + 1][0], o_hi[2 * jp + 1][1]);
         }
       }
     }
   }
 
-  // Sum the per-lane partial row sums over the 4 lanes of each row.
+  // Sum the per-lane partial row sums over the 4 lanes of each row; with 8 rows, also
+  // add the lo-part products (o_hi) into o_lo.  Call once, before reading the outputs.
   __device__ __forceinline__ void reduce_l() {
     constexpr unsigned kFull = 0xffffffffu;
+    if constexpr (!C::ROWS16) {
+#pragma unroll
+      for (int j = 0; j < C::NT; ++j) {
+        o_lo[j][0] += o_hi[j][0];
+        o_lo[j][1] += o_hi[j][1];
+      }
+    }
     l_lo += __shfl_xor_sync(kFull, l_lo, 1);
     l_lo += __shfl_xor_sync(kFull, l_lo, 2);
     if constexpr (C::ROWS16) {
