@@ -55,6 +55,9 @@ struct WarpAcc {
   float o_lo[C::NT][2];
   float o_hi[C::NT][2];
   float m_lo, m_hi, l_lo, l_hi;
+  // 8-row mode (tile_t): running max and this lane's partial sum of heads 2tig, 2tig+1;
+  // reduce_l() turns them into m_lo / l_lo of row g.
+  float mh[2], lh[2];
   uint32_t qa[QSMEM ? 1 : C::KSTEPS][2];  // Q rows g as A fragments (register mode)
   uint32_t qh[QSMEM ? 1 : C::KSTEPS][2];  // Q rows g+8
   uint32_t qs = 0;                         // shared address of the Q tile (shared mode)
@@ -132,6 +135,8 @@ struct WarpAcc {
       o_hi[j][0] = o_hi[j][1] = 0.f;
     }
     m_lo = m_hi = -INFINITY;
+    mh[0] = mh[1] = -INFINITY;
+    lh[0] = lh[1] = 0.f;
     l_lo = l_hi = 0.f;
   }
 
@@ -185,6 +190,11 @@ struct WarpAcc {
   template <bool ROWMASK = false>
   __device__ __forceinline__ void tile(uint32_t kbase, int valid, float sl2, int lane,
                                        int row_lo = 0, int row_hi = 16) {
+    static_assert(!ROWMASK || C::ROWS16, "row masks are kept for 16-row tiles only");
+    if constexpr (!C::ROWS16) {
+      tile_t(kbase, valid, sl2, lane);
+      return;
+    }
     const uint32_t vbase = kbase + C::TILE_BYTES;
     const int tig = lane & 3;
     const int mi = lane >> 3, mr = lane & 7;
@@ -267,8 +277,93 @@ struct WarpAcc {
     }
   }
 
-  // Sum the per-lane partial row sums over the 4 lanes of each row; with 8 rows, also
-  // add the lo-part products (o_hi) into o_lo.  Call once, before reading the outputs.
+  // 8 query rows: S is computed transposed, S^T = K.Q^T, with the sub-tile's 16 tokens as
+  // the MMA rows and the (up to 8) heads as its 8 columns: one MMA per k-step instead of
+  // two whose rows 8-15 would be empty.  Lane (g, tig) then holds tokens g and g+8 of
+  // heads 2tig and 2tig+1, so the softmax state is kept per head (mh, lh: max over the
+  // 8 lanes of a column by shuffles, sums per lane until reduce_l), and movmatrix
+  // transposes P back into A-operand layout (heads as rows) for O += P.V.  P.V then runs
+  // as in tile(), with the lo part of P in the A rows 8-15 and its products in o_hi.
+  __device__ __forceinline__ void tile_t(uint32_t kbase, int valid, float sl2, int lane) {
+    constexpr unsigned kFull = 0xffffffffu;
+    const uint32_t vbase = kbase + C::TILE_BYTES;
+    const int g = lane >> 2;
+    const int mi = lane >> 3, mr = lane & 7;
+#pragma unroll
+    for (int st = 0; st < C::SUBT; ++st) {
+      const int r0 = st * 16;
+      if (r0 >= valid) break;
+      float c0 = 0.f, c1 = 0.f, c2 = 0.f, c3 = 0.f;
+#pragma unroll
+      for (int k = 0; k < C::KSTEPS; ++k) {
+        // A = K rows r0..r0+15 x columns 16k..16k+15; matrices (rows 0-7, 8-15) x
+        // (columns 0-7, 8-15) in A-fragment order
+        const int row = r0 + (mi & 1) * 8 + mr;
+        const int d = 16 * k + (mi >> 1) * 8;
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4(kbase + (d >> 6) * C::CHUNK_BYTES + sw128(row, (d & 63) >> 3), a0, a1, a2,
+                    a3);
+        // B = Q^T: Q[g][16k+2tig..] and Q[g][16k+8+2tig..] are its two fragments
+        uint32_t q0, q1, q2, q3;
+        q_frag(k, lane, q0, q1, q2, q3);
+        mma_bf16_16816(c0, c1, c2, c3, a0, a1, a2, a3, q0, q2, c0, c1, c2, c3);
+      }
+      const bool va = r0 + g < valid, vb = r0 + g + 8 < valid;
+      const float x0 = va ? c0 * sl2 : -INFINITY;  // token g,   head 2tig
+      const float x1 = va ? c1 * sl2 : -INFINITY;  // token g,   head 2tig+1
+      const float x2 = vb ? c2 * sl2 : -INFINITY;  // token g+8, head 2tig
+      const float x3 = vb ? c3 * sl2 : -INFINITY;  // token g+8, head 2tig+1
+      float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, off));
+      }
+      const float mn0 = fmaxf(mh[0], mx0), mn1 = fmaxf(mh[1], mx1);  // token r0 is valid
+      const float al0 = exp2f(mh[0] - mn0), al1 = exp2f(mh[1] - mn1);
+      mh[0] = mn0;
+      mh[1] = mn1;
+      const float e0 = exp2f(x0 - mn0), e1 = exp2f(x1 - mn1);
+      const float e2 = exp2f(x2 - mn0), e3 = exp2f(x3 - mn1);
+      lh[0] = lh[0] * al0 + (e0 + e2);
+      lh[1] = lh[1] * al1 + (e1 + e3);
+      uint32_t h01, l01, h23, l23;
+      split_bf16x2(e0, e1, h01, l01);  // P^T row g (token), columns 2tig, 2tig+1 (heads)
+      split_bf16x2(e2, e3, h23, l23);  // P^T row g+8
+      // P row g (head): tokens 2tig, 2tig+1 and 8+2tig, 9+2tig, hi and lo parts
+      const uint32_t pa0 = movmatrix_trans(h01), pa2 = movmatrix_trans(h23);
+      const uint32_t pr0 = movmatrix_trans(l01), pr2 = movmatrix_trans(l23);
+      // rescale of output row g (head g): its factor sits in the lanes with tig = g/2
+      const float s0 = __shfl_sync(kFull, al0, g >> 1), s1 = __shfl_sync(kFull, al1, g >> 1);
+      const float alpha = (g & 1) ? s1 : s0;
+#pragma unroll
+      for (int j = 0; j < C::NT; ++j) {
+        o_lo[j][0] *= alpha;
+        o_lo[j][1] *= alpha;
+        o_hi[j][0] *= alpha;
+        o_hi[j][1] *= alpha;
+      }
+#pragma unroll
+      for (int jp = 0; jp < C::NT / 2; ++jp) {
+        const int row = r0 + (mi & 1) * 8 + mr;
+        const int d = 16 * jp + (mi >> 1) * 8;
+        uint32_t w0, w1, w2, w3;
+        ldmatrix_x4_trans(vbase + (d >> 6) * C::CHUNK_BYTES + sw128(row, (d & 63) >> 3), w0, w1,
+                          w2, w3);
+        mma_bf16_16816(o_lo[2 * jp][0], o_lo[2 * jp][1], o_hi[2 * jp][0], o_hi[2 * jp][1], pa0,
+                       pr0, pa2, pr2, w0, w1, o_lo[2 * jp][0], o_lo[2 * jp][1], o_hi[2 * jp][0],
+                       o_hi[2 * jp][1]);
+        mma_bf16_16816(o_lo[2 * jp + 1][0], o_lo[2 * jp + 1][1], o_hi[2 * jp + 1][0],
+                       o_hi[2 * jp + 1][1], pa0, pr0, pa2, pr2, w2, w3, o_lo[2 * jp + 1][0],
+                       o_lo[2 * jp + 1][1], o_hi[2 * jp + 1][0], o_hi[2 * jp + 1][1]);
+      }
+    }
+  }
+
+  // Finish the unit's sums: the per-lane partial row sums over the 4 lanes of each row;
+  // with 8 rows (tile_t), the per-head state over the 8 lanes of each column, moved to
+  // row g's m_lo / l_lo, and the lo-part products (o_hi) added into o_lo.  Call once,
+  // before reading the outputs.
   __device__ __forceinline__ void reduce_l() {
     constexpr unsigned kFull = 0xffffffffu;
     if constexpr (!C::ROWS16) {
@@ -277,6 +372,17 @@ struct WarpAcc {
         o_lo[j][0] += o_hi[j][0];
         o_lo[j][1] += o_hi[j][1];
       }
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        lh[0] += __shfl_xor_sync(kFull, lh[0], off);
+        lh[1] += __shfl_xor_sync(kFull, lh[1], off);
+      }
+      const int g = (threadIdx.x & 31) >> 2;
+      const float m0 = __shfl_sync(kFull, mh[0], g >> 1), m1 = __shfl_sync(kFull, mh[1], g >> 1);
+      const float s0 = __shfl_sync(kFull, lh[0], g >> 1), s1 = __shfl_sync(kFull, lh[1], g >> 1);
+      m_lo = (g & 1) ? m1 : m0;
+      l_lo = (g & 1) ? s1 : s0;
+      return;
     }
     l_lo += __shfl_xor_sync(kFull, l_lo, 1);
     l_lo += __shfl_xor_sync(kFull, l_lo, 2);
