@@ -90,7 +90,7 @@ size_t pa_decode_workspace_size(int B, int Hq, int Hkv, int D, int max_seq_len,
       pa::tc_eligible(G, D, block_size, PA_BF16)) {
     int grid = pa::stream_grid(D, block_size, G, B);
     if (grid <= 0) grid = kStreamGridBound;  // no device to ask: an upper bound
-    const size_t s = pa::stream_workspace_bytes(grid * pa::stream_warps_per_cta(), G, D);
+    const size_t s = pa::stream_workspace_bytes(grid * pa::stream_warps_per_cta(block_size), G, D);
     if (s > need) need = s;
   }
   return need;
@@ -134,7 +134,7 @@ static pa_status plan_decode(int B, int Hq, int Hkv, int D, int block_size, int 
   if (tc_ok && partition == 0 && B <= kStreamMaxB && tile_bound < (int64_t(1) << 31)) {
     int grid = pa::stream_grid(D, block_size, G, B);
     if (max_ctas > 0 && grid > max_ctas) grid = max_ctas;
-    if (grid > 0 && have_ws && workspace_bytes >= pa::stream_workspace_bytes(grid * pa::stream_warps_per_cta(), G, D)) {
+    if (grid > 0 && have_ws && workspace_bytes >= pa::stream_workspace_bytes(grid * pa::stream_warps_per_cta(block_size), G, D)) {
       info->kernel = PA_KERNEL_TC_STREAM;
       info->grid = grid;
       info->max_parts = 1;
@@ -218,7 +218,7 @@ static pa_status decode_call(void* out, const void* q, const void* k_new, const 
   if (plan.kernel == PA_KERNEL_TC_STREAM) {
     pa::StreamParams sp{};
     sp.d = p;
-    sp.streams = plan.grid * pa::stream_warps_per_cta();
+    sp.streams = plan.grid * pa::stream_warps_per_cta(block_size);
     pa::stream_carve(&sp, workspace);
     if (append) {  // the decode kernel writes the step's token itself
       sp.k_new = k_new;

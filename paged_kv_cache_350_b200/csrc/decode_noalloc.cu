@@ -89,7 +89,7 @@ extern "C" pa_status pa_decode_no_alloc(void* out, const void* q, const void* k_
 
   const int grid = pa::stream_grid(D, block_size, G, B);
   if (grid <= 0) return PA_ERR_CUDA;
-  if (pa::stream_workspace_bytes(grid * pa::stream_warps_per_cta(), G, D) > kScratchBytes) return PA_ERR_SCRATCH_LIMIT;
+  if (pa::stream_workspace_bytes(grid * pa::stream_warps_per_cta(block_size), G, D) > kScratchBytes) return PA_ERR_SCRATCH_LIMIT;
   void* scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) return PA_ERR_CUDA;
 
@@ -112,7 +112,7 @@ extern "C" pa_status pa_decode_no_alloc(void* out, const void* q, const void* k_
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.max_parts = 1;
   p.err = dev_err_flag;
-  sp.streams = grid * pa::stream_warps_per_cta();
+  sp.streams = grid * pa::stream_warps_per_cta(block_size);
   pa::stream_carve(&sp, scratch);
   const cudaError_t e =
       pa::launch_decode_stream(sp, grid, reinterpret_cast<cudaStream_t>(stream));

@@ -35,13 +35,9 @@ namespace pa {
 
 namespace {
 
-// Build-time tunables: ring stages per stream, and the CTAs per SM the register
-// allocation is bounded for (0 = let the compiler choose).
+// Build-time tunable: ring stages per stream.
 #ifndef PA_STREAM_SPW
 #define PA_STREAM_SPW 2
-#endif
-#ifndef PA_STREAM_MIN_CTAS
-#define PA_STREAM_MIN_CTAS 3
 #endif
 // Launch the reduce as a programmatic dependent of the main kernel (its launch overlaps
 // the main kernel's tail; it waits for the main grid's completion before reading).
@@ -49,29 +45,47 @@ namespace {
 #define PA_STREAM_PDL 1
 #endif
 
-// Warps (= streams) per CTA and tokens per pipeline stage.
-#ifndef PA_STREAM_NCW
-#define PA_STREAM_NCW 2
-#endif
-#ifndef PA_STREAM_TILE
-#define PA_STREAM_TILE 32
-#endif
-
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kNCW = PA_STREAM_NCW;          // warps (= streams) per CTA
-constexpr int kThreads = kNCW * 32;
+
+// Stage and CTA shape by block size.  Blocks of <= 16 tokens: 16-token stages (8 KB with
+// D = 128), 4 warps per CTA and 2 CTAs per SM, so every SM runs 8 streams, two on each of
+// its four sub-partitions (the tile math's issue and tensor rate per sub-partition is
+// part of the pace: 6 streams per SM left two sub-partitions with double load).  A
+// 32-token block needs a 32-token stage (16 KB): 2 warps per CTA, 3 CTAs per SM.
+// PA_STREAM_TILE / PA_STREAM_NCW / PA_STREAM_MIN_CTAS override all block sizes (sweeps).
+template <int BS>
+struct StreamShape {
+#ifdef PA_STREAM_TILE
+  static constexpr int TILE = PA_STREAM_TILE;
+#else
+  static constexpr int TILE = BS <= 16 ? 16 : 32;
+#endif
+#ifdef PA_STREAM_NCW
+  static constexpr int NCW = PA_STREAM_NCW;
+#else
+  static constexpr int NCW = BS <= 16 ? 4 : 2;
+#endif
+#ifdef PA_STREAM_MIN_CTAS
+  static constexpr int MIN_CTAS = PA_STREAM_MIN_CTAS;
+#else
+  static constexpr int MIN_CTAS = BS <= 16 ? 2 : 3;
+#endif
+};
 
 template <int D_, int BS_, bool ROWS16_, int SPW_>
-struct StreamCfg : TileCfg<D_, BS_, ROWS16_, PA_STREAM_TILE> {
+struct StreamCfg : TileCfg<D_, BS_, ROWS16_, StreamShape<BS_>::TILE> {
+  static constexpr int NCW = StreamShape<BS_>::NCW;  // warps (= streams) per CTA
+  static constexpr int THREADS = NCW * 32;
+  static constexpr int MIN_CTAS = StreamShape<BS_>::MIN_CTAS;  // register bound
   static constexpr int SPW = SPW_;                 // ring stages per stream
-  static constexpr int NST = kNCW * SPW;
+  static constexpr int NST = NCW * SPW;
   static constexpr int RING_BYTES = NST * StreamCfg::STAGE_BYTES;
   static constexpr int Q_BYTES = WarpAcc<StreamCfg, true>::Q_BYTES;  // per consumer warp
-  // Q tiles per warp: with 8 query rows two, so that the next unit's Q is copied in
-  // while the current unit streams (16 rows would cost the third CTA per SM: one tile,
-  // and the next unit's Q is only prefetched into L2).
-  static constexpr int QBUF = StreamCfg::ROWS16 ? 1 : 2;
-  static constexpr int FIXED_BYTES = RING_BYTES + kNCW * QBUF * Q_BYTES;
+  // Q tiles per warp: two, so that the next unit's Q is copied in while the current unit
+  // streams; one for 16 query rows with 32-token stages, where a second would cost the
+  // third CTA per SM (the next unit's Q is then only prefetched into L2).
+  static constexpr int QBUF = (StreamCfg::ROWS16 && StreamCfg::TILE_T == 32) ? 1 : 2;
+  static constexpr int FIXED_BYTES = RING_BYTES + NCW * QBUF * Q_BYTES;
 };
 
 template <class C>
@@ -163,10 +177,11 @@ __device__ __forceinline__ void put_token(uint8_t* stage_ptr, int r, const uint4
 }
 
 template <class C>
-__global__ void __launch_bounds__(kThreads, PA_STREAM_MIN_CTAS)
+__global__ void __launch_bounds__(C::THREADS, C::MIN_CTAS)
     decode_stream_kernel(const __grid_constant__ CUtensorMap tmk,
                          const __grid_constant__ CUtensorMap tmv, const StreamParams sp) {
   constexpr int D = C::D, BS = C::BS, TILE_T = C::TILE_T, SPW = C::SPW, NST = C::NST;
+  constexpr int kNCW = C::NCW, kThreads = C::THREADS;
   const DecodeParams& p = sp.d;
   const int B = p.B, Hkv = p.Hkv, G = p.G;
   const int warp = threadIdx.x >> 5;
@@ -503,7 +518,7 @@ int stream_grid_for(int B, int device_sms) {
   if (cudaFuncSetAttribute(decode_stream_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_stream_kernel<C>, kThreads,
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_stream_kernel<C>, C::THREADS,
                                                     smem) != cudaSuccess)
     return 0;
   return occ * device_sms;
@@ -521,7 +536,7 @@ cudaError_t launch_stream_cfg(const StreamParams& sp, int grid, cudaStream_t str
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  decode_stream_kernel<C><<<grid, kThreads, smem, stream>>>(tmk, tmv, sp);
+  decode_stream_kernel<C><<<grid, C::THREADS, smem, stream>>>(tmk, tmv, sp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 #if PA_STREAM_PDL
@@ -558,7 +573,14 @@ cudaError_t launch_d_bs(const StreamParams& sp, int grid, cudaStream_t stream) {
 
 }  // namespace
 
-int stream_warps_per_cta() { return kNCW; }
+int stream_warps_per_cta(int block_size) {
+  switch (block_size) {
+    case 8: return StreamShape<8>::NCW;
+    case 16: return StreamShape<16>::NCW;
+    case 32: return StreamShape<32>::NCW;
+    default: return 0;
+  }
+}
 
 int stream_grid(int D, int block_size, int G, int B) {
   int dev = 0, sms = 0;

@@ -43,8 +43,9 @@ struct StreamParams {
 
 // One wave of the stream kernel for this shape on the current device (0 if unknown).
 int stream_grid(int D, int block_size, int G, int B);
-// Streams (warps) per CTA of the stream kernel: streams = grid * stream_warps_per_cta().
-int stream_warps_per_cta();
+// Streams (warps) per CTA of the stream kernel for this block size:
+// streams = grid * stream_warps_per_cta(block_size).
+int stream_warps_per_cta(int block_size);
 size_t stream_workspace_bytes(int streams, int G, int D);
 void stream_carve(StreamParams* sp, void* workspace);
 cudaError_t launch_decode_stream(const StreamParams& sp, int grid, cudaStream_t stream);
