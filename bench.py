@@ -15,8 +15,8 @@ step (the cache writes are idempotent), over pools larger than the 126 MB L2.
 Prints ONE JSON line (rank 0).  ``value`` = algorithmic KV bytes of pa_decode
 per step x steps x ranks / max-over-ranks device time, in GB/s (the whole step
 is in the denominator).  ``e2e`` = the same metric through
-``PagedKVCache.step_staged`` with host buffers: allocator, host->device copy,
-kernels, device->host copy of the output, per step.  ``roofline`` is the decode
+``PagedKVCache.pipeline`` with host buffers: per step the allocator, a host->device
+copy, the kernels and a device->host copy of the output, steps queued back to back.  ``roofline`` is the decode
 call alone (pa_decode_append, or pa_decode with ``--unfused``) against the
 measured HBM copy bandwidth.
 
@@ -70,7 +70,7 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--config", default="gqa", choices=sorted(CONFIG_TEXT))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--e2e-steps", type=int, default=60)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -437,37 +437,54 @@ def run_ours(args):
     roof_bytes += append_bytes
     achieved = roof_bytes / (dec_avg_ms / 1e3) / 1e9
 
-    # ---- end to end through PagedKVCache.step with host buffers -------------------
+    # ---- end to end through the public API with host buffers -------------------------
+    # PagedKVCache.pipeline: every step runs the C allocator, one host->device copy of the
+    # step input (q, new K/V, tables, lengths, copy pairs), pa_copy_blocks +
+    # pa_decode_append and a device->host copy of the output; steps are queued back to
+    # back with double-buffered staging, and each step's output is read one step later.
     e2e = None
     if not args.no_e2e and args.e2e_steps > 0 and not args.shared_prefix:
         cache = pa.PagedKVCache(w.num_blocks, w.block_size, w.Hkv, w.D, dtype=kp.dtype, device=device,
                                 shuffle_seed=w.alloc_seed, pop_order=w.pop_order, k_pool=kp, v_pool=vp)
         workloads.run_setup(w, cache.alloc)
-        q_h, k_h, v_h = cache.host_inputs(w.B, w.Hq, MB)
-        q_h.copy_(q.cpu())
-        k_h.copy_(nk.cpu())
-        v_h.copy_(nv.cpu())
+        pipe = cache.pipeline(w.B, w.Hq, MB, stream=stream)
+        q_c, nk_c, nv_c = q.cpu(), nk.cpu(), nv.cpu()
         ids = np.asarray(w.step_seqs, dtype=np.int64)
-        times, nbytes = [], []
-        h2d = d2h = 0
+        warm = max(2, pipe.depth)
+        nbytes = []
         cur = lens.astype(np.int64).copy()
-        for i in range(args.e2e_steps + 2):
-            barrier(dist, device)
-            t0 = time.perf_counter()
-            _, (h2d, d2h) = cache.step_staged(ids, w.scale, MB, stream=stream)
-            dt = time.perf_counter() - t0
-            if i >= 2:  # the first two steps warm the staging buffers
-                times.append(dt)
+        t0 = None
+        done = 0
+        for i in range(warm + args.e2e_steps):
+            if i < pipe.depth:  # the same inputs every step: each staging slot written once
+                for dst, src in zip(pipe.inputs(), (q_c, nk_c, nv_c)):
+                    dst.copy_(src)
+            if i == warm:
+                pipe.sync()
+                barrier(dist, device)
+                t0 = time.perf_counter()
+            try:
+                pipe.submit(ids, w.scale)
+            except pa.PAError:  # the pool ran out of blocks for more appends
+                break
+            if i >= 1:
+                pipe.result(i - 1)
+            if i >= warm:
                 nbytes.append(decode_bytes(cur, w.B, w.Hq, w.Hkv, w.D, w.block_size, esize)[0])
+                done += 1
             cur += 1
+        pipe.result(pipe.next - 1)
+        dt = time.perf_counter() - t0 if t0 is not None else 0.0
         cache.check_device_errors()
-        mean_dt = max_over_ranks(statistics.fmean(times), dist, device)
-        e2e = {"value": statistics.fmean(nbytes) * world / mean_dt / 1e9, "unit": UNIT,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": 1e3 * mean_dt, "steps": len(times),
-               "timing": "host perf_counter per step of PagedKVCache.step_staged: C allocator, "
-                         "one host->device copy of the step input, kernels, device->host "
-                         "copy of the output, stream sync"}
+        if done:
+            dt = max_over_ranks(dt, dist, device)
+            e2e = {"value": sum(nbytes) * world / dt / 1e9, "unit": UNIT,
+                   "h2d_bytes_per_step": int(pipe.bytes_in), "d2h_bytes_per_step": int(pipe.bytes_out),
+                   "ms_per_step": 1e3 * dt / done, "steps": done,
+                   "timing": "host perf_counter over the steps of PagedKVCache.pipeline: per step the C "
+                             "allocator, one host->device copy of the step input, kernels, a "
+                             "device->host copy of the output (read one step later); steps queued "
+                             "back to back, double-buffered staging"}
 
     # ---- CPU oracle baseline (rank 0, one GPU only) --------------------------------
     cpu = None

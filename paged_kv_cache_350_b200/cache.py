@@ -20,6 +20,10 @@ Everything between the copies runs in the library's kernels.
 caller writes the step's q / new K / new V straight into the cache's pinned
 input buffer, the allocator writes slots, tables and lengths behind them, and a
 single copy moves the whole step input.
+
+``pipeline`` (``StepPipeline``) queues such steps back to back: double-buffered
+staging, the copies on their own streams, so the host and the copy engines work on
+neighbouring steps while the GPU decodes the current one.
 """
 
 from __future__ import annotations
@@ -188,6 +192,10 @@ class PagedKVCache:
         stream.synchronize()
         return self._out_h, (used, self._out_h.numel() * self._out_h.element_size())
 
+    def pipeline(self, B, Hq, max_blocks, depth=2, stream=None):
+        """A StepPipeline over this cache: decode steps queued back to back."""
+        return StepPipeline(self, B, Hq, max_blocks, depth=depth, stream=stream)
+
     # -- sequence management ------------------------------------------------------------
     def admit(self, seq_id, k_host, v_host, stream=None):
         """Register a sequence and write its prompt's K/V ([n, Hkv, D] host) into its blocks."""
@@ -225,3 +233,122 @@ class PagedKVCache:
         flag = int(self.err.item())
         if flag:
             raise _b.PAError(_b.pa_status_from_device_flag(flag), "device")
+
+
+class StepPipeline:
+    """Decode steps of a fixed batch shape queued back to back, host and device overlapped.
+
+    Each step is the same work as ``PagedKVCache.step_staged``: the allocator reserves a
+    slot per sequence, one host->device copy moves the step's q / new K / new V, tables,
+    lengths and copy pairs, ``pa_copy_blocks`` + ``pa_decode_append`` run, and the output
+    is copied back to pinned host memory.  Here the step input and output buffers come in
+    ``depth`` slots, the copies run on their own streams, and ``submit`` returns once the
+    step is queued.  So the host prepares step t+1 and the copy engines move its input
+    and step t-1's output while the GPU decodes step t.  Events order every reuse of a
+    slot: a host input buffer is rewritten only after its copy has finished, a device
+    input buffer only after the kernels that read it, a device output buffer only after
+    its copy to the host.
+
+        pipe = cache.pipeline(B, Hq, max_blocks)
+        q, k, v = pipe.inputs()        # pinned views of the next step's input slot
+        ...                            # write the step's q [B,Hq,D], k/v [B,Hkv,D]
+        t = pipe.submit(seq_ids, scale)
+        out = pipe.result(t)           # waits for step t's output copy (pinned [B,Hq,D])
+
+    ``result(t)`` stays valid until step t + depth is submitted.
+    """
+
+    def __init__(self, cache, B, Hq, max_blocks, depth=2, stream=None):
+        assert depth >= 1
+        self.cache, self.B, self.Hq, self.max_blocks, self.depth = cache, B, Hq, max_blocks, depth
+        self.dev = cache.device
+        self.stream = stream or torch.cuda.current_stream(self.dev)
+        self.copy_in = torch.cuda.Stream(self.dev)
+        self.copy_out = torch.cuda.Stream(self.dev)
+        self.lay, total = cache._layout(B, Hq, max_blocks)
+        n_out = B * Hq * cache.D
+        self.h_in = [torch.empty(total, dtype=torch.uint8, pin_memory=True) for _ in range(depth)]
+        self.d_in = [torch.empty(total, dtype=torch.uint8, device=self.dev) for _ in range(depth)]
+        self.h_out = [torch.empty(n_out, dtype=cache.dtype, pin_memory=True).view(B, Hq, cache.D)
+                      for _ in range(depth)]
+        self.d_out = [torch.empty(n_out, dtype=cache.dtype, device=self.dev).view(B, Hq, cache.D)
+                      for _ in range(depth)]
+        ev = lambda: [torch.cuda.Event() for _ in range(depth)]  # noqa: E731
+        self.h2d_done, self.kern_done, self.d2h_done = ev(), ev(), ev()
+        self.used = [False] * depth   # slot has a step in flight (its events are recorded)
+        self.next = 0                 # index of the next step to submit
+        self.bytes_in = self.bytes_out = 0
+        cache.workspace(B, Hq, max_blocks)
+
+    def _view(self, buf, name, shape, dtype):
+        off, n = self.lay[name]
+        return buf[off:off + n].view(dtype).view(shape)
+
+    def inputs(self):
+        """Pinned host (q, k, v) of the next step's slot, once its previous copy is done."""
+        k = self.next % self.depth
+        if self.used[k]:
+            self.h2d_done[k].synchronize()
+        c, h = self.cache, self.h_in[k]
+        return (self._view(h, "q", (self.B, self.Hq, c.D), c.dtype),
+                self._view(h, "k", (self.B, c.Hkv, c.D), c.dtype),
+                self._view(h, "v", (self.B, c.Hkv, c.D), c.dtype))
+
+    def submit(self, seq_ids, scale):
+        """Queue one decode step for seq_ids (the inputs() of this step must be written)."""
+        c, B, MB = self.cache, self.B, self.max_blocks
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        assert ids.size == B, "the batch shape is fixed per pipeline"
+        t, k = self.next, self.next % self.depth
+        h, d = self.h_in[k], self.d_in[k]
+        if self.used[k]:
+            self.h2d_done[k].synchronize()   # normally long done: the copy of step t - depth
+        _, pairs = c.alloc.append_slots(ids, slot_out=self._view(h, "slots", (B,), torch.int64).numpy(),
+                                        pairs_out=self._view(h, "pairs", (B, 2), torch.int32).numpy())
+        c.alloc.block_tables(ids, MB, tables_out=self._view(h, "tables", (B, MB), torch.int32).numpy(),
+                             lens_out=self._view(h, "lens", (B,), torch.int32).numpy())
+        npairs = pairs.shape[0]
+        used = self.lay["pairs"][0] + npairs * 8 if npairs else self.lay["lens"][0] + B * 4
+        if self.used[k]:
+            self.copy_in.wait_event(self.kern_done[k])     # step t - depth has read d_in[k]
+        with torch.cuda.stream(self.copy_in):
+            d[:used].copy_(h[:used], non_blocking=True)
+        self.h2d_done[k].record(self.copy_in)
+        s = self.stream
+        s.wait_event(self.h2d_done[k])
+        if self.used[k]:
+            s.wait_event(self.d2h_done[k])                 # d_out[k] was copied out
+        with torch.cuda.stream(s):
+            if npairs:
+                _b.pa_copy_blocks(c.k_pool, c.v_pool,
+                                  self._view(d, "pairs", (B, 2), torch.int32)[:npairs],
+                                  err_flag=c.err, stream=s)
+            _b.pa_decode_append(self.d_out[k], self._view(d, "q", (B, self.Hq, c.D), c.dtype),
+                                self._view(d, "k", (B, c.Hkv, c.D), c.dtype),
+                                self._view(d, "v", (B, c.Hkv, c.D), c.dtype), c.k_pool, c.v_pool,
+                                self._view(d, "tables", (B, MB), torch.int32),
+                                self._view(d, "lens", (B,), torch.int32), scale,
+                                workspace=c.workspace(B, self.Hq, MB), err_flag=c.err, stream=s)
+        self.kern_done[k].record(s)
+        self.copy_out.wait_event(self.kern_done[k])
+        with torch.cuda.stream(self.copy_out):
+            self.h_out[k].copy_(self.d_out[k], non_blocking=True)
+        self.d2h_done[k].record(self.copy_out)
+        self.used[k] = True
+        self.bytes_in = used
+        self.bytes_out = self.h_out[k].numel() * self.h_out[k].element_size()
+        self.next = t + 1
+        return t
+
+    def result(self, t):
+        """Pinned host output [B, Hq, D] of step t (waits for its copy)."""
+        assert self.next - self.depth <= t < self.next, "step no longer (or not yet) held"
+        k = t % self.depth
+        self.d2h_done[k].synchronize()
+        return self.h_out[k]
+
+    def sync(self):
+        """Wait for every queued step."""
+        for k in range(self.depth):
+            if self.used[k]:
+                self.d2h_done[k].synchronize()

@@ -147,3 +147,72 @@ def test_serving_trace_matches_oracle_replay(name):
     vd = cache.v_pool.view(torch.int16).cpu().numpy().view(np.uint16)
     assert np.array_equal(kd, ref_kp) and np.array_equal(vd, ref_vp)
     assert cache.alloc.free_list() == list(ref_alloc.free)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("depth", [1, 2, 3])
+def test_step_pipeline_matches_oracle_step_by_step(depth):
+    """StepPipeline: steps queued back to back over `depth` staging slots, with different
+    inputs every step and copy-on-write in the first; each step's output (read one step
+    late, as a serving loop would) must match the oracle, the final pools bit for bit."""
+    import paged_kv_cache_350_b200 as pa
+    w = workloads.prefix_cow(prompts=2, prompt_len=100)
+    steps = 7
+    MB = w.max_blocks + steps // w.block_size + 2
+    B = len(w.step_seqs)
+
+    def draws(t):
+        shapes = ((B, w.Hq, w.D), (B, w.Hkv, w.D), (B, w.Hkv, w.D))
+        return [workloads.draw_normal(s, w.seed + 17, 5000 + 3 * t + i, w.dtype)
+                for i, s in enumerate(shapes)]
+
+    # oracle replay
+    ref = RefAllocator(w.num_blocks, w.block_size, shuffle_seed=w.alloc_seed, pop_order=w.pop_order)
+    kp, vp = ref_copy_blocks(w.k_pool(), w.v_pool(), workloads.run_setup(w, ref))
+    outs = []
+    for t in range(steps):
+        q, nk, nv = draws(t)
+        slots, pairs = [], []
+        for sid in w.step_seqs:
+            slot, src, dst = ref.append_slot(sid)
+            slots.append(slot)
+            if src >= 0:
+                pairs.append((src, dst))
+        if t == 0:
+            assert pairs, "the first step copies on write"
+        kp, vp = ref_copy_blocks(kp, vp, pairs)
+        kp, vp = ref_reshape_and_cache(nk, nv, kp, vp, np.array(slots))
+        tables = np.full((B, MB), -1, dtype=np.int32)
+        lens = np.zeros(B, dtype=np.int32)
+        for i, sid in enumerate(w.step_seqs):
+            tab, n = ref.block_table(sid)
+            tables[i, :len(tab)] = tab
+            lens[i] = n
+        outs.append(ref_decode(q, kp, vp, tables, lens, w.scale))
+
+    def dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+
+    cache = pa.PagedKVCache(w.num_blocks, w.block_size, w.Hkv, w.D, shuffle_seed=w.alloc_seed,
+                            pop_order=w.pop_order, k_pool=dev(w.k_pool()), v_pool=dev(w.v_pool()))
+    setup_pairs = workloads.run_setup(w, cache.alloc)
+    pa.pa_copy_blocks(cache.k_pool, cache.v_pool,
+                      torch.tensor(setup_pairs, dtype=torch.int32, device="cuda").reshape(-1, 2))
+    pipe = cache.pipeline(B, w.Hq, MB, depth=depth)
+    got = []
+    lag = min(1, depth - 1)  # a slot holds its output until it is reused
+    for t in range(steps):
+        qh, kh, vh = pipe.inputs()
+        for dst, src in zip((qh, kh, vh), draws(t)):
+            dst.copy_(torch.from_numpy(np.ascontiguousarray(src).view(np.int16)).view(torch.bfloat16))
+        assert pipe.submit(w.step_seqs, w.scale) == t
+        if t >= lag:
+            got.append(pipe.result(t - lag).clone())
+    for t in range(steps - lag, steps):
+        got.append(pipe.result(t).clone())
+    pipe.sync()
+    cache.check_device_errors()
+    for t in range(steps):
+        assert_close(w, got[t], outs[t])
+    assert np.array_equal(cache.k_pool.view(torch.int16).cpu().numpy().view(np.uint16), kp)
+    assert np.array_equal(cache.v_pool.view(torch.int16).cpu().numpy().view(np.uint16), vp)
