@@ -130,7 +130,7 @@ static pa_status plan_decode(int B, int Hq, int Hkv, int D, int block_size, int 
 
   // Balanced persistent tensor-core kernel: the default for bf16 batches whose total
   // tile count (16-token tiles x KV heads) stays below 2^31.
-  const int64_t tile_bound = static_cast<int64_t>(B) * Hkv * ceil_div(max_seq, tc_tile);
+  const int64_t tile_bound = static_cast<int64_t>(B) * Hkv * ceil_div(max_seq, 16);
   if (tc_ok && partition == 0 && B <= kStreamMaxB && tile_bound < (int64_t(1) << 31)) {
     int grid = pa::stream_grid(D, block_size, G, B);
     if (max_ctas > 0 && grid > max_ctas) grid = max_ctas;

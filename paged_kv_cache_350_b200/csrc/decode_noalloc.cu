@@ -75,7 +75,7 @@ extern "C" pa_status pa_decode_no_alloc(void* out, const void* q, const void* k_
     return PA_ERR_INVALID_ARG;
   const int G = Hq / Hkv;
   if (!pa::tc_eligible(G, D, block_size, dtype) || B > kStreamMaxB) return PA_ERR_UNSUPPORTED;
-  const int tile = block_size > 16 ? block_size : 16;
+  const int tile = 16;  // the stream kernel's tokens per tile
   const int64_t max_seq = static_cast<int64_t>(max_blocks) * block_size;
   if (max_seq > 0x7fffffffLL) return PA_ERR_INVALID_ARG;
   if (static_cast<int64_t>(B) * Hkv * ((max_seq + tile - 1) / tile) >= (int64_t(1) << 31))

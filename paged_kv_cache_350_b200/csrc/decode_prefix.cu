@@ -563,8 +563,8 @@ template <class C>
 cudaError_t launch_pref_cfg(PrefixParams pp, int grid, cudaStream_t stream) {
   CUtensorMap tmk, tmv;
   const DecodeParams& p = pp.d;
-  if (!make_pool_map(&tmk, p.k_pool, p.num_blocks, C::BS, p.Hkv, C::D) ||
-      !make_pool_map(&tmv, p.v_pool, p.num_blocks, C::BS, p.Hkv, C::D))
+  if (!make_pool_map(&tmk, p.k_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BS) ||
+      !make_pool_map(&tmv, p.v_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BS))
     return cudaErrorInvalidValue;
   prefix_plan_kernel<C::TILE_T><<<1, kPlanThreads, 0, stream>>>(pp);
   cudaError_t e = cudaGetLastError();

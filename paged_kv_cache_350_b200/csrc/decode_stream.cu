@@ -5,10 +5,10 @@
 //
 // Schedule ("streams"):
 //   * Every (sequence b, KV head) is a unit of nt(b) = ceil(L_b / TILE_T) tiles of
-//     TILE_T tokens (32 by default: two blocks of 16); units are laid end to end in
-//     (b, KV head) order, T = Hkv * sum_b nt(b) tiles in all.
-//   * The grid is one wave of persistent CTAs (SM count x occupancy: 3 CTAs of 2 warps
-//     per SM by default).  Every warp is one stream: stream s owns the global tiles
+//     TILE_T = 16 tokens (one block of 16, two of 8, or half of a block of 32); units
+//     are laid end to end in (b, KV head) order, T = Hkv * sum_b nt(b) tiles in all.
+//   * The grid is one wave of persistent CTAs (SM count x occupancy: 2 CTAs of 4 warps
+//     per SM).  Every warp is one stream: stream s owns the global tiles
 //     [s*per, (s+1)*per), per = ceil(T / streams).  Work is balanced to one tile.
 //   * Each CTA first computes the prefix sums of nt(b) in shared memory; a global tile
 //     index maps to (b, KV head, tile) by binary search.
@@ -47,33 +47,33 @@ namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
 
-// Stage and CTA shape by block size.  Blocks of <= 16 tokens: 16-token stages (8 KB with
-// D = 128), 4 warps per CTA and 2 CTAs per SM, so every SM runs 8 streams, two on each of
-// its four sub-partitions (the tile math's issue and tensor rate per sub-partition is
-// part of the pace: 6 streams per SM left two sub-partitions with double load).  A
-// 32-token block needs a 32-token stage (16 KB): 2 warps per CTA, 3 CTAs per SM.
-// PA_STREAM_TILE / PA_STREAM_NCW / PA_STREAM_MIN_CTAS override all block sizes (sweeps).
+// Stage and CTA shape: 16-token stages (8 KB with D = 128; a 32-token block is staged
+// in two halves), 4 warps per CTA and 2 CTAs per SM, so every SM runs 8 streams, two on
+// each of its four sub-partitions (the tile math's issue and tensor rate per
+// sub-partition is part of the pace: 6 streams per SM left two sub-partitions with
+// double load).  PA_STREAM_TILE / PA_STREAM_NCW / PA_STREAM_MIN_CTAS override them
+// (sweeps).
 template <int BS>
 struct StreamShape {
 #ifdef PA_STREAM_TILE
   static constexpr int TILE = PA_STREAM_TILE;
 #else
-  static constexpr int TILE = BS <= 16 ? 16 : 32;
+  static constexpr int TILE = 16;
 #endif
 #ifdef PA_STREAM_NCW
   static constexpr int NCW = PA_STREAM_NCW;
 #else
-  static constexpr int NCW = BS <= 16 ? 4 : 2;
+  static constexpr int NCW = 4;
 #endif
 #ifdef PA_STREAM_MIN_CTAS
   static constexpr int MIN_CTAS = PA_STREAM_MIN_CTAS;
 #else
-  static constexpr int MIN_CTAS = BS <= 16 ? 2 : 3;
+  static constexpr int MIN_CTAS = 2;
 #endif
 };
 
 template <int D_, int BS_, bool ROWS16_, int SPW_>
-struct StreamCfg : TileCfg<D_, BS_, ROWS16_, StreamShape<BS_>::TILE> {
+struct StreamCfg : TileCfg<D_, BS_, ROWS16_, StreamShape<BS_>::TILE, true> {
   static constexpr int NCW = StreamShape<BS_>::NCW;  // warps (= streams) per CTA
   static constexpr int THREADS = NCW * 32;
   static constexpr int MIN_CTAS = StreamShape<BS_>::MIN_CTAS;  // register bound
@@ -82,8 +82,8 @@ struct StreamCfg : TileCfg<D_, BS_, ROWS16_, StreamShape<BS_>::TILE> {
   static constexpr int RING_BYTES = NST * StreamCfg::STAGE_BYTES;
   static constexpr int Q_BYTES = WarpAcc<StreamCfg, true>::Q_BYTES;  // per consumer warp
   // Q tiles per warp: two, so that the next unit's Q is copied in while the current unit
-  // streams; one for 16 query rows with 32-token stages, where a second would cost the
-  // third CTA per SM (the next unit's Q is then only prefetched into L2).
+  // streams; one for 16 query rows with 32-token stages (a sweep shape), where a second
+  // would cost a CTA per SM (the next unit's Q is then only prefetched into L2).
   static constexpr int QBUF = (StreamCfg::ROWS16 && StreamCfg::TILE_T == 32) ? 1 : 2;
   static constexpr int FIXED_BYTES = RING_BYTES + NCW * QBUF * Q_BYTES;
 };
@@ -130,22 +130,25 @@ __device__ __forceinline__ TilePos locate(const int* P, int B, int Hkv, int g) {
   return t;
 }
 
-// Block ids, KV head and block count of one tile, resolved by one lane.
+// Block ids, KV head, block count and first row inside the (first) block of one tile,
+// resolved by one lane.
 struct TileIds {
-  int kvh, nb;
+  int kvh, nb, row0;
   int id[4];
 };
 
 template <class C>
 __device__ __forceinline__ TileIds resolve_tile(const DecodeParams& p, const int* P, int g,
                                                 int end) {
-  TileIds r{0, 0, {0, 0, 0, 0}};
+  TileIds r{0, 0, 0, {0, 0, 0, 0}};
   if (g >= end) return r;
   const TilePos t = locate(P, p.B, p.Hkv, g);
   r.kvh = t.kvh;
   const int L = clamp_len(p, t.b, false);
   const int nblk = (L + C::BS - 1) / C::BS;
-  const int blk = t.j * C::BPS;
+  const int tok0 = t.j * C::TILE_T;
+  const int blk = tok0 / C::BS;
+  r.row0 = tok0 % C::BS;  // non-zero only when a stage holds part of a block
   r.nb = min(C::BPS, nblk - blk);
   const int32_t* tab = p.block_tables + static_cast<size_t>(t.b) * p.max_blocks + blk;
 #pragma unroll
@@ -276,6 +279,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_CTAS)
     const int src = k & 31;
     const int kv = __shfl_sync(kFull, cur.kvh, src);
     const int n = __shfl_sync(kFull, cur.nb, src);
+    const int row0 = __shfl_sync(kFull, cur.row0, src);
     int ids[C::BPS];
 #pragma unroll
     for (int q = 0; q < C::BPS; ++q) ids[q] = __shfl_sync(kFull, cur.id[q], src);
@@ -285,7 +289,7 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_CTAS)
       const uint32_t kt = smem_addr(smem + stage * C::STAGE_BYTES);
       const uint32_t vt = kt + C::TILE_BYTES;
       fence_proxy_async_smem();  // this stage's earlier generic reads/writes come first
-      mbar_arrive_expect_tx(fb, static_cast<uint32_t>(n * BS * D * 2 * 2));
+      mbar_arrive_expect_tx(fb, static_cast<uint32_t>(n * C::BOXR * D * 2 * 2));
 #pragma unroll
       for (int sub = 0; sub < C::BPS; ++sub) {
         if (sub >= n) break;
@@ -296,10 +300,10 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_CTAS)
         }
 #pragma unroll
         for (int c = 0; c < C::DCH; ++c) {
-          tma_load_4d(kt + c * C::CHUNK_BYTES + sub * BS * 128, &tmk, c * 64, kv, 0, phys, fb,
-                      policy);
-          tma_load_4d(vt + c * C::CHUNK_BYTES + sub * BS * 128, &tmv, c * 64, kv, 0, phys, fb,
-                      policy);
+          tma_load_4d(kt + c * C::CHUNK_BYTES + sub * C::BOXR * 128, &tmk, c * 64, kv, row0,
+                      phys, fb, policy);
+          tma_load_4d(vt + c * C::CHUNK_BYTES + sub * C::BOXR * 128, &tmv, c * 64, kv, row0,
+                      phys, fb, policy);
         }
       }
     }
@@ -311,7 +315,9 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_CTAS)
   const float sl2 = p.scale_log2;
   const bool append = sp.k_new != nullptr;
   constexpr int VPR = D / 8;
-  int unit_a = -1, a_starts = 0, unit_b = -1;
+  // The cut unit this stream owns (it starts in this stream's range and continues past
+  // it): unit id, slot of this stream's piece, number of pieces.
+  int own_u = -1, own_slot = 0, own_n = 0;
   int i = 0;  // tiles consumed by this stream (ring position)
   bool ok = true;
   WarpAcc<C, true> acc;
@@ -410,12 +416,10 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_CTAS)
           *reinterpret_cast<float2*>(sp.pacc + (row0 + g + 8) * D + 8 * jn + 2 * tig) =
               make_float2(acc.o_hi[jn][0], acc.o_hi[jn][1]);
       }
-      const int u = t.b * Hkv + t.kvh;
-      if (slot == 0) {
-        unit_a = u;
-        a_starts = gpos == ubeg ? 1 : 0;
-      } else {
-        unit_b = u;
+      if (ubeg >= beg) {  // the unit starts here: its pieces are streams s .. (uend-1)/per
+        own_u = t.b * Hkv + t.kvh;
+        own_slot = slot;
+        own_n = (uend - 1) / per - s + 1;
       }
     }
     gpos = pend;
@@ -431,20 +435,19 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_CTAS)
     }
   }
   if (lane == 0) {
-    int4 m = make_int4(ok ? unit_a : -1, ok ? a_starts : 0, ok ? unit_b : -1, 0);
+    int4 m = make_int4(ok ? own_u : -1, own_slot, own_n, 0);
     *reinterpret_cast<int4*>(sp.meta + s * 4) = m;
   }
 }
 
-// Merge the pieces of every unit cut by a stream boundary.  Block s owns the unit that
-// STARTS in stream s and continues into later streams: its piece is slot 1 of s (or
-// slot 0 when it spans the whole stream from its first tile); the other pieces are
-// slot 0 of the following streams, as long as their first piece is the same unit.
+// Merge the pieces of every unit cut by a stream boundary.  Block s merges the unit that
+// starts in stream s and continues into the following streams, recorded by stream s with
+// its piece count n: piece i is slot 0 of stream s + i, except the first, which is in
+// the slot stream s recorded.
 //
-// One thread per (query-head row, 4 output columns) of the owned unit: G * D/4 threads,
-// rounded up to whole warps.
-// Each thread merges the pieces online (running max, sum, output; base 2) with the
-// piece loop unrolled so their loads overlap; each warp counts the pieces itself.
+// One thread per (query-head row, 4 output columns) of the unit: G * D/4 threads,
+// rounded up to whole warps.  Each thread merges the pieces online (running max, sum,
+// output; base 2) with the piece loop unrolled so that their loads overlap.
 template <int D>
 __global__ void __launch_bounds__(512) stream_reduce_kernel(const StreamParams sp) {
 #if PA_STREAM_PDL
@@ -454,29 +457,8 @@ __global__ void __launch_bounds__(512) stream_reduce_kernel(const StreamParams s
   const DecodeParams& p = sp.d;
   const int s = blockIdx.x;
   const int4 m = *reinterpret_cast<const int4*>(sp.meta + static_cast<size_t>(s) * 4);
-  int u, slot;
-  if (m.z >= 0) {
-    u = m.z;
-    slot = 1;
-  } else if (m.x >= 0 && m.y) {
-    u = m.x;
-    slot = 0;
-  } else {
-    return;
-  }
-  const int lane = threadIdx.x & 31;
-  // Pieces are streams s .. s+n-1: find n with a warp-wide scan of the following streams.
-  int n = 1;
-  for (int base = s + 1;; base += 32) {
-    const int q = base + lane;
-    const bool same = q < sp.streams && sp.meta[static_cast<size_t>(q) * 4] == u;
-    const unsigned stop = __ballot_sync(kFull, !same);
-    if (stop) {
-      n += __ffs(stop) - 1;
-      break;
-    }
-    n += 32;
-  }
+  if (m.x < 0) return;
+  const int u = m.x, slot0 = m.y, n = m.z;
   const int G = p.G;
   const int r = threadIdx.x / (D / 4);
   const int c = (threadIdx.x % (D / 4)) * 4;
@@ -484,7 +466,7 @@ __global__ void __launch_bounds__(512) stream_reduce_kernel(const StreamParams s
   float M = -INFINITY, l = 0.f, a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll 4
   for (int i = 0; i < n; ++i) {
-    const size_t row = (static_cast<size_t>(s + i) * 2 + (i == 0 ? slot : 0)) * G + r;
+    const size_t row = (static_cast<size_t>(s + i) * 2 + (i == 0 ? slot0 : 0)) * G + r;
     const float2 ml = *reinterpret_cast<const float2*>(sp.pml + row * 2);
     const float4 a = *reinterpret_cast<const float4*>(sp.pacc + row * D + c);
     const float Mn = fmaxf(M, ml.x);
@@ -528,8 +510,8 @@ template <class C>
 cudaError_t launch_stream_cfg(const StreamParams& sp, int grid, cudaStream_t stream) {
   CUtensorMap tmk, tmv;
   const DecodeParams& p = sp.d;
-  if (!make_pool_map(&tmk, p.k_pool, p.num_blocks, C::BS, p.Hkv, C::D) ||
-      !make_pool_map(&tmv, p.v_pool, p.num_blocks, C::BS, p.Hkv, C::D))
+  if (!make_pool_map(&tmk, p.k_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BOXR) ||
+      !make_pool_map(&tmv, p.v_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BOXR))
     return cudaErrorInvalidValue;
   const size_t smem = stream_smem_bytes<C>(p.B);
   cudaError_t e = cudaFuncSetAttribute(decode_stream_kernel<C>,

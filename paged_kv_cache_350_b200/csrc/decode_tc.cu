@@ -257,7 +257,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 // columns of one KV head, 128-byte swizzled in shared memory.
 }  // namespace
 
-bool make_pool_map(CUtensorMap* map, const void* pool, int NB, int BS, int Hkv, int D) {
+bool make_pool_map(CUtensorMap* map, const void* pool, int NB, int BS, int Hkv, int D,
+                   int box_rows) {
   auto encode = get_encode_fn();
   if (!encode) return false;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hkv),
@@ -265,7 +266,7 @@ bool make_pool_map(CUtensorMap* map, const void* pool, int NB, int BS, int Hkv, 
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2,
                            static_cast<cuuint64_t>(Hkv) * D * 2,
                            static_cast<cuuint64_t>(BS) * Hkv * D * 2};
-  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(BS), 1};
+  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(pool), dims,
                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -279,8 +280,8 @@ namespace {
 template <class C>
 cudaError_t launch_cfg(const DecodeParams& p, cudaStream_t stream) {
   CUtensorMap tmk, tmv;
-  if (!make_pool_map(&tmk, p.k_pool, p.num_blocks, C::BS, p.Hkv, C::D) ||
-      !make_pool_map(&tmv, p.v_pool, p.num_blocks, C::BS, p.Hkv, C::D))
+  if (!make_pool_map(&tmk, p.k_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BS) ||
+      !make_pool_map(&tmv, p.v_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BS))
     return cudaErrorInvalidValue;
   auto kern = decode_tc_kernel<C>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -69,8 +69,10 @@ size_t prefix_workspace_bytes(int streams, int rows, int D);
 void prefix_carve(PrefixParams* pp, void* workspace, int rows);
 cudaError_t launch_decode_prefix(const PrefixParams& pp, int grid, cudaStream_t stream);
 
-// 4-D TMA view of a bf16 pool [NB][BS][Hkv][D]: box = BS rows x 64 columns of one head.
-bool make_pool_map(CUtensorMap* map, const void* pool, int NB, int BS, int Hkv, int D);
+// 4-D TMA view of a bf16 pool [NB][BS][Hkv][D]: box = box_rows rows (BS, or a part of a
+// block starting at a row coordinate) x 64 columns of one head.
+bool make_pool_map(CUtensorMap* map, const void* pool, int NB, int BS, int Hkv, int D,
+                   int box_rows);
 
 // Launch the bf16 tensor-core decode kernel (+ reduce when max_parts > 1).
 cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t stream);

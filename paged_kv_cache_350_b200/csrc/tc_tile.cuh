@@ -15,13 +15,16 @@
 namespace pa {
 
 // TT: tokens per pipeline stage when blocks are smaller (a stage holds whole blocks).
-template <int D_, int BS_, bool ROWS16_, int TT_ = 16>
+// SPLIT: a block larger than TT is staged as TT-token parts (a stage holds part of one
+// block) instead of the stage growing to the block.
+template <int D_, int BS_, bool ROWS16_, int TT_ = 16, bool SPLIT_ = false>
 struct TileCfg {
   static constexpr int D = D_;
   static constexpr int BS = BS_;
   static constexpr bool ROWS16 = ROWS16_;
-  static constexpr int TILE_T = BS > TT_ ? BS : TT_;  // tokens per pipeline stage
-  static constexpr int BPS = TILE_T / BS;            // blocks per stage
+  static constexpr int TILE_T = (SPLIT_ || BS <= TT_) ? TT_ : BS;  // tokens per pipeline stage
+  static constexpr int BPS = TILE_T >= BS ? TILE_T / BS : 1;      // blocks per stage
+  static constexpr int BOXR = BS < TILE_T ? BS : TILE_T;          // rows per TMA box
   static constexpr int SUBT = TILE_T / 16;           // 16-token sub-tiles per stage
   static constexpr int DCH = D / 64;                 // 128-byte column chunks per row
   static constexpr int CHUNK_BYTES = TILE_T * 128;
@@ -32,7 +35,8 @@ struct TileCfg {
   static constexpr int NT = D / 8;                      // output n-tiles of 8 columns
   static_assert(D == 64 || D == 128, "head dim");
   static_assert(BS == 8 || BS == 16 || BS == 32, "block size");
-  static_assert(TILE_T % 16 == 0 && BPS <= 4, "stage tokens");
+  static_assert(TILE_T % 16 == 0 && BPS <= 4 && (TILE_T % BS == 0 || BS % TILE_T == 0),
+                "stage tokens");
 };
 
 __device__ __forceinline__ uint32_t sw128(int row, int c16) {
