@@ -252,6 +252,39 @@ def pa_decode_append(out, q, k_new, v_new, k_pool, v_pool, block_tables, seq_len
     return out
 
 
+def decode_append_args(out, q, k_new, v_new, k_pool, v_pool, block_tables, seq_lens,
+                       workspace=None, err_flag=None, stream=None, partition_tokens=0,
+                       path=PA_PATH_AUTO, max_ctas=0):
+    """The checked argument list of a pa_decode_append call whose tensors stay fixed (a
+    caller that repeats the call, such as StepPipeline); run it with decode_append_call."""
+    import torch
+    _need(q.dim() == 3 and out.shape == q.shape, "q/out must be [B, Hq, D]")
+    _need(k_pool.dim() == 4 and v_pool.shape == k_pool.shape, "pools must be [NB, bs, Hkv, D]")
+    _need(block_tables.dim() == 2 and block_tables.dtype == torch.int32, "block_tables int32 [B, MB]")
+    _need(seq_lens.dtype == torch.int32 and seq_lens.numel() == q.shape[0], "seq_lens int32 [B]")
+    B, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_pool.shape
+    _need(D2 == D and block_tables.shape[0] == B, "shape mismatch")
+    _need(k_new.shape == (B, Hkv, D) and v_new.shape == k_new.shape, "k_new/v_new must be [B, Hkv, D]")
+    for t in (out, q, k_new, v_new, k_pool, v_pool, block_tables, seq_lens):
+        _need(t.is_contiguous(), "tensors must be contiguous")
+    _need(q.dtype == out.dtype == k_new.dtype == v_new.dtype == k_pool.dtype == v_pool.dtype,
+          "q, out, new K/V and pools share a dtype")
+    wbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    opts = pa_decode_opts(partition_tokens, path, max_ctas)
+    return [_ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool),
+            _ptr(block_tables), _ptr(seq_lens), B, Hq, Hkv, D, bs, block_tables.shape[1], NB,
+            0.0, _dtype_of(q), _ptr(workspace), wbytes, _ptr(err_flag), _stream(stream),
+            ctypes.byref(opts), opts]
+
+
+def decode_append_call(args, scale):
+    """Run a pa_decode_append argument list from decode_append_args with this scale."""
+    a = list(args[:-1])
+    a[15] = float(scale)
+    _check(lib.pa_decode_append(*a), "pa_decode_append")
+
+
 def pa_decode_no_alloc(out, q, k_pool, v_pool, block_tables, seq_lens, scale, err_flag=None,
                        stream=None):
     """pa_decode without a workspace, for callers that cannot allocate device memory.

@@ -278,7 +278,25 @@ class StepPipeline:
         self.used = [False] * depth   # slot has a step in flight (its events are recorded)
         self.next = 0                 # index of the next step to submit
         self.bytes_in = self.bytes_out = 0
-        cache.workspace(B, Hq, max_blocks)
+        self.ws = cache.workspace(B, Hq, max_blocks)
+        # Per slot, built once (the per-step host work is the allocator and the queueing):
+        # the allocator's output views in the pinned input, the device views the kernels
+        # read, and the argument list of the pa_decode_append call.
+        D, Hkv, dt = cache.D, cache.Hkv, cache.dtype
+        self.h_views, self.d_pairs, self.decode_args = [], [], []
+        for k in range(depth):
+            h, d = self.h_in[k], self.d_in[k]
+            self.h_views.append((self._view(h, "slots", (B,), torch.int64).numpy(),
+                                 self._view(h, "pairs", (B, 2), torch.int32).numpy(),
+                                 self._view(h, "tables", (B, max_blocks), torch.int32).numpy(),
+                                 self._view(h, "lens", (B,), torch.int32).numpy()))
+            self.d_pairs.append(self._view(d, "pairs", (B, 2), torch.int32))
+            self.decode_args.append(_b.decode_append_args(
+                self.d_out[k], self._view(d, "q", (B, Hq, D), dt), self._view(d, "k", (B, Hkv, D), dt),
+                self._view(d, "v", (B, Hkv, D), dt), cache.k_pool, cache.v_pool,
+                self._view(d, "tables", (B, max_blocks), torch.int32),
+                self._view(d, "lens", (B,), torch.int32), workspace=self.ws, err_flag=cache.err,
+                stream=self.stream))
 
     def _view(self, buf, name, shape, dtype):
         off, n = self.lay[name]
@@ -296,17 +314,16 @@ class StepPipeline:
 
     def submit(self, seq_ids, scale):
         """Queue one decode step for seq_ids (the inputs() of this step must be written)."""
-        c, B, MB = self.cache, self.B, self.max_blocks
+        c, B = self.cache, self.B
         ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
         assert ids.size == B, "the batch shape is fixed per pipeline"
         t, k = self.next, self.next % self.depth
         h, d = self.h_in[k], self.d_in[k]
+        slots_h, pairs_h, tables_h, lens_h = self.h_views[k]
         if self.used[k]:
             self.h2d_done[k].synchronize()   # normally long done: the copy of step t - depth
-        _, pairs = c.alloc.append_slots(ids, slot_out=self._view(h, "slots", (B,), torch.int64).numpy(),
-                                        pairs_out=self._view(h, "pairs", (B, 2), torch.int32).numpy())
-        c.alloc.block_tables(ids, MB, tables_out=self._view(h, "tables", (B, MB), torch.int32).numpy(),
-                             lens_out=self._view(h, "lens", (B,), torch.int32).numpy())
+        _, pairs = c.alloc.append_slots(ids, slot_out=slots_h, pairs_out=pairs_h)
+        c.alloc.block_tables(ids, self.max_blocks, tables_out=tables_h, lens_out=lens_h)
         npairs = pairs.shape[0]
         used = self.lay["pairs"][0] + npairs * 8 if npairs else self.lay["lens"][0] + B * 4
         if self.used[k]:
@@ -318,17 +335,10 @@ class StepPipeline:
         s.wait_event(self.h2d_done[k])
         if self.used[k]:
             s.wait_event(self.d2h_done[k])                 # d_out[k] was copied out
-        with torch.cuda.stream(s):
-            if npairs:
-                _b.pa_copy_blocks(c.k_pool, c.v_pool,
-                                  self._view(d, "pairs", (B, 2), torch.int32)[:npairs],
-                                  err_flag=c.err, stream=s)
-            _b.pa_decode_append(self.d_out[k], self._view(d, "q", (B, self.Hq, c.D), c.dtype),
-                                self._view(d, "k", (B, c.Hkv, c.D), c.dtype),
-                                self._view(d, "v", (B, c.Hkv, c.D), c.dtype), c.k_pool, c.v_pool,
-                                self._view(d, "tables", (B, MB), torch.int32),
-                                self._view(d, "lens", (B,), torch.int32), scale,
-                                workspace=c.workspace(B, self.Hq, MB), err_flag=c.err, stream=s)
+        if npairs:
+            _b.pa_copy_blocks(c.k_pool, c.v_pool, self.d_pairs[k][:npairs], err_flag=c.err,
+                              stream=s)
+        _b.decode_append_call(self.decode_args[k], scale)
         self.kern_done[k].record(s)
         self.copy_out.wait_event(self.kern_done[k])
         with torch.cuda.stream(self.copy_out):
