@@ -29,13 +29,19 @@ namespace pa {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kNCW = 2;                 // warps (= streams) per CTA
+// As in decode_stream.cu: 16-token stages (half of a 32-token block each), 4 warps per
+// CTA and 2 CTAs per SM, so every SM sub-partition runs two streams.  Shared prefixes
+// are multiples of PA_SHARED_PREFIX_ALIGN tokens, so no stage straddles a prefix end.
+constexpr int kNCW = 4;                 // warps (= streams) per CTA
 constexpr int kThreads = kNCW * 32;
+constexpr int kMinCtas = 2;             // CTAs per SM the register allocation allows
 constexpr int kSPW = 2;                 // ring stages per stream
 constexpr int kRows = 16;               // MMA rows of a unit (members x G of a group)
+constexpr int kTT = 16;                 // tokens per stage
+static_assert(PA_SHARED_PREFIX_ALIGN % kTT == 0, "a prefix ends on a stage boundary");
 
 template <int D_, int BS_>
-struct PrefCfg : TileCfg<D_, BS_, true, PA_SHARED_PREFIX_ALIGN> {
+struct PrefCfg : TileCfg<D_, BS_, true, kTT, true> {
   static constexpr int SPW = kSPW;
   static constexpr int NST = kNCW * SPW;
   static constexpr int RING_BYTES = NST * PrefCfg::STAGE_BYTES;
@@ -209,20 +215,21 @@ __device__ __forceinline__ TilePos locate(const int* P, int R, int Hkv, int g) {
 }
 
 struct TileIds {
-  int kvh, nb;
+  int kvh, nb, row0;
   int id[4];
 };
 
 template <class C>
 __device__ __forceinline__ TileIds resolve_tile(const PrefixParams& pp, const int* P, int R, int g,
                                                 int end) {
-  TileIds out{0, 0, {0, 0, 0, 0}};
+  TileIds out{0, 0, 0, {0, 0, 0, 0}};
   if (g >= end) return out;
   const DecodeParams& p = pp.d;
   const TilePos t = locate(P, R, p.Hkv, g);
   out.kvh = t.kvh;
   const TileSrc s = tile_src<C::TILE_T>(pp, t.r, t.j);
   const int blk = s.tok0 / C::BS;
+  out.row0 = s.tok0 % C::BS;  // non-zero only when a stage holds part of a block
   const int nblk = (s.tok1 + C::BS - 1) / C::BS;
   out.nb = min(C::BPS, nblk - blk);
   const int32_t* tab = p.block_tables + static_cast<size_t>(s.table_b) * p.max_blocks + blk;
@@ -282,10 +289,10 @@ __global__ void __launch_bounds__(kPlanThreads) prefix_plan_kernel(const PrefixP
 }
 
 template <class C>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, kMinCtas)
     decode_prefix_kernel(const __grid_constant__ CUtensorMap tmk,
                          const __grid_constant__ CUtensorMap tmv, const PrefixParams pp) {
-  constexpr int D = C::D, BS = C::BS, TILE_T = C::TILE_T, SPW = C::SPW, NST = C::NST;
+  constexpr int D = C::D, TILE_T = C::TILE_T, SPW = C::SPW, NST = C::NST;
   const DecodeParams& p = pp.d;
   const int B = p.B, Hkv = p.Hkv, G = p.G, NG = pp.ngroups;
   const int R = NG + B;
@@ -343,6 +350,7 @@ __global__ void __launch_bounds__(kThreads)
     const int src = k & 31;
     const int kv = __shfl_sync(kFull, cur.kvh, src);
     const int n = __shfl_sync(kFull, cur.nb, src);
+    const int row0 = __shfl_sync(kFull, cur.row0, src);
     int ids[C::BPS];
 #pragma unroll
     for (int q = 0; q < C::BPS; ++q) ids[q] = __shfl_sync(kFull, cur.id[q], src);
@@ -352,7 +360,7 @@ __global__ void __launch_bounds__(kThreads)
       const uint32_t kt = smem_addr(smem + stage * C::STAGE_BYTES);
       const uint32_t vt = kt + C::TILE_BYTES;
       fence_proxy_async_smem();
-      mbar_arrive_expect_tx(fb, static_cast<uint32_t>(n * BS * D * 2 * 2));
+      mbar_arrive_expect_tx(fb, static_cast<uint32_t>(n * C::BOXR * D * 2 * 2));
 #pragma unroll
       for (int sub = 0; sub < C::BPS; ++sub) {
         if (sub >= n) break;
@@ -363,10 +371,10 @@ __global__ void __launch_bounds__(kThreads)
         }
 #pragma unroll
         for (int c = 0; c < C::DCH; ++c) {
-          tma_load_4d(kt + c * C::CHUNK_BYTES + sub * BS * 128, &tmk, c * 64, kv, 0, phys, fb,
-                      policy);
-          tma_load_4d(vt + c * C::CHUNK_BYTES + sub * BS * 128, &tmv, c * 64, kv, 0, phys, fb,
-                      policy);
+          tma_load_4d(kt + c * C::CHUNK_BYTES + sub * C::BOXR * 128, &tmk, c * 64, kv, row0,
+                      phys, fb, policy);
+          tma_load_4d(vt + c * C::CHUNK_BYTES + sub * C::BOXR * 128, &tmv, c * 64, kv, row0,
+                      phys, fb, policy);
         }
       }
     }
@@ -391,21 +399,54 @@ __global__ void __launch_bounds__(kThreads)
     const int pend = min(end, uend);
     const int u = t.r * Hkv + t.kvh;
     const bool is_group = t.r < NG;
-    const int nrows = is_group ? group_size(pp, t.r) * G : G;
+    // The unit's sources, resolved once (the same rules as row_tiles / tile_src): for a
+    // group, lane m < gs holds member m's batch row mb, length mL and the unit tile mst
+    // where its own tokens start (after the np shared tiles); a tile's member is then a
+    // ballot, with no global load per tile.  An ungrouped sequence: its row and length.
+    int gs = 1, np = 0, pre = 0, mb = -1, mL = 0, mst = 0x7fffffff;
+    if (is_group) {
+      pre = group_prefix_tokens(pp, t.r, false);
+      np = pre / TILE_T;
+      const int id = lane < pp.max_members ? member_of(pp, t.r, lane) : -1;
+      gs = __ffs(~__ballot_sync(kFull, id >= 0)) - 1;  // members before the first -1
+      int own = 0;
+      if (lane < gs) {
+        mb = id;
+        if (id < B) {
+          mL = clamp_len(p, id, false);
+          if (mL >= pre) own = (mL - pre + TILE_T - 1) / TILE_T;
+        }
+      }
+      int incl = own;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(kFull, incl, off);
+        if (lane >= off) incl += v;
+      }
+      if (lane < gs) mst = np + incl - own;
+    } else {
+      mb = t.r - NG;
+      mL = clamp_len(p, mb, false);
+    }
+    const int nrows = is_group ? gs * G : G;
+    // batch row of MMA row rr (member rr / G of a group, or the sequence)
+    auto row_b = [&](int rr) { return __shfl_sync(kFull, mb, is_group ? rr / G : 0); };
     // Stage the unit's Q rows: a group's members' heads of this KV head, or the sequence's.
     {
       constexpr int CPR = D * 2 / 16;
       __syncwarp();
-      for (int idx = lane; idx < kRows * CPR; idx += 32) {
+      for (int idx0 = 0; idx0 < kRows * CPR; idx0 += 32) {
+        const int idx = idx0 + lane;
         const int rr = idx / CPR, c = idx - rr * CPR;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (rr < nrows) {
-          int b, h;
-          row_target(pp, t.r, t.kvh, rr, b, h);
-          if (b >= 0 && b < B)
+        const int b = row_b(rr < kRows ? rr : 0);
+        if (idx < kRows * CPR) {
+          uint4 v = make_uint4(0u, 0u, 0u, 0u);
+          if (rr < nrows && b >= 0 && b < B) {
+            const int h = t.kvh * G + (is_group ? rr % G : rr);
             v = __ldg(reinterpret_cast<const uint4*>(qbase + (static_cast<size_t>(b) * p.Hq + h) * D) + c);
+          }
+          *reinterpret_cast<uint4*>(my_q + WarpAcc<C, true>::q_off(rr, c)) = v;
         }
-        *reinterpret_cast<uint4*>(my_q + WarpAcc<C, true>::q_off(rr, c)) = v;
       }
       acc.qs = smem_addr(my_q);
       __syncwarp();
@@ -418,12 +459,23 @@ __global__ void __launch_bounds__(kThreads)
         ok = false;
         break;
       }
-      const TileSrc src = tile_src<TILE_T>(pp, t.r, j);
+      int valid, row_lo = 0, row_hi = kRows;
+      if (!is_group) {
+        valid = min(TILE_T, mL - j * TILE_T);
+      } else if (j < np) {
+        valid = TILE_T;  // shared tokens: the prefix is a whole number of stages
+      } else {
+        const unsigned mk = __ballot_sync(kFull, lane < gs && mst <= j);
+        const int m = 31 - __clz(mk);
+        const int Lm = __shfl_sync(kFull, mL, m), sm = __shfl_sync(kFull, mst, m);
+        valid = min(TILE_T, Lm - (pre + (j - sm) * TILE_T));
+        row_lo = m * G;
+        row_hi = row_lo + G;
+      }
       uint8_t* st_ptr = smem + stage * C::STAGE_BYTES;
-      const int valid = min(TILE_T, src.tok1 - src.tok0);
       if (valid < TILE_T) zero_tail_rows<C>(st_ptr, valid, lane);
       if (is_group)
-        acc.template tile<true>(smem_addr(st_ptr), valid, sl2, lane, src.row_lo, src.row_hi);
+        acc.template tile<true>(smem_addr(st_ptr), valid, sl2, lane, row_lo, row_hi);
       else
         acc.tile(smem_addr(st_ptr), valid, sl2, lane);
       __syncwarp();
@@ -434,15 +486,15 @@ __global__ void __launch_bounds__(kThreads)
     const bool complete = (gpos == ubeg) && (pend == uend);
     if (complete) {
       const float inv_lo = 1.f / acc.l_lo, inv_hi = 1.f / acc.l_hi;
-      int b0, h0, b1, h1;
-      row_target(pp, t.r, t.kvh, g, b0, h0);
-      row_target(pp, t.r, t.kvh, g + 8, b1, h1);
+      const int b0 = row_b(g), b1 = row_b(g + 8);
+      const int h0 = t.kvh * G + (is_group ? g % G : g);
+      const int h1 = t.kvh * G + (is_group ? (g + 8) % G : g + 8);
 #pragma unroll
       for (int jn = 0; jn < C::NT; ++jn) {
-        if (g < nrows)
+        if (g < nrows && b0 >= 0 && b0 < B)  // a member id outside [0, B) has no output row
           *reinterpret_cast<uint32_t*>(out + (static_cast<size_t>(b0) * p.Hq + h0) * D + 8 * jn + 2 * tig) =
               pack_bf16x2(acc.o_lo[jn][0] * inv_lo, acc.o_lo[jn][1] * inv_lo);
-        if (g + 8 < nrows)
+        if (g + 8 < nrows && b1 >= 0 && b1 < B)
           *reinterpret_cast<uint32_t*>(out + (static_cast<size_t>(b1) * p.Hq + h1) * D + 8 * jn + 2 * tig) =
               pack_bf16x2(acc.o_hi[jn][0] * inv_hi, acc.o_hi[jn][1] * inv_hi);
       }
@@ -563,8 +615,8 @@ template <class C>
 cudaError_t launch_pref_cfg(PrefixParams pp, int grid, cudaStream_t stream) {
   CUtensorMap tmk, tmv;
   const DecodeParams& p = pp.d;
-  if (!make_pool_map(&tmk, p.k_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BS) ||
-      !make_pool_map(&tmv, p.v_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BS))
+  if (!make_pool_map(&tmk, p.k_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BOXR) ||
+      !make_pool_map(&tmv, p.v_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BOXR))
     return cudaErrorInvalidValue;
   prefix_plan_kernel<C::TILE_T><<<1, kPlanThreads, 0, stream>>>(pp);
   cudaError_t e = cudaGetLastError();
