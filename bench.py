@@ -373,8 +373,8 @@ def run_ours(args):
         pre_of = np.where(gof >= 0, np.asarray(gpre, dtype=np.int64)[np.maximum(gof, 0)] if ng else 0, 0)
         tok_unique = int(np.asarray(gpre, dtype=np.int64).sum()) + int((lens - pre_of).sum())
         unique_kv = 2 * tok_unique * w.Hkv * w.D * esize
-        plan = {"kernel": "shared_prefix", "groups": ng, "max_members": maxm, "launches": 3}
-        launches_per_step = 3 + 1 + (1 if npairs else 0)
+        plan = {"kernel": "shared_prefix", "groups": ng, "max_members": maxm, "launches": 2}
+        launches_per_step = 2 + 1 + (1 if npairs else 0)
 
     def step(ev=None):
         if npairs:

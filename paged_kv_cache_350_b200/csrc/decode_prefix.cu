@@ -252,42 +252,6 @@ __device__ __forceinline__ void row_target(const PrefixParams& pp, int r, int kv
   }
 }
 
-// Tile counts of every unit row, scanned: P[r] = tiles of rows before r, P[R] = total (in
-// rows of Hkv units).  One block; one row per thread per pass, so the dependent loads of
-// different rows (group -> members -> lengths) overlap.
-constexpr int kPlanThreads = 1024;
-
-template <int TT>
-__global__ void __launch_bounds__(kPlanThreads) prefix_plan_kernel(const PrefixParams pp) {
-  // The main kernel may launch now: it waits for this grid before reading the plan.
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int R = pp.ngroups + pp.d.B;
-  __shared__ int carry;
-  __shared__ int warp_tot[kPlanThreads / 32];
-  if (threadIdx.x == 0) carry = 0;
-  __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int base = 0; base < R; base += kPlanThreads) {
-    const int r = base + static_cast<int>(threadIdx.x);
-    const int n = r < R ? row_tiles<TT>(pp, r, true) : 0;
-    int incl = n;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int v = __shfl_up_sync(kFull, incl, off);
-      if (lane >= off) incl += v;
-    }
-    if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
-    int before = carry;
-    for (int w = 0; w < warp; ++w) before += warp_tot[w];
-    if (r < R) pp.plan[r] = before + incl - n;
-    __syncthreads();
-    if (threadIdx.x == kPlanThreads - 1) carry = before + incl;
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) pp.plan[R] = carry;
-}
-
 template <class C>
 __global__ void __launch_bounds__(kThreads, kMinCtas)
     decode_prefix_kernel(const __grid_constant__ CUtensorMap tmk,
@@ -306,16 +270,44 @@ __global__ void __launch_bounds__(kThreads, kMinCtas)
   int* P = reinterpret_cast<int*>(smem + C::FIXED_BYTES);  // [R + 1] tiles before row r
   __shared__ __align__(8) uint64_t full_bar[NST];
 
+  __shared__ int warp_sum[kNCW];
   if (threadIdx.x == 0) {
     for (int st = 0; st < NST; ++st) mbar_init(smem_addr(&full_bar[st]), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_proxy_async_smem();
   }
-  // Everything below reads what earlier kernels wrote: wait for the plan kernel (which
-  // itself ran after every earlier kernel on the stream) to complete.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  for (int r = threadIdx.x; r <= R; r += kThreads) P[r] = pp.plan[r];
+  // ---- tile counts of every unit row, scanned (every CTA, identical): P[r] = tiles of
+  // the rows before r, P[R] = total.  Rows first, with their dependent loads (group ->
+  // members -> lengths) overlapping across threads, then an in-place scan.
+  for (int r = threadIdx.x; r < R; r += kThreads) P[r] = row_tiles<TILE_T>(pp, r, blockIdx.x == 0);
+  __syncthreads();
+  {
+    const int chunk = (R + kThreads - 1) / kThreads;
+    const int lo = min(R, static_cast<int>(threadIdx.x) * chunk);
+    const int hi = min(R, lo + chunk);
+    int sum = 0;
+    for (int r = lo; r < hi; ++r) sum += P[r];
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(kFull, incl, off);
+      if (lane >= off) incl += v;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
+    __syncthreads();
+    int run = incl - sum;
+    for (int w = 0; w < warp; ++w) run += warp_sum[w];
+    for (int r = lo; r < hi; ++r) {
+      const int n = P[r];
+      P[r] = run;
+      run += n;
+    }
+    if (threadIdx.x == 0) {
+      int total = 0;
+      for (int w = 0; w < kNCW; ++w) total += warp_sum[w];
+      P[R] = total;
+    }
+  }
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
   for (int b = blockIdx.x; b < B; b += gridDim.x) {
     if (clamp_len(p, b, false) == 0) {
@@ -332,6 +324,8 @@ __global__ void __launch_bounds__(kThreads, kMinCtas)
   const int T = Hkv * P[R];
   const int S = static_cast<int>(gridDim.x) * kNCW;
   const int per = (T + S - 1) / S;
+  // Let the cut reduce be launched now; it waits for this grid to complete.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int s = static_cast<int>(blockIdx.x) * kNCW + warp;
   const int beg = min(T, s * per);
   const int end = min(T, beg + per);
@@ -384,7 +378,9 @@ __global__ void __launch_bounds__(kThreads, kMinCtas)
 
   const int g = lane >> 2, tig = lane & 3;
   const float sl2 = p.scale_log2;
-  int unit_a = -1, a_starts = 0, unit_b = -1;
+  // The cut unit this stream owns (it starts in this stream's range and continues past
+  // it): unit id, slot of this stream's piece, number of pieces.
+  int own_u = -1, own_slot = 0, own_n = 0;
   int i = 0;
   bool ok = true;
   WarpAcc<C, true> acc;
@@ -501,11 +497,10 @@ __global__ void __launch_bounds__(kThreads, kMinCtas)
     } else {
       const int slot = gpos == beg ? 0 : 1;  // a cut piece is the stream's first or last
       const size_t row0 = (static_cast<size_t>(s) * 2 + slot) * kRows;
-      if (slot == 0) {
-        unit_a = u;
-        a_starts = gpos == ubeg ? 1 : 0;
-      } else {
-        unit_b = u;
+      if (ubeg >= beg) {  // the unit starts here: its pieces are streams s .. (uend-1)/per
+        own_u = u;
+        own_slot = slot;
+        own_n = (uend - 1) / per - s + 1;
       }
       if (tig == 0) {
         if (g < nrows)
@@ -532,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtas)
     }
   }
   if (lane == 0) {
-    int4 m = make_int4(ok ? unit_a : -1, ok ? a_starts : 0, ok ? unit_b : -1, 0);
+    int4 m = make_int4(ok ? own_u : -1, own_slot, own_n, 0);
     *reinterpret_cast<int4*>(pp.meta + s * 4) = m;
   }
 }
@@ -545,29 +540,10 @@ __global__ void __launch_bounds__(512) prefix_cut_reduce_kernel(const PrefixPara
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const DecodeParams& p = pp.d;
   const int s = blockIdx.x;
+  // the unit stream s owns, recorded with the slot of its first piece and the piece count
   const int4 m = *reinterpret_cast<const int4*>(pp.meta + static_cast<size_t>(s) * 4);
-  int u, slot;
-  if (m.z >= 0) {
-    u = m.z;
-    slot = 1;
-  } else if (m.x >= 0 && m.y) {
-    u = m.x;
-    slot = 0;
-  } else {
-    return;
-  }
-  const int lane = threadIdx.x & 31;
-  int n = 1;
-  for (int base = s + 1;; base += 32) {
-    const int q = base + lane;
-    const bool same = q < pp.streams && pp.meta[static_cast<size_t>(q) * 4] == u;
-    const unsigned stop = __ballot_sync(kFull, !same);
-    if (stop) {
-      n += __ffs(stop) - 1;
-      break;
-    }
-    n += 32;
-  }
+  if (m.x < 0) return;
+  const int u = m.x, slot = m.y, n = m.z;
   const int r = u / p.Hkv, kvh = u - r * p.Hkv;
   const int nrows = r < pp.ngroups ? group_size(pp, r) * p.G : p.G;
   const int row = threadIdx.x / (D / 4);
@@ -618,25 +594,21 @@ cudaError_t launch_pref_cfg(PrefixParams pp, int grid, cudaStream_t stream) {
   if (!make_pool_map(&tmk, p.k_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BOXR) ||
       !make_pool_map(&tmv, p.v_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BOXR))
     return cudaErrorInvalidValue;
-  prefix_plan_kernel<C::TILE_T><<<1, kPlanThreads, 0, stream>>>(pp);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
   const size_t smem = pref_smem_bytes<C>(pp.ngroups + p.B);
-  e = cudaFuncSetAttribute(decode_prefix_kernel<C>,
+  cudaError_t e = cudaFuncSetAttribute(decode_prefix_kernel<C>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
+  decode_prefix_kernel<C><<<grid, kThreads, smem, stream>>>(tmk, tmv, pp);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // the cut reduce, as a programmatic dependent of the main kernel
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if ((e = cudaLaunchKernelEx(&cfg, decode_prefix_kernel<C>, tmk, tmv, pp)) != cudaSuccess) return e;
   cfg.gridDim = dim3(static_cast<unsigned>(pp.streams));
   cfg.blockDim = dim3(kRows * C::D / 4);
   cfg.dynamicSmemBytes = 0;
@@ -665,22 +637,19 @@ int prefix_warps_per_cta() { return kNCW; }
 
 size_t prefix_workspace_bytes(int streams, int rows, int D) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  (void)rows;
   return up(static_cast<size_t>(streams) * 16) + up(static_cast<size_t>(streams) * 2 * kRows * 8) +
-         up(static_cast<size_t>(streams) * 2 * kRows * D * 4) +
-         static_cast<size_t>(rows + 1) * 4;
+         static_cast<size_t>(streams) * 2 * kRows * D * 4;
 }
 
 void prefix_carve(PrefixParams* pp, void* workspace, int rows) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   char* w = static_cast<char*>(workspace);
-  const int D = pp->d.D;
   pp->meta = reinterpret_cast<int32_t*>(w);
   w += up(static_cast<size_t>(pp->streams) * 16);
   pp->pml = reinterpret_cast<float*>(w);
   w += up(static_cast<size_t>(pp->streams) * 2 * kRows * 8);
   pp->pacc = reinterpret_cast<float*>(w);
-  w += up(static_cast<size_t>(pp->streams) * 2 * kRows * D * 4);
-  pp->plan = reinterpret_cast<int32_t*>(w);
   (void)rows;
 }
 

@@ -61,7 +61,6 @@ struct PrefixParams {
   int32_t* meta;   // [streams][4] cut-unit slot metadata
   float* pml;      // [streams][2][16][2]
   float* pacc;     // [streams][2][16][D]
-  int32_t* plan;   // [ngroups + B + 1] scanned tile counts of the unit rows
 };
 int prefix_grid(int D, int block_size, int R);
 int prefix_warps_per_cta();
