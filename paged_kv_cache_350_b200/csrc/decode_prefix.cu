@@ -46,7 +46,8 @@ struct PrefCfg : TileCfg<D_, BS_, true, kTT, true> {
   static constexpr int NST = kNCW * SPW;
   static constexpr int RING_BYTES = NST * PrefCfg::STAGE_BYTES;
   static constexpr int Q_BYTES = WarpAcc<PrefCfg, true>::Q_BYTES;
-  static constexpr int FIXED_BYTES = RING_BYTES + kNCW * Q_BYTES;
+  // two Q tiles per warp: the next unit's rows are copied in while the current streams
+  static constexpr int FIXED_BYTES = RING_BYTES + kNCW * 2 * Q_BYTES;
 };
 
 template <class C>
@@ -384,35 +385,71 @@ __global__ void __launch_bounds__(kThreads, kMinCtas)
   int i = 0;
   bool ok = true;
   WarpAcc<C, true> acc;
-  uint8_t* my_q = qtiles + warp * C::Q_BYTES;
+  uint8_t* my_q = qtiles + warp * 2 * C::Q_BYTES;
   const __nv_bfloat16* qbase = static_cast<const __nv_bfloat16*>(p.q);
+  // A unit's inputs, lane-distributed: a group's member ids (lane m) and shared tokens, or
+  // an ungrouped sequence's row; then their lengths.  The next unit's are loaded while
+  // the current one streams: ids at its start, lengths after its first tile.
+  auto load_ids = [&](const TilePos& u, int& id, int& pre) {
+    if (u.r < NG) {
+      id = lane < pp.max_members ? member_of(pp, u.r, lane) : -1;
+      pre = group_prefix_tokens(pp, u.r, false);
+    } else {
+      id = u.r - NG;
+      pre = 0;
+    }
+  };
+  auto load_len = [&](const TilePos& u, int id) {
+    if (u.r < NG) return (id >= 0 && id < B) ? clamp_len(p, id, false) : 0;
+    return clamp_len(p, id, false);
+  };
+  // Copy unit u's Q rows into a Q tile with cp.async (rows past the unit's, or of a
+  // member id outside [0, B), zero-filled): a group's members' heads of its KV head,
+  // or the sequence's.
+  auto prefetch_q = [&](const TilePos& u, int id, uint8_t* tile) {
+    constexpr int CPR = D * 2 / 16;
+    const bool grp = u.r < NG;
+    const int gs = grp ? __ffs(~__ballot_sync(kFull, id >= 0)) - 1 : 1;
+    const int nrows = grp ? gs * G : G;
+    for (int idx0 = 0; idx0 < kRows * CPR; idx0 += 32) {
+      const int idx = idx0 + lane;
+      const int rr = idx / CPR, c = idx - rr * CPR;
+      const int b = __shfl_sync(kFull, id, grp ? (rr < kRows ? rr : 0) / G : 0);
+      const bool live = rr < nrows && b >= 0 && b < B;
+      const int h = u.kvh * G + (grp ? rr % G : rr);
+      const __nv_bfloat16* src = qbase + (live ? (static_cast<size_t>(b) * p.Hq + h) * D : 0);
+      if (idx < kRows * CPR)
+        cp_async_16_zfill(smem_addr(tile + WarpAcc<C, true>::q_off(rr, c)),
+                          reinterpret_cast<const uint4*>(src) + (live ? c : 0), live ? 16 : 0);
+    }
+    cp_async_commit();
+  };
 
   int gpos = beg;
+  int qb = 0;                  // Q tile of the current unit
+  TilePos t{};
+  int cid = -1, cpre = 0, cL = 0;  // the current unit's inputs
+  if (gpos < end) {
+    t = locate(P, R, Hkv, gpos);
+    load_ids(t, cid, cpre);
+    cL = load_len(t, cid);
+    prefetch_q(t, cid, my_q);
+  }
   while (gpos < end && ok) {
-    const TilePos t = locate(P, R, Hkv, gpos);
     const int ubeg = Hkv * P[t.r] + t.kvh * t.nt;
     const int uend = ubeg + t.nt;
     const int pend = min(end, uend);
     const int u = t.r * Hkv + t.kvh;
     const bool is_group = t.r < NG;
-    // The unit's sources, resolved once (the same rules as row_tiles / tile_src): for a
-    // group, lane m < gs holds member m's batch row mb, length mL and the unit tile mst
-    // where its own tokens start (after the np shared tiles); a tile's member is then a
-    // ballot, with no global load per tile.  An ungrouped sequence: its row and length.
-    int gs = 1, np = 0, pre = 0, mb = -1, mL = 0, mst = 0x7fffffff;
+    // The unit's sources (the same rules as row_tiles / tile_src): for a group, lane
+    // m < gs holds member m's batch row mb, length mL and the unit tile mst where its own
+    // tokens start (after the np shared tiles); a tile's member is then a ballot, with no
+    // global load per tile.  An ungrouped sequence: its row and length.
+    int gs = 1, mb = cid, mL = cL, mst = 0x7fffffff;
+    const int pre = cpre, np = cpre / TILE_T;
     if (is_group) {
-      pre = group_prefix_tokens(pp, t.r, false);
-      np = pre / TILE_T;
-      const int id = lane < pp.max_members ? member_of(pp, t.r, lane) : -1;
-      gs = __ffs(~__ballot_sync(kFull, id >= 0)) - 1;  // members before the first -1
-      int own = 0;
-      if (lane < gs) {
-        mb = id;
-        if (id < B) {
-          mL = clamp_len(p, id, false);
-          if (mL >= pre) own = (mL - pre + TILE_T - 1) / TILE_T;
-        }
-      }
+      gs = __ffs(~__ballot_sync(kFull, cid >= 0)) - 1;  // members before the first -1
+      const int own = (lane < gs && cid < B && cL >= pre) ? (cL - pre + TILE_T - 1) / TILE_T : 0;
       int incl = own;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -420,33 +457,20 @@ __global__ void __launch_bounds__(kThreads, kMinCtas)
         if (lane >= off) incl += v;
       }
       if (lane < gs) mst = np + incl - own;
-    } else {
-      mb = t.r - NG;
-      mL = clamp_len(p, mb, false);
+      else mb = -1;
     }
     const int nrows = is_group ? gs * G : G;
     // batch row of MMA row rr (member rr / G of a group, or the sequence)
     auto row_b = [&](int rr) { return __shfl_sync(kFull, mb, is_group ? rr / G : 0); };
-    // Stage the unit's Q rows: a group's members' heads of this KV head, or the sequence's.
-    {
-      constexpr int CPR = D * 2 / 16;
-      __syncwarp();
-      for (int idx0 = 0; idx0 < kRows * CPR; idx0 += 32) {
-        const int idx = idx0 + lane;
-        const int rr = idx / CPR, c = idx - rr * CPR;
-        const int b = row_b(rr < kRows ? rr : 0);
-        if (idx < kRows * CPR) {
-          uint4 v = make_uint4(0u, 0u, 0u, 0u);
-          if (rr < nrows && b >= 0 && b < B) {
-            const int h = t.kvh * G + (is_group ? rr % G : rr);
-            v = __ldg(reinterpret_cast<const uint4*>(qbase + (static_cast<size_t>(b) * p.Hq + h) * D) + c);
-          }
-          *reinterpret_cast<uint4*>(my_q + WarpAcc<C, true>::q_off(rr, c)) = v;
-        }
-      }
-      acc.qs = smem_addr(my_q);
-      __syncwarp();
+    // the next unit of this stream (if any) starts at tile pend
+    const bool has_next = pend < end;
+    TilePos tn{};
+    int nid = -1, npre = 0, nL = 0;
+    if (has_next) {
+      tn = locate(P, R, Hkv, pend);
+      load_ids(tn, nid, npre);
     }
+    acc.use_q(my_q + qb * C::Q_BYTES);
     acc.reset();
     const int jend = t.j + (pend - gpos);
     for (int j = t.j; j < jend; ++j, ++i) {
@@ -476,6 +500,10 @@ __global__ void __launch_bounds__(kThreads, kMinCtas)
         acc.tile(smem_addr(st_ptr), valid, sl2, lane);
       __syncwarp();
       if (i + SPW < cnt) issue(i + SPW);
+      if (j == t.j && has_next) {  // the next unit's ids have landed by now
+        nL = load_len(tn, nid);
+        prefetch_q(tn, nid, my_q + (qb ^ 1) * C::Q_BYTES);
+      }
     }
     if (!ok) break;
     acc.reduce_l();
@@ -519,7 +547,13 @@ __global__ void __launch_bounds__(kThreads, kMinCtas)
       }
     }
     gpos = pend;
+    t = tn;
+    cid = nid;
+    cpre = npre;
+    cL = nL;
+    qb ^= 1;
   }
+  cp_async_wait_all();  // a Q copy still in flight after an early exit
   if (!ok) {
     for (int k = i; k < cnt && k < i + SPW; ++k) {
       const int stage = warp * SPW + k % SPW;
