@@ -157,3 +157,61 @@ def test_bad_table_entry_and_bad_length_write_nothing_and_flag():
         assert err & pa.binding.PA_DEVERR_BAD_SEQ_LEN
         assert (k1 != kp).any(dim=-1).any(dim=-1).nonzero().tolist() == [[2, 4]]
 
+
+
+def test_workspace_contents_do_not_matter():
+    """The workspace needs no initialisation: NaN- or garbage-filled, the result is the
+    same bit for bit as with a zeroed one (every word a call reads it writes first)."""
+    import paged_kv_cache_350_b200 as pa
+    w = SCALED["gqa"]()
+    g = gpu_step(w, keep=True, fused=True, max_ctas=5)  # few CTAs: many cut units
+    outs = []
+    for fill in (0, 0xFF, 0x7F):
+        ws = torch.full_like(g["ws"], fill)
+        kp, vp = g["k_pool"].clone(), g["v_pool"].clone()
+        out = torch.empty_like(g["q"])
+        nk, nv = g["nk"], g["nv"]
+        pa.pa_decode_append(out, g["q"], nk, nv, kp, vp, g["t_d"], g["l_d"], w.scale,
+                            workspace=ws, max_ctas=5)
+        torch.cuda.synchronize()
+        outs.append(out)
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+    assert torch.equal(outs[0], g["out"])
+
+
+def test_step_replayed_from_a_cuda_graph():
+    """One fused decode step captured in a CUDA graph and replayed: every replay gives the
+    eager call's output bit for bit (the cache write is idempotent for a repeated step)."""
+    import paged_kv_cache_350_b200 as pa
+    w = SCALED["gqa"]()
+    g = gpu_step(w, keep=True, fused=True)
+    kp, vp = g["k_pool"], g["v_pool"]
+    out = torch.empty_like(g["q"])
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):  # warm-up on the capture stream (first-call setup)
+        pa.pa_decode_append(out, g["q"], g["nk"], g["nv"], kp, vp, g["t_d"], g["l_d"], w.scale,
+                            workspace=g["ws"], err_flag=err, stream=s)
+    s.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        pa.pa_decode_append(out, g["q"], g["nk"], g["nv"], kp, vp, g["t_d"], g["l_d"], w.scale,
+                            workspace=g["ws"], err_flag=err, stream=s)
+    for _ in range(3):
+        out.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        assert torch.equal(out, g["out"])
+    del graph
+
+
+def test_plan_on_b200_takes_the_stream_kernel_for_every_block_size():
+    import paged_kv_cache_350_b200 as pa
+    for bs in (8, 16, 32):
+        n = pa.pa_decode_workspace_size(256, 32, 8, 128, 4096, bs, 0)
+        plan = pa.pa_decode_plan(256, 32, 8, 128, bs, 4096 // bs, pa.PA_BF16, n)
+        assert plan["kernel"] == pa.binding.PA_KERNEL_TC_STREAM
+        assert plan["launches"] == 2  # the kernel and its cut-unit reduce
+        assert plan["grid"] % torch.cuda.get_device_properties(0).multi_processor_count == 0
