@@ -21,7 +21,8 @@
 //     lies wholly inside the range is finished in place: normalised bf16 output.  A unit
 //     cut by a range boundary leaves a partial (max, sum, unnormalised O) in one of the
 //     stream's two slots; the reduce kernel merges the pieces of each cut unit by
-//     log-sum-exp.  Each stream records which units its slots hold every launch.
+//     log-sum-exp.  The stream in which a cut unit starts records it, with its piece
+//     count, every launch.
 //   * pa_decode_append fuses the step's cache write: the stream that consumes a unit's
 //     last tile writes the new token's K/V to its slot and into the staged tile.
 
