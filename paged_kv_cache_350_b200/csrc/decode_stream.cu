@@ -446,11 +446,16 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_CTAS)
 // its piece count n: piece i is slot 0 of stream s + i, except the first, which is in
 // the slot stream s recorded.
 //
-// One thread per (query-head row, 4 output columns) of the unit: G * D/4 threads,
-// rounded up to whole warps.  Each thread merges the pieces online (running max, sum,
-// output; base 2) with the piece loop unrolled so that their loads overlap.
+// Threads: PS groups of BT = G * D/4 threads (rounded up to whole warps); in a group, one
+// thread per (query-head row, 4 output columns).  Group k merges pieces k, k + PS, ...
+// online (running max, sum, output; base 2), with the piece loop unrolled so that the
+// loads overlap; with PS > 1 the groups' results are then combined through shared
+// memory.  PS > 1 only when units are fewer than streams: then every unit spans several
+// streams (a long sequence's unit can have tens of pieces), while with many short units
+// a bigger block would only slow the launch of the many blocks that find no unit.
 template <int D>
-__global__ void __launch_bounds__(512) stream_reduce_kernel(const StreamParams sp) {
+__global__ void __launch_bounds__(1024) stream_reduce_kernel(const StreamParams sp, int BT,
+                                                             int PS) {
 #if PA_STREAM_PDL
   // Wait until the main kernel has completed and its writes are visible.
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -461,24 +466,53 @@ __global__ void __launch_bounds__(512) stream_reduce_kernel(const StreamParams s
   if (m.x < 0) return;
   const int u = m.x, slot0 = m.y, n = m.z;
   const int G = p.G;
-  const int r = threadIdx.x / (D / 4);
-  const int c = (threadIdx.x % (D / 4)) * 4;
-  if (r >= G) return;
+  const int grp = threadIdx.x / BT, idx = threadIdx.x - grp * BT;
+  const int r = idx / (D / 4);
+  const int c = (idx % (D / 4)) * 4;
+  const bool live = r < G;
   float M = -INFINITY, l = 0.f, a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  if (live) {
 #pragma unroll 4
-  for (int i = 0; i < n; ++i) {
-    const size_t row = (static_cast<size_t>(s + i) * 2 + (i == 0 ? slot0 : 0)) * G + r;
-    const float2 ml = *reinterpret_cast<const float2*>(sp.pml + row * 2);
-    const float4 a = *reinterpret_cast<const float4*>(sp.pacc + row * D + c);
-    const float Mn = fmaxf(M, ml.x);
-    const float so = exp2f(M - Mn), sn = exp2f(ml.x - Mn);
-    l = l * so + ml.y * sn;
-    a0 = a0 * so + a.x * sn;
-    a1 = a1 * so + a.y * sn;
-    a2 = a2 * so + a.z * sn;
-    a3 = a3 * so + a.w * sn;
-    M = Mn;
+    for (int i = grp; i < n; i += PS) {
+      const size_t row = (static_cast<size_t>(s + i) * 2 + (i == 0 ? slot0 : 0)) * G + r;
+      const float2 ml = *reinterpret_cast<const float2*>(sp.pml + row * 2);
+      const float4 a = *reinterpret_cast<const float4*>(sp.pacc + row * D + c);
+      const float Mn = fmaxf(M, ml.x);
+      const float so = exp2f(M - Mn), sn = exp2f(ml.x - Mn);
+      l = l * so + ml.y * sn;
+      a0 = a0 * so + a.x * sn;
+      a1 = a1 * so + a.y * sn;
+      a2 = a2 * so + a.z * sn;
+      a3 = a3 * so + a.w * sn;
+      M = Mn;
+    }
   }
+  if (PS > 1) {
+    extern __shared__ float red[];  // [PS][BT][6]
+    float* mine = red + (static_cast<size_t>(grp) * BT + idx) * 6;
+    mine[0] = M;
+    mine[1] = l;
+    mine[2] = a0;
+    mine[3] = a1;
+    mine[4] = a2;
+    mine[5] = a3;
+    __syncthreads();
+    if (grp != 0) return;
+    for (int k = 1; k < PS; ++k) {
+      const float* o = red + (static_cast<size_t>(k) * BT + idx) * 6;
+      const float Mn = fmaxf(M, o[0]);
+      // a group with no piece (n < PS) holds max -inf and adds nothing
+      const float so = M == -INFINITY ? 0.f : exp2f(M - Mn);
+      const float sn = o[0] == -INFINITY ? 0.f : exp2f(o[0] - Mn);
+      l = l * so + o[1] * sn;
+      a0 = a0 * so + o[2] * sn;
+      a1 = a1 * so + o[3] * sn;
+      a2 = a2 * so + o[4] * sn;
+      a3 = a3 * so + o[5] * sn;
+      M = Mn;
+    }
+  }
+  if (!live) return;
   const int b = u / p.Hkv, kvh = u - b * p.Hkv;
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) +
                        (static_cast<size_t>(b) * p.Hq + static_cast<size_t>(kvh) * G + r) * D + c;
@@ -487,11 +521,20 @@ __global__ void __launch_bounds__(512) stream_reduce_kernel(const StreamParams s
                                               pack_bf16x2(a2 * inv, a3 * inv));
 }
 
-// Threads of a reduce block: G * D/4, rounded up to whole warps (the piece count is
-// found with full-warp ballots).
+// Reduce block shape: BT = G * D/4 threads rounded up to whole warps, and PS piece groups
+// (4 when the units, B * Hkv, are fewer than the streams; at most 1024 threads).
+struct ReduceShape {
+  int BT, PS;
+};
+
 template <int D>
-int reduce_threads(int G) {
-  return ((G * D / 4 + 31) / 32) * 32;
+ReduceShape reduce_shape(const StreamParams& sp) {
+  ReduceShape r;
+  r.BT = ((sp.d.G * D / 4 + 31) / 32) * 32;
+  const long long units = static_cast<long long>(sp.d.B) * sp.d.Hkv;
+  r.PS = units < sp.streams ? (1024 / r.BT < 4 ? 1024 / r.BT : 4) : 1;
+  if (r.PS < 1) r.PS = 1;
+  return r;
 }
 
 template <class C>
@@ -522,20 +565,22 @@ cudaError_t launch_stream_cfg(const StreamParams& sp, int grid, cudaStream_t str
   decode_stream_kernel<C><<<grid, C::THREADS, smem, stream>>>(tmk, tmv, sp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  const ReduceShape rs = reduce_shape<C::D>(sp);
+  const size_t red_smem = rs.PS > 1 ? static_cast<size_t>(rs.PS) * rs.BT * 6 * sizeof(float) : 0;
 #if PA_STREAM_PDL
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(sp.streams));
-  cfg.blockDim = dim3(static_cast<unsigned>(reduce_threads<C::D>(sp.d.G)));
-  cfg.dynamicSmemBytes = 0;
+  cfg.blockDim = dim3(static_cast<unsigned>(rs.BT * rs.PS));
+  cfg.dynamicSmemBytes = red_smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, stream_reduce_kernel<C::D>, sp);
+  return cudaLaunchKernelEx(&cfg, stream_reduce_kernel<C::D>, sp, rs.BT, rs.PS);
 #else
-  stream_reduce_kernel<C::D><<<sp.streams, reduce_threads<C::D>(sp.d.G), 0, stream>>>(sp);
+  stream_reduce_kernel<C::D><<<sp.streams, rs.BT * rs.PS, red_smem, stream>>>(sp, rs.BT, rs.PS);
   return cudaGetLastError();
 #endif
 }
