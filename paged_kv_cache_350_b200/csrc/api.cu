@@ -134,7 +134,10 @@ static pa_status plan_decode(int B, int Hq, int Hkv, int D, int block_size, int 
   if (tc_ok && partition == 0 && B <= kStreamMaxB && tile_bound < (int64_t(1) << 31)) {
     int grid = pa::stream_grid(D, block_size, G, B);
     if (max_ctas > 0 && grid > max_ctas) grid = max_ctas;
-    if (grid > 0 && have_ws && workspace_bytes >= pa::stream_workspace_bytes(grid * pa::stream_warps_per_cta(block_size), G, D)) {
+    const size_t need = grid > 0 ? pa::stream_workspace_bytes(
+                                       grid * pa::stream_warps_per_cta(block_size), G, D)
+                                 : 0;
+    if (grid > 0 && have_ws && workspace_bytes >= need) {
       info->kernel = PA_KERNEL_TC_STREAM;
       info->grid = grid;
       info->max_parts = 1;

@@ -277,7 +277,8 @@ cudaError_t launch_decode_generic(const DecodeParams& p, pa_dtype dtype, cudaStr
     e = p.D == 64 ? launch_generic_t<__nv_bfloat16, 64>(p, stream)
                   : launch_generic_t<__nv_bfloat16, 128>(p, stream);
   else
-    e = p.D == 64 ? launch_generic_t<float, 64>(p, stream) : launch_generic_t<float, 128>(p, stream);
+    e = p.D == 64 ? launch_generic_t<float, 64>(p, stream)
+                  : launch_generic_t<float, 128>(p, stream);
   if (e != cudaSuccess || p.max_parts <= 1) return e;
   return launch_decode_reduce(p, dtype, stream);
 }

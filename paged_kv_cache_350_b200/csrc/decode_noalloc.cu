@@ -89,7 +89,9 @@ extern "C" pa_status pa_decode_no_alloc(void* out, const void* q, const void* k_
 
   const int grid = pa::stream_grid(D, block_size, G, B);
   if (grid <= 0) return PA_ERR_CUDA;
-  if (pa::stream_workspace_bytes(grid * pa::stream_warps_per_cta(block_size), G, D) > kScratchBytes) return PA_ERR_SCRATCH_LIMIT;
+  if (pa::stream_workspace_bytes(grid * pa::stream_warps_per_cta(block_size), G, D) >
+      kScratchBytes)
+    return PA_ERR_SCRATCH_LIMIT;
   void* scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) return PA_ERR_CUDA;
 

@@ -515,11 +515,12 @@ __global__ void __launch_bounds__(kThreads, kMinCtas)
       const int h1 = t.kvh * G + (is_group ? (g + 8) % G : g + 8);
 #pragma unroll
       for (int jn = 0; jn < C::NT; ++jn) {
+        const size_t col = 8 * jn + 2 * tig;
         if (g < nrows && b0 >= 0 && b0 < B)  // a member id outside [0, B) has no output row
-          *reinterpret_cast<uint32_t*>(out + (static_cast<size_t>(b0) * p.Hq + h0) * D + 8 * jn + 2 * tig) =
+          *reinterpret_cast<uint32_t*>(out + (static_cast<size_t>(b0) * p.Hq + h0) * D + col) =
               pack_bf16x2(acc.o_lo[jn][0] * inv_lo, acc.o_lo[jn][1] * inv_lo);
         if (g + 8 < nrows && b1 >= 0 && b1 < B)
-          *reinterpret_cast<uint32_t*>(out + (static_cast<size_t>(b1) * p.Hq + h1) * D + 8 * jn + 2 * tig) =
+          *reinterpret_cast<uint32_t*>(out + (static_cast<size_t>(b1) * p.Hq + h1) * D + col) =
               pack_bf16x2(acc.o_hi[jn][0] * inv_hi, acc.o_hi[jn][1] * inv_hi);
       }
     } else {
@@ -602,7 +603,8 @@ __global__ void __launch_bounds__(512) prefix_cut_reduce_kernel(const PrefixPara
   int b, h;
   row_target(pp, r, kvh, row, b, h);
   if (b < 0 || b >= p.B) return;
-  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + (static_cast<size_t>(b) * p.Hq + h) * D + c;
+  __nv_bfloat16* o =
+      static_cast<__nv_bfloat16*>(p.out) + (static_cast<size_t>(b) * p.Hq + h) * D + c;
   const float inv = 1.f / l;
   *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf16x2(a0 * inv, a1 * inv),
                                             pack_bf16x2(a2 * inv, a3 * inv));
