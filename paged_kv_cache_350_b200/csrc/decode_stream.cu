@@ -199,6 +199,20 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_CTAS)
   __shared__ __align__(8) uint64_t full_bar[NST];
   __shared__ int warp_sum[kThreads / 32];
 
+  // Set-up that reads no global data, then wait for the kernel before this one on the
+  // stream (launched as its programmatic dependent, this CTA may start while it drains;
+  // everything it wrote is visible after the wait, and this kernel reads or writes global
+  // memory only after it).
+  if (threadIdx.x == 0) {
+    prefetch_tensormap(&tmk);
+    prefetch_tensormap(&tmv);
+    for (int st = 0; st < NST; ++st) mbar_init(smem_addr(&full_bar[st]), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    fence_proxy_async_smem();
+  }
+#if PA_STREAM_PDL
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+#endif
   // ---- prefix sums of per-sequence tile counts (every CTA, identical) --------------
   {
     // tile counts first, read with independent coalesced loads, then scanned in place
@@ -240,13 +254,6 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_CTAS)
       uint32_t* row = reinterpret_cast<uint32_t*>(out + static_cast<size_t>(b) * p.Hq * D);
       for (int i = threadIdx.x; i < p.Hq * D / 2; i += kThreads) row[i] = 0u;
     }
-  }
-  if (threadIdx.x == 0) {
-    prefetch_tensormap(&tmk);
-    prefetch_tensormap(&tmv);
-    for (int st = 0; st < NST; ++st) mbar_init(smem_addr(&full_bar[st]), 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    fence_proxy_async_smem();
   }
   __syncthreads();
 
@@ -457,8 +464,10 @@ template <int D>
 __global__ void __launch_bounds__(1024) stream_reduce_kernel(const StreamParams sp, int BT,
                                                              int PS) {
 #if PA_STREAM_PDL
-  // Wait until the main kernel has completed and its writes are visible.
+  // Wait until the main kernel has completed and its writes are visible; the next kernel
+  // on the stream may launch now (it waits for this grid before reading).
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 #endif
   const DecodeParams& p = sp.d;
   const int s = blockIdx.x;
@@ -562,8 +571,26 @@ cudaError_t launch_stream_cfg(const StreamParams& sp, int grid, cudaStream_t str
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
+#if PA_STREAM_PDL
+  {
+    // a programmatic dependent of the previous kernel on the stream (see the kernel's
+    // griddepcontrol.wait)
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_stream_kernel<C>, tmk, tmv, sp);
+  }
+#else
   decode_stream_kernel<C><<<grid, C::THREADS, smem, stream>>>(tmk, tmv, sp);
   e = cudaGetLastError();
+#endif
   if (e != cudaSuccess) return e;
   const ReduceShape rs = reduce_shape<C::D>(sp);
   const size_t red_smem = rs.PS > 1 ? static_cast<size_t>(rs.PS) * rs.BT * 6 * sizeof(float) : 0;
