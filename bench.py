@@ -450,13 +450,15 @@ def run_ours(args):
     # PagedKVCache.pipeline: every step runs the C allocator, one host->device copy of the
     # step input (q, new K/V, tables, lengths, copy pairs), pa_copy_blocks +
     # pa_decode_append and a device->host copy of the output; steps are queued back to
-    # back with double-buffered staging, and each step's output is read one step later.
+    # back over three staging slots, and each step's output is read two steps later (so
+    # the host and the copies of neighbouring steps stay off the GPU's critical path).
     e2e = None
     if not args.no_e2e and args.e2e_steps > 0 and not args.shared_prefix:
         cache = pa.PagedKVCache(w.num_blocks, w.block_size, w.Hkv, w.D, dtype=kp.dtype, device=device,
                                 shuffle_seed=w.alloc_seed, pop_order=w.pop_order, k_pool=kp, v_pool=vp)
         workloads.run_setup(w, cache.alloc)
-        pipe = cache.pipeline(w.B, w.Hq, MB, stream=stream)
+        pipe = cache.pipeline(w.B, w.Hq, MB, depth=3, stream=stream)
+        lag = pipe.depth - 1
         q_c, nk_c, nv_c = q.cpu(), nk.cpu(), nv.cpu()
         ids = np.asarray(w.step_seqs, dtype=np.int64)
         warm = max(2, pipe.depth)
@@ -476,8 +478,8 @@ def run_ours(args):
                 pipe.submit(ids, w.scale)
             except pa.PAError:  # the pool ran out of blocks for more appends
                 break
-            if i >= 1:
-                pipe.result(i - 1)
+            if i >= lag:
+                pipe.result(i - lag)
             if i >= warm:
                 nbytes.append(decode_bytes(cur, w.B, w.Hq, w.Hkv, w.D, w.block_size, esize)[0])
                 done += 1
@@ -492,8 +494,8 @@ def run_ours(args):
                    "ms_per_step": 1e3 * dt / done, "steps": done,
                    "timing": "host perf_counter over the steps of PagedKVCache.pipeline: per step the C "
                              "allocator, one host->device copy of the step input, kernels, a "
-                             "device->host copy of the output (read one step later); steps queued "
-                             "back to back, double-buffered staging"}
+                             "device->host copy of the output (read two steps later); steps queued "
+                             "back to back over three staging slots"}
 
     # ---- CPU oracle baseline (rank 0, one GPU only) --------------------------------
     cpu = None

@@ -31,6 +31,8 @@ __global__ void reshape_and_cache_kernel(const uint4* __restrict__ key,
                                          uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
                                          const int64_t* __restrict__ slot_mapping,
                                          int vec_per_row, int64_t num_slots, int32_t* err) {
+  // a decode launched as this kernel's programmatic dependent may start its set-up now
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int t = blockIdx.y;
   const int64_t s = __ldg(slot_mapping + t);
   if (s < 0) return;
@@ -56,6 +58,7 @@ __global__ void append_kv_kernel(const uint4* __restrict__ k_new, const uint4* _
                                  const int32_t* __restrict__ block_tables,
                                  const int32_t* __restrict__ seq_lens, int max_blocks,
                                  int block_size, int num_blocks, int vec_per_row, int32_t* err) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int b = blockIdx.x;
   const int L = __ldg(seq_lens + b);
   if (L == 0) return;
@@ -80,6 +83,7 @@ __global__ void append_kv_kernel(const uint4* __restrict__ k_new, const uint4* _
 __global__ void copy_blocks_kernel(uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
                                    const int32_t* __restrict__ pairs, int64_t vec_per_block,
                                    int num_blocks, int32_t* err) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int i = blockIdx.y;
   const int src = __ldg(pairs + 2 * i);
   const int dst = __ldg(pairs + 2 * i + 1);

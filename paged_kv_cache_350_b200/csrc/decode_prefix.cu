@@ -277,6 +277,9 @@ __global__ void __launch_bounds__(kThreads, kMinCtas)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     fence_proxy_async_smem();
   }
+  // Launched as a programmatic dependent of the previous kernel on the stream: nothing
+  // above reads global memory; wait for that kernel before anything below does.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // ---- tile counts of every unit row, scanned (every CTA, identical): P[r] = tiles of
   // the rows before r, P[R] = total.  Rows first, with their dependent loads (group ->
   // members -> lengths) overlapping across threads, then an in-place scan.
@@ -573,6 +576,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtas)
 template <int D>
 __global__ void __launch_bounds__(512) prefix_cut_reduce_kernel(const PrefixParams pp) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const DecodeParams& p = pp.d;
   const int s = blockIdx.x;
   // the unit stream s owns, recorded with the slot of its first piece and the piece count
@@ -635,9 +639,8 @@ cudaError_t launch_pref_cfg(PrefixParams pp, int grid, cudaStream_t stream) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  decode_prefix_kernel<C><<<grid, kThreads, smem, stream>>>(tmk, tmv, pp);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // the cut reduce, as a programmatic dependent of the main kernel
+  // the main kernel as a programmatic dependent of the previous kernel on the stream,
+  // the cut reduce as one of the main kernel
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -645,6 +648,10 @@ cudaError_t launch_pref_cfg(PrefixParams pp, int grid, cudaStream_t stream) {
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  if ((e = cudaLaunchKernelEx(&cfg, decode_prefix_kernel<C>, tmk, tmv, pp)) != cudaSuccess) return e;
   cfg.gridDim = dim3(static_cast<unsigned>(pp.streams));
   cfg.blockDim = dim3(kRows * C::D / 4);
   cfg.dynamicSmemBytes = 0;
