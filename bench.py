@@ -73,6 +73,8 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=60)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-all-cores", type=int, default=1,
+                    help="also time the oracle in one spawned process per host core (0: off)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--shared-prefix", action="store_true",
                     help="decode with pa_decode_shared_prefix (fork groups read shared blocks once)")
@@ -270,6 +272,69 @@ def oracle_sample_rate(w, tables, lens, seconds, row_order=None, max_tokens=None
     desc = (f"oracle.ref_decode (float64 NumPy, 1 BLAS thread) on {done_rows} sequence(s) "
             f"({tokens} tokens x {w.Hkv} KV heads) of the {w.name} batch")
     return done_bytes / dt / 1e9, desc, dt
+
+
+def _oracle_worker(task):
+    """One spawned worker of oracle_rate_all_cores: ref_decode on its rows until the time
+    budget passes, reading the pools from shared memory.  Returns (bytes, seconds)."""
+    from multiprocessing import shared_memory
+    from oracle import ref_decode
+    try:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(limits=1)
+    except Exception:
+        pass
+    name, shape, dtype, q, tables, lens, rows, scale, seconds, Hq, Hkv, D, bs, esize = task
+    shm = shared_memory.SharedMemory(name=name)
+    try:
+        n = int(np.prod(shape))
+        kp = np.ndarray(shape, dtype=dtype, buffer=shm.buf)
+        vp = np.ndarray(shape, dtype=dtype, buffer=shm.buf, offset=n * np.dtype(dtype).itemsize)
+        done = 0
+        t0 = time.perf_counter()
+        for r in rows:
+            ref_decode(q[r:r + 1], kp, vp, tables[r:r + 1], lens[r:r + 1], scale)
+            done += decode_bytes([int(lens[r])], 1, Hq, Hkv, D, bs, esize)[0]
+            if time.perf_counter() - t0 >= seconds:
+                break
+        dt = time.perf_counter() - t0
+        del kp, vp
+    finally:
+        shm.close()
+    return done, dt
+
+
+def oracle_rate_all_cores(w, tables, lens, seconds, workers=None):
+    """The same oracle on every host core: one spawned process per core, each on its own
+    rows of the batch (round robin), the pools shared read-only through shared memory.
+    Returns (GB/s = all bytes / the slowest worker's time, processes, description)."""
+    import multiprocessing as mp
+    from multiprocessing import shared_memory
+    workers = workers or len(os.sched_getaffinity(0))
+    kp, vp = w.k_pool(), w.v_pool()
+    shm = shared_memory.SharedMemory(create=True, size=kp.nbytes + vp.nbytes)
+    try:
+        np.ndarray(kp.shape, dtype=kp.dtype, buffer=shm.buf)[...] = kp
+        np.ndarray(vp.shape, dtype=vp.dtype, buffer=shm.buf, offset=kp.nbytes)[...] = vp
+        esize = 2 if w.dtype == "bf16" else 4
+        q = w.q()
+        tasks = [(shm.name, kp.shape, kp.dtype, q, tables, lens, list(range(i, w.B, workers)),
+                  w.scale, seconds, w.Hq, w.Hkv, w.D, w.block_size, esize)
+                 for i in range(min(workers, w.B))]
+        del kp, vp
+        # a worker that dies raises here instead of being respawned for ever
+        from concurrent.futures import ProcessPoolExecutor
+        with ProcessPoolExecutor(len(tasks), mp_context=mp.get_context("spawn")) as ex:
+            res = list(ex.map(_oracle_worker, tasks, timeout=10 * seconds + 120))
+    finally:
+        shm.close()
+        shm.unlink()
+    total = sum(r[0] for r in res)
+    slowest = max(r[1] for r in res)
+    desc = (f"oracle.ref_decode (float64 NumPy) in {len(tasks)} spawned processes, one per "
+            f"core, each on every {len(tasks)}-th sequence of the {w.name} batch for about "
+            f"{seconds:.0f} s; the pools shared read-only")
+    return total / slowest / 1e9, len(tasks), desc
 
 
 def run_reference(args):
@@ -502,6 +567,16 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, desc, _ = oracle_sample_rate(w, tables, lens, args.cpu_seconds)
         cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
+        if args.cpu_all_cores:
+            try:
+                need = 2 * w.k_pool().nbytes
+                st = os.statvfs("/dev/shm")
+                if st.f_bavail * st.f_frsize < 1.2 * need:
+                    raise RuntimeError(f"/dev/shm has less than {1.2 * need / 1e9:.1f} GB free")
+                rate_n, procs, desc_n = oracle_rate_all_cores(w, tables, lens, args.cpu_seconds / 2)
+                cpu["all_cores"] = {"value": rate_n, "unit": UNIT, "cores": procs, "sample": desc_n}
+            except Exception as exc:  # the single-thread figure stands on its own
+                cpu["all_cores"] = {"skipped": f"{type(exc).__name__}: {exc}"}
 
     if dist is not None:
         barrier(dist, device)

@@ -51,3 +51,17 @@ def test_whole_job_value_counts_every_rank():
     alg, kv = bench.decode_bytes([10, 20], 2, 8, 2, 128, 16, 2)
     assert kv == 2 * 30 * 2 * 128 * 2
     assert alg == kv + 2 * 2 * 8 * 128 * 2 + (1 + 2) * 4 + 4 * 2
+
+
+def test_oracle_all_cores_rate_runs_in_spawned_workers():
+    """The all-cores oracle timing of bench.py (spawned processes, pools in shared memory)
+    on the tiny batch: every worker reports, and the rate is positive."""
+    import bench
+    import workloads
+    from oracle import RefAllocator
+    w = workloads.tiny()
+    alloc = RefAllocator(w.num_blocks, w.block_size, shuffle_seed=w.alloc_seed)
+    workloads.run_setup(w, alloc)
+    _, _, tables, lens = workloads.run_step_allocation(w, alloc)
+    rate, procs, desc = bench.oracle_rate_all_cores(w, tables, lens, 0.2, workers=2)
+    assert procs == 2 and rate > 0 and "spawned" in desc
