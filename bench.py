@@ -284,12 +284,13 @@ def _oracle_worker(task):
         threadpool_limits(limits=1)
     except Exception:
         pass
-    name, shape, dtype, q, tables, lens, rows, scale, seconds, Hq, Hkv, D, bs, esize = task
+    name, shape, dtype, qshape, tables, lens, rows, scale, seconds, Hq, Hkv, D, bs, esize = task
     shm = shared_memory.SharedMemory(name=name)
     try:
-        n = int(np.prod(shape))
+        nb = int(np.prod(shape)) * np.dtype(dtype).itemsize
         kp = np.ndarray(shape, dtype=dtype, buffer=shm.buf)
-        vp = np.ndarray(shape, dtype=dtype, buffer=shm.buf, offset=n * np.dtype(dtype).itemsize)
+        vp = np.ndarray(shape, dtype=dtype, buffer=shm.buf, offset=nb)
+        q = np.ndarray(qshape, dtype=dtype, buffer=shm.buf, offset=2 * nb)
         done = 0
         t0 = time.perf_counter()
         for r in rows:
@@ -298,7 +299,7 @@ def _oracle_worker(task):
             if time.perf_counter() - t0 >= seconds:
                 break
         dt = time.perf_counter() - t0
-        del kp, vp
+        del kp, vp, q
     finally:
         shm.close()
     return done, dt
@@ -311,17 +312,18 @@ def oracle_rate_all_cores(w, tables, lens, seconds, workers=None):
     import multiprocessing as mp
     from multiprocessing import shared_memory
     workers = workers or len(os.sched_getaffinity(0))
-    kp, vp = w.k_pool(), w.v_pool()
-    shm = shared_memory.SharedMemory(create=True, size=kp.nbytes + vp.nbytes)
+    kp, vp, q = w.k_pool(), w.v_pool(), w.q()
+    shm = shared_memory.SharedMemory(create=True, size=kp.nbytes + vp.nbytes + q.nbytes)
     try:
         np.ndarray(kp.shape, dtype=kp.dtype, buffer=shm.buf)[...] = kp
         np.ndarray(vp.shape, dtype=vp.dtype, buffer=shm.buf, offset=kp.nbytes)[...] = vp
+        np.ndarray(q.shape, dtype=q.dtype, buffer=shm.buf, offset=2 * kp.nbytes)[...] = q
         esize = 2 if w.dtype == "bf16" else 4
-        q = w.q()
-        tasks = [(shm.name, kp.shape, kp.dtype, q, tables, lens, list(range(i, w.B, workers)),
-                  w.scale, seconds, w.Hq, w.Hkv, w.D, w.block_size, esize)
+        tasks = [(shm.name, kp.shape, kp.dtype, q.shape, tables, lens,
+                  list(range(i, w.B, workers)), w.scale, seconds, w.Hq, w.Hkv, w.D,
+                  w.block_size, esize)
                  for i in range(min(workers, w.B))]
-        del kp, vp
+        del kp, vp, q
         # a worker that dies raises here instead of being respawned for ever
         from concurrent.futures import ProcessPoolExecutor
         with ProcessPoolExecutor(len(tasks), mp_context=mp.get_context("spawn")) as ex:
@@ -569,7 +571,7 @@ def run_ours(args):
         cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
         if args.cpu_all_cores:
             try:
-                need = 2 * w.k_pool().nbytes
+                need = 2 * w.k_pool().nbytes + w.q().nbytes
                 st = os.statvfs("/dev/shm")
                 if st.f_bavail * st.f_frsize < 1.2 * need:
                     raise RuntimeError(f"/dev/shm has less than {1.2 * need / 1e9:.1f} GB free")
