@@ -215,3 +215,17 @@ def test_plan_on_b200_takes_the_stream_kernel_for_every_block_size():
         assert plan["kernel"] == pa.binding.PA_KERNEL_TC_STREAM
         assert plan["launches"] == 2  # the kernel and its cut-unit reduce
         assert plan["grid"] % torch.cuda.get_device_properties(0).multi_processor_count == 0
+
+
+def test_batch_beyond_the_stream_kernel_limit():
+    """B > 8192 (the balanced kernel's prefix sums live in shared memory): the plan falls
+    back to the partition kernel, and the fused call to the append kernel + that decode."""
+    import paged_kv_cache_350_b200 as pa
+    rng = np.random.default_rng(4400)
+    lens = rng.integers(1, 41, size=8200)
+    w = workloads.independent(lens, Hq=8, Hkv=2, bs=16, seed=4401)
+    n = pa.pa_decode_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.max_blocks * w.block_size,
+                                    w.block_size, 0)
+    plan = pa.pa_decode_plan(w.B, w.Hq, w.Hkv, w.D, w.block_size, w.max_blocks, pa.PA_BF16, n)
+    assert plan["kernel"] == pa.binding.PA_KERNEL_TC_PARTITION
+    check_fused(w)
