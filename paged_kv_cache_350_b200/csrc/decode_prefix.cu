@@ -384,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtas)
   const float sl2 = p.scale_log2;
   // The cut unit this stream owns (it starts in this stream's range and continues past
   // it): unit id, slot of this stream's piece, number of pieces.
-  int own_u = -1, own_slot = 0, own_n = 0;
+  int own_u = -1, own_slot = 0, own_n = 0, own_rows = 0;
   int i = 0;
   bool ok = true;
   WarpAcc<C, true> acc;
@@ -533,6 +533,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtas)
         own_u = u;
         own_slot = slot;
         own_n = (uend - 1) / per - s + 1;
+        own_rows = nrows;
       }
       if (tig == 0) {
         if (g < nrows)
@@ -565,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtas)
     }
   }
   if (lane == 0) {
-    int4 m = make_int4(ok ? own_u : -1, own_slot, own_n, 0);
+    int4 m = make_int4(ok ? own_u : -1, own_slot, own_n, own_rows);
     *reinterpret_cast<int4*>(pp.meta + s * 4) = m;
   }
 }
@@ -579,24 +580,28 @@ __global__ void __launch_bounds__(512) prefix_cut_reduce_kernel(const PrefixPara
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const DecodeParams& p = pp.d;
   const int s = blockIdx.x;
-  // the unit stream s owns, recorded with the slot of its first piece and the piece count
+  // the unit stream s owns, recorded with the slot of its first piece, the piece count and
+  // the unit's rows (no dependent loads of group members here)
   const int4 m = *reinterpret_cast<const int4*>(pp.meta + static_cast<size_t>(s) * 4);
   if (m.x < 0) return;
-  const int u = m.x, slot = m.y, n = m.z;
+  const int u = m.x, slot = m.y, n = m.z, nrows = m.w;
   const int r = u / p.Hkv, kvh = u - r * p.Hkv;
-  const int nrows = r < pp.ngroups ? group_size(pp, r) * p.G : p.G;
   const int row = threadIdx.x / (D / 4);
   const int c = (threadIdx.x % (D / 4)) * 4;
   if (row >= nrows) return;
+  int b, h;
+  row_target(pp, r, kvh, row, b, h);  // its load overlaps the pieces' loads
   float M = -INFINITY, l = 0.f, a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll 4
   for (int i = 0; i < n; ++i) {
     const size_t pr = (static_cast<size_t>(s + i) * 2 + (i == 0 ? slot : 0)) * kRows + row;
     const float2 ml = *reinterpret_cast<const float2*>(pp.pml + pr * 2);
     const float4 a = *reinterpret_cast<const float4*>(pp.pacc + pr * D + c);
-    if (ml.x == -INFINITY) continue;
+    // no branch (a piece with no tile of this row has max -inf and weight 0), so that the
+    // unrolled pieces' loads are all issued up front
     const float Mn = fmaxf(M, ml.x);
-    const float so = exp2f(M - Mn), sn = exp2f(ml.x - Mn);
+    const float so = M == -INFINITY ? 0.f : exp2f(M - Mn);
+    const float sn = ml.x == -INFINITY ? 0.f : exp2f(ml.x - Mn);
     l = l * so + ml.y * sn;
     a0 = a0 * so + a.x * sn;
     a1 = a1 * so + a.y * sn;
@@ -604,8 +609,6 @@ __global__ void __launch_bounds__(512) prefix_cut_reduce_kernel(const PrefixPara
     a3 = a3 * so + a.w * sn;
     M = Mn;
   }
-  int b, h;
-  row_target(pp, r, kvh, row, b, h);
   if (b < 0 || b >= p.B) return;
   __nv_bfloat16* o =
       static_cast<__nv_bfloat16*>(p.out) + (static_cast<size_t>(b) * p.Hq + h) * D + c;
