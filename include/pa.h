@@ -252,6 +252,15 @@ pa_status pa_decode_no_alloc(void* out, const void* q, const void* k_pool, const
                              float scale, pa_dtype dtype, int32_t* dev_err_flag,
                              pa_stream_t stream);
 
+/* Self-test of the kernels' bounded waits (the pages have no counterpart; it exists for
+ * the failure-detection test).  One warp waits, through the same bounded wait the decode
+ * kernels use, on a barrier phase that nothing completes, limited to limit_us
+ * (1 .. 1000000) microseconds.  The wait runs out, ORs PA_DEVERR_TIMEOUT into
+ * *dev_err_flag (device memory, required) and the kernel returns: the context stays
+ * usable.  PA_ERR_INVALID_ARG for a NULL flag or a limit out of range. */
+pa_status pa_selftest_bounded_wait(int32_t* dev_err_flag, unsigned limit_us,
+                                   pa_stream_t stream);
+
 /* ---------------------------------------------------------------------------
  * Cache maintenance
  * ------------------------------------------------------------------------- */

@@ -102,6 +102,7 @@ def _load():
         "pa_alloc_prefix_groups": (i32, [vp, pi64, i32, i32, i32, pi32, pi32, pi32, pint]),
         "pa_decode_no_alloc": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                      f32, i32, vp, vp]),
+        "pa_selftest_bounded_wait": (i32, [vp, ctypes.c_uint, vp]),
         "pa_reshape_and_cache": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]),
         "pa_copy_blocks": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]),
         "pa_alloc_create": (i32, [i32, i32, ctypes.c_uint64, ctypes.POINTER(vp)]),
@@ -137,7 +138,7 @@ EXPORTED = (
     "pa_status_string", "pa_status_from_device_flag", "pa_version", "pa_decode_workspace_size",
     "pa_decode", "pa_decode_ex", "pa_decode_append", "pa_decode_plan", "pa_decode_no_alloc",
     "pa_decode_shared_prefix_workspace_size", "pa_decode_shared_prefix", "pa_alloc_prefix_groups",
-    "pa_reshape_and_cache", "pa_copy_blocks", "pa_alloc_create",
+    "pa_reshape_and_cache", "pa_copy_blocks", "pa_selftest_bounded_wait", "pa_alloc_create",
     "pa_alloc_create_ordered", "pa_alloc_destroy", "pa_alloc_add_seq", "pa_alloc_fork",
     "pa_alloc_append_slot", "pa_alloc_append_slots", "pa_alloc_free_seq", "pa_alloc_truncate",
     "pa_alloc_beam_select", "pa_alloc_block_table",
@@ -375,6 +376,12 @@ def pa_copy_blocks(k_pool, v_pool, pairs, err_flag=None, stream=None):
     st = lib.pa_copy_blocks(_ptr(k_pool), _ptr(v_pool), _ptr(pairs), n, bs, Hkv, D, NB,
                             _dtype_of(k_pool), _ptr(err_flag), _stream(stream))
     _check(st, "pa_copy_blocks")
+
+
+def pa_selftest_bounded_wait(err_flag, limit_us, stream=None):
+    """Run the bounded-wait self-test (see include/pa.h): err_flag gets PA_DEVERR_TIMEOUT."""
+    _check(lib.pa_selftest_bounded_wait(_ptr(err_flag), int(limit_us), _stream(stream)),
+           "pa_selftest_bounded_wait")
 
 
 def pa_status_from_device_flag(flag):

@@ -259,3 +259,19 @@ def test_bad_block_id_and_bad_length_set_the_flag():
                                   torch.tensor([17, -1], dtype=torch.int32, device="cuda"), 0.1,
                                   path=path, partition=part)
         assert err & pa.binding.PA_DEVERR_BAD_SEQ_LEN
+
+
+def test_bounded_wait_runs_out_sets_the_flag_and_the_context_survives():
+    """Failure detection on the GPU without a fault: a wait on a barrier phase nothing
+    completes (the decode kernels' bounded wait, limited to 20 ms) ends with
+    PA_DEVERR_TIMEOUT; afterwards the same context runs a decode correctly."""
+    import time
+    import paged_kv_cache_350_b200 as pa
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t0 = time.perf_counter()
+    pa.binding.pa_selftest_bounded_wait(err, 20000)
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 < 5.0
+    assert int(err.item()) == pa.binding.PA_DEVERR_TIMEOUT
+    assert pa.pa_status_from_device_flag(int(err.item())) == pa.binding.PA_ERR_TIMEOUT
+    check(SCALED["gqa"](), path=TENSOR)

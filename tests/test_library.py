@@ -113,6 +113,14 @@ def test_decode_append_argument_errors_are_reported_before_any_launch():
     assert _call_append(Hq=6, Hkv=4) == b.PA_ERR_INVALID_ARG
 
 
+def test_selftest_rejects_bad_arguments_before_any_launch():
+    from paged_kv_cache_350_b200 import binding as b
+    vp = ctypes.c_void_p
+    assert b.lib.pa_selftest_bounded_wait(vp(0), 1000, vp(0)) == b.PA_ERR_INVALID_ARG
+    assert b.lib.pa_selftest_bounded_wait(vp(16), 0, vp(0)) == b.PA_ERR_INVALID_ARG
+    assert b.lib.pa_selftest_bounded_wait(vp(16), 2000000, vp(0)) == b.PA_ERR_INVALID_ARG
+
+
 def test_cache_op_argument_errors():
     from paged_kv_cache_350_b200 import binding as b
     vp = ctypes.c_void_p
