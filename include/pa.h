@@ -206,7 +206,8 @@ pa_status pa_decode_append(void* out, const void* q, const void* k_new, const vo
  *   group_of      [B] device int32: group of batch row b, or -1
  *   group_prefix  [ngroups] device int32: shared tokens of the group, a multiple of
  *                 PA_SHARED_PREFIX_ALIGN and <= every member's length; members' tables must
- *                 hold the same block ids for those tokens
+ *                 hold the same block ids for those tokens.  0 is allowed (the group then
+ *                 shares no tokens; its members' own tokens are still read as one unit)
  *   group_members [ngroups][max_members] device int32: the group's batch rows, -1 padded
  * pa_alloc_prefix_groups builds these from the allocator.  bf16 tensor-core shapes only
  * (PA_ERR_UNSUPPORTED otherwise); max_members * (Hq/Hkv) <= 16; B + ngroups <= 8192.
@@ -263,6 +264,11 @@ pa_status pa_selftest_bounded_wait(int32_t* dev_err_flag, unsigned limit_us,
 
 /* ---------------------------------------------------------------------------
  * Cache maintenance
+ *
+ * Both kernels are queued as programmatic dependents of the kernel before them on the
+ * stream: their blocks may be scheduled while that kernel drains, and wait for its
+ * completion before any memory access.  Stream order is unchanged; a step of copy,
+ * cache write and decode just pays no launch gap between its kernels.
  * ------------------------------------------------------------------------- */
 
 /* For t < T with s = slot_mapping[t] >= 0: k_pool[s / block_size][s % block_size][:][:]

@@ -31,8 +31,10 @@ __global__ void reshape_and_cache_kernel(const uint4* __restrict__ key,
                                          uint4* __restrict__ k_pool, uint4* __restrict__ v_pool,
                                          const int64_t* __restrict__ slot_mapping,
                                          int vec_per_row, int64_t num_slots, int32_t* err) {
-  // a decode launched as this kernel's programmatic dependent may start its set-up now
+  // a decode launched as this kernel's programmatic dependent may start its set-up now;
+  // this kernel, launched as one of the previous kernel, waits for it before any access
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int t = blockIdx.y;
   const int64_t s = __ldg(slot_mapping + t);
   if (s < 0) return;
@@ -59,6 +61,7 @@ __global__ void append_kv_kernel(const uint4* __restrict__ k_new, const uint4* _
                                  const int32_t* __restrict__ seq_lens, int max_blocks,
                                  int block_size, int num_blocks, int vec_per_row, int32_t* err) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int b = blockIdx.x;
   const int L = __ldg(seq_lens + b);
   if (L == 0) return;
@@ -84,6 +87,7 @@ __global__ void copy_blocks_kernel(uint4* __restrict__ k_pool, uint4* __restrict
                                    const int32_t* __restrict__ pairs, int64_t vec_per_block,
                                    int num_blocks, int32_t* err) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int i = blockIdx.y;
   const int src = __ldg(pairs + 2 * i);
   const int dst = __ldg(pairs + 2 * i + 1);
@@ -98,6 +102,25 @@ __global__ void copy_blocks_kernel(uint4* __restrict__ k_pool, uint4* __restrict
     k_pool[d_o + v] = k_pool[so + v];
     v_pool[d_o + v] = v_pool[so + v];
   }
+}
+
+// Launch as a programmatic dependent of the previous kernel on the stream: the grid may
+// be scheduled while that kernel drains, and waits for it (griddepcontrol.wait) before
+// touching memory, so a step of cache kernels and a decode pays no launch gap between
+// them.  Without a previous kernel this is an ordinary launch.
+template <class... KArgs, class... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, int threads,
+                             cudaStream_t stream, Args... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
 }  // namespace
@@ -115,21 +138,20 @@ cudaError_t launch_reshape_and_cache(const void* key, const void* value, void* k
     // one launch per 65535 tokens (grid.y limit)
     for (int t0 = 0; t0 < T; t0 += 65535) {
       const int n = T - t0 < 65535 ? T - t0 : 65535;
-      reshape_and_cache_kernel<<<dim3(gx, n), threads, 0, stream>>>(
+      cudaError_t e = launch_dependent(
+          reshape_and_cache_kernel, dim3(gx, n), threads, stream,
           static_cast<const uint4*>(key) + static_cast<int64_t>(t0) * vec,
           static_cast<const uint4*>(value) + static_cast<int64_t>(t0) * vec,
           static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), slot_mapping + t0, vec,
           num_slots, err);
-      cudaError_t e = cudaGetLastError();
       if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
   }
-  reshape_and_cache_kernel<<<dim3(gx, T), threads, 0, stream>>>(
-      static_cast<const uint4*>(key), static_cast<const uint4*>(value),
-      static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), slot_mapping, vec, num_slots,
-      err);
-  return cudaGetLastError();
+  return launch_dependent(reshape_and_cache_kernel, dim3(gx, T), threads, stream,
+                          static_cast<const uint4*>(key), static_cast<const uint4*>(value),
+                          static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), slot_mapping,
+                          vec, num_slots, err);
 }
 
 cudaError_t launch_append_kv(const void* k_new, const void* v_new, void* k_pool, void* v_pool,
@@ -139,11 +161,10 @@ cudaError_t launch_append_kv(const void* k_new, const void* v_new, void* k_pool,
   if (B <= 0) return cudaSuccess;
   const int vec = row_bytes / 16;
   const int threads = vec < 256 ? ((vec + 31) / 32) * 32 : 256;
-  append_kv_kernel<<<B, threads, 0, stream>>>(
-      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
-      static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), block_tables, seq_lens,
-      max_blocks, block_size, num_blocks, vec, err);
-  return cudaGetLastError();
+  return launch_dependent(append_kv_kernel, dim3(static_cast<unsigned>(B)), threads, stream,
+                          static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
+                          static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), block_tables,
+                          seq_lens, max_blocks, block_size, num_blocks, vec, err);
 }
 
 cudaError_t launch_copy_blocks(void* k_pool, void* v_pool, const int32_t* pairs, int n,
@@ -156,10 +177,10 @@ cudaError_t launch_copy_blocks(void* k_pool, void* v_pool, const int32_t* pairs,
   if (gx > 64) gx = 64;
   for (int i0 = 0; i0 < n; i0 += 65535) {
     const int m = n - i0 < 65535 ? n - i0 : 65535;
-    copy_blocks_kernel<<<dim3(static_cast<unsigned>(gx), m), threads, 0, stream>>>(
-        static_cast<uint4*>(k_pool), static_cast<uint4*>(v_pool), pairs + 2 * i0, vec,
-        num_blocks, err);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_dependent(copy_blocks_kernel, dim3(static_cast<unsigned>(gx), m),
+                                     threads, stream, static_cast<uint4*>(k_pool),
+                                     static_cast<uint4*>(v_pool), pairs + 2 * i0, vec, num_blocks,
+                                     err);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -95,13 +95,14 @@ __device__ __forceinline__ int group_size(const PrefixParams& pp, int r) {
   return n;
 }
 
-// Shared tokens of group r (0 for a malformed group, flagged).
+// Shared tokens of group r; -1 for a malformed group (flagged), whose rows then get no
+// tile.  A prefix of 0 is valid: the unit streams only the members' own tokens.
 __device__ __forceinline__ int group_prefix_tokens(const PrefixParams& pp, int r, bool flag) {
   const int b0 = member_of(pp, r, 0);
   const int pre = __ldg(pp.group_prefix + r);
   if (b0 < 0 || b0 >= pp.d.B || pre < 0 || pre % PA_SHARED_PREFIX_ALIGN != 0) {
     if (flag) flag_error(pp.d.err, PA_DEVERR_BAD_SEQ_LEN);
-    return 0;
+    return -1;
   }
   return pre;
 }
@@ -125,7 +126,7 @@ template <int TT>
 __device__ __forceinline__ int row_tiles(const PrefixParams& pp, int r, bool flag) {
   if (r < pp.ngroups) {
     const int pre = group_prefix_tokens(pp, r, flag);
-    if (pre == 0) return 0;
+    if (pre < 0) return 0;
     // member ids first (independent loads), then their lengths (independent loads)
     int ids[kRows];
 #pragma unroll
@@ -170,7 +171,7 @@ __device__ __forceinline__ TileSrc tile_src(const PrefixParams& pp, int r, int j
     t.row_hi = 16;
     return t;
   }
-  const int pre = group_prefix_tokens(pp, r, false);
+  const int pre = max(group_prefix_tokens(pp, r, false), 0);
   const int np = pre / TT;
   if (j < np) {
     t.table_b = member_of(pp, r, 0);
@@ -396,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtas)
   auto load_ids = [&](const TilePos& u, int& id, int& pre) {
     if (u.r < NG) {
       id = lane < pp.max_members ? member_of(pp, u.r, lane) : -1;
-      pre = group_prefix_tokens(pp, u.r, false);
+      pre = max(group_prefix_tokens(pp, u.r, false), 0);
     } else {
       id = u.r - NG;
       pre = 0;
@@ -465,6 +466,10 @@ __global__ void __launch_bounds__(kThreads, kMinCtas)
     const int nrows = is_group ? gs * G : G;
     // batch row of MMA row rr (member rr / G of a group, or the sequence)
     auto row_b = [&](int rr) { return __shfl_sync(kFull, mb, is_group ? rr / G : 0); };
+    // whether MMA row rr has an output here: a row of length 0 (a member of a group with
+    // no shared tokens, or one flagged for being shorter than the prefix) is left to the
+    // zero fill of the prologue, which writes every such row and nothing else
+    auto row_live = [&](int rr) { return __shfl_sync(kFull, mL, is_group ? rr / G : 0) > 0; };
     // the next unit of this stream (if any) starts at tile pend
     const bool has_next = pend < end;
     TilePos tn{};
@@ -513,7 +518,10 @@ __global__ void __launch_bounds__(kThreads, kMinCtas)
     const bool complete = (gpos == ubeg) && (pend == uend);
     if (complete) {
       const float inv_lo = 1.f / acc.l_lo, inv_hi = 1.f / acc.l_hi;
-      const int b0 = row_b(g), b1 = row_b(g + 8);
+      // shuffles first, by every lane; then the per-lane choice
+      const int rb0 = row_b(g), rb1 = row_b(g + 8);
+      const bool live0 = row_live(g), live1 = row_live(g + 8);
+      const int b0 = live0 ? rb0 : -1, b1 = live1 ? rb1 : -1;
       const int h0 = t.kvh * G + (is_group ? g % G : g);
       const int h1 = t.kvh * G + (is_group ? (g + 8) % G : g + 8);
 #pragma unroll
@@ -535,11 +543,15 @@ __global__ void __launch_bounds__(kThreads, kMinCtas)
         own_n = (uend - 1) / per - s + 1;
         own_rows = nrows;
       }
+      // a row without output gets sum 0 in every piece, so the reduce skips it
+      const bool live0 = row_live(g), live1 = row_live(g + 8);
       if (tig == 0) {
         if (g < nrows)
-          *reinterpret_cast<float2*>(pp.pml + (row0 + g) * 2) = make_float2(acc.m_lo, acc.l_lo);
+          *reinterpret_cast<float2*>(pp.pml + (row0 + g) * 2) =
+              make_float2(acc.m_lo, live0 ? acc.l_lo : 0.f);
         if (g + 8 < nrows)
-          *reinterpret_cast<float2*>(pp.pml + (row0 + g + 8) * 2) = make_float2(acc.m_hi, acc.l_hi);
+          *reinterpret_cast<float2*>(pp.pml + (row0 + g + 8) * 2) =
+              make_float2(acc.m_hi, live1 ? acc.l_hi : 0.f);
       }
 #pragma unroll
       for (int jn = 0; jn < C::NT; ++jn) {
@@ -609,7 +621,7 @@ __global__ void __launch_bounds__(512) prefix_cut_reduce_kernel(const PrefixPara
     a3 = a3 * so + a.w * sn;
     M = Mn;
   }
-  if (b < 0 || b >= p.B) return;
+  if (b < 0 || b >= p.B || !(l > 0.f)) return;  // no output row, or one left to the zero fill
   __nv_bfloat16* o =
       static_cast<__nv_bfloat16*>(p.out) + (static_cast<size_t>(b) * p.Hq + h) * D + c;
   const float inv = 1.f / l;

@@ -113,3 +113,38 @@ def test_member_with_no_own_tokens_and_empty_rows():
     torch.cuda.synchronize()
     assert int(err.item()) == 0
     assert_close(workloads.independent([1]), out, ref)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("all_empty", [False, True])
+def test_group_with_no_shared_tokens(all_empty):
+    """A group whose prefix is 0 streams only its members' own tokens.  A member of length
+    0 gets a zero row; so does every member when all are empty (the group has no tile)."""
+    import paged_kv_cache_350_b200 as pa
+    from oracle import ref_decode
+    rng = np.random.default_rng(12)
+    B, Hq, Hkv, D, bs, NB = 4, 8, 2, 128, 16, 16
+    kp = torch.from_numpy(rng.standard_normal((NB, bs, Hkv, D)).astype(np.float32)).to(torch.bfloat16)
+    vp = torch.from_numpy(rng.standard_normal((NB, bs, Hkv, D)).astype(np.float32)).to(torch.bfloat16)
+    q = torch.from_numpy(rng.standard_normal((B, Hq, D)).astype(np.float32)).to(torch.bfloat16)
+    tables = np.array([[3, 7, 1, -1], [2, 9, -1, -1], [-1, -1, -1, -1], [5, 11, 0, 4]],
+                      dtype=np.int32)
+    lens = np.array([0, 0, 0, 50] if all_empty else [40, 21, 0, 50], dtype=np.int32)
+    h = lambda t: t.view(torch.int16).numpy().view(np.uint16)
+    ref = ref_decode(h(q), h(kp), h(vp), tables, lens, 0.1)
+    n = pa.pa_decode_shared_prefix_workspace_size(B, Hq, Hkv, D, bs, 1)
+    ws = torch.full((n,), 0xA5, dtype=torch.uint8, device="cuda")
+    out = torch.full_like(q, float("nan")).cuda()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.pa_decode_shared_prefix(out, q.cuda(), kp.cuda(), vp.cuda(), torch.from_numpy(tables).cuda(),
+                               torch.from_numpy(lens).cuda(), 0.1,
+                               torch.tensor([0, 0, 0, -1], dtype=torch.int32, device="cuda"),
+                               torch.tensor([0], dtype=torch.int32, device="cuda"),
+                               torch.tensor([[0, 1, 2, -1]], dtype=torch.int32, device="cuda"),
+                               ws, err_flag=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    got = out.float().cpu().numpy()
+    for b in np.flatnonzero(lens == 0):
+        assert (got[b] == 0).all()
+    assert_close(workloads.independent([1]), out, ref)
