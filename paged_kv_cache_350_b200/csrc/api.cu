@@ -321,6 +321,7 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_pool,
     return PA_ERR_INVALID_ARG;
   if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) ||
       !aligned(block_tables, 4) || !aligned(seq_lens, 4) || !aligned(group_of, 4) ||
+      (ngroups > 0 && (!aligned(group_prefix, 4) || !aligned(group_members, 4))) ||
       (dev_err_flag && !aligned(dev_err_flag, 4)) || !workspace || !aligned(workspace, 256))
     return PA_ERR_INVALID_ARG;
   const int grid = pa::prefix_grid(D, block_size, B + ngroups);

@@ -137,3 +137,42 @@ def test_cache_op_argument_errors():
                             vp(0)) == b.PA_ERR_INVALID_ARG
     assert L.pa_copy_blocks(vp(16), vp(16), vp(16), -1, 16, 8, 128, 4, b.PA_BF16, vp(0),
                             vp(0)) == b.PA_ERR_INVALID_ARG
+
+
+def _call_shared_prefix(**kw):
+    from paged_kv_cache_350_b200 import binding as b
+    a = dict(out=16, q=16, k=16, v=16, t=16, l=16, B=2, Hq=8, Hkv=2, D=128, bs=16, MB=4, NB=8,
+             scale=0.1, dtype=b.PA_BF16, gof=16, gpre=16, gmem=16, ng=1, maxm=2, ws=256, wsb=1 << 20,
+             err=0)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    return b.lib.pa_decode_shared_prefix(
+        vp(a["out"]), vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["t"]), vp(a["l"]), a["B"], a["Hq"],
+        a["Hkv"], a["D"], a["bs"], a["MB"], a["NB"], a["scale"], a["dtype"], vp(a["gof"]),
+        vp(a["gpre"]), vp(a["gmem"]), a["ng"], a["maxm"], vp(a["ws"]), a["wsb"], vp(a["err"]),
+        vp(0))
+
+
+def test_shared_prefix_argument_errors_are_reported_before_any_launch():
+    from paged_kv_cache_350_b200 import binding as b
+    assert _call_shared_prefix(B=0) == b.PA_OK                    # empty batch: nothing to do
+    assert _call_shared_prefix(Hq=6, Hkv=4) == b.PA_ERR_INVALID_ARG
+    assert _call_shared_prefix(maxm=0) == b.PA_ERR_INVALID_ARG
+    assert _call_shared_prefix(ng=-1) == b.PA_ERR_INVALID_ARG
+    assert _call_shared_prefix(scale=float("inf")) == b.PA_ERR_INVALID_ARG
+    assert _call_shared_prefix(maxm=5) == b.PA_ERR_UNSUPPORTED    # 5 members x 4 heads > 16 rows
+    assert _call_shared_prefix(dtype=b.PA_F32) == b.PA_ERR_UNSUPPORTED
+    assert _call_shared_prefix(D=96) == b.PA_ERR_UNSUPPORTED
+    assert _call_shared_prefix(B=8000, ng=500) == b.PA_ERR_UNSUPPORTED  # more rows than the kernel takes
+    assert _call_shared_prefix(gof=0) == b.PA_ERR_INVALID_ARG
+    assert _call_shared_prefix(gmem=0) == b.PA_ERR_INVALID_ARG    # groups without member lists
+    assert _call_shared_prefix(gpre=18) == b.PA_ERR_INVALID_ARG   # misaligned int32 arrays
+    assert _call_shared_prefix(gmem=18) == b.PA_ERR_INVALID_ARG
+    assert _call_shared_prefix(gof=18) == b.PA_ERR_INVALID_ARG
+    assert _call_shared_prefix(out=8) == b.PA_ERR_INVALID_ARG
+    assert _call_shared_prefix(ws=0) == b.PA_ERR_INVALID_ARG
+    assert _call_shared_prefix(ws=128) == b.PA_ERR_INVALID_ARG    # workspace not 256-byte aligned
+    assert _call_shared_prefix(err=2) == b.PA_ERR_INVALID_ARG
+    # no groups: the group arrays other than group_of may be NULL
+    assert _call_shared_prefix(ng=0, gpre=0, gmem=0, out=8) == b.PA_ERR_INVALID_ARG
+    assert b.pa_decode_shared_prefix_workspace_size(2, 8, 2, 128, 16, 1) > 0
