@@ -177,6 +177,21 @@ def _need(cond, msg):
         raise ValueError(msg)
 
 
+def _on_device(*ts, err_flag=None):
+    """Every tensor (None skipped) must live on the current CUDA device: the library takes
+    raw device pointers and launches there, so a host tensor would be read by a kernel.
+    err_flag, when given, is an int32 device tensor of at least one element."""
+    import torch
+    dev = torch.cuda.current_device() if torch.cuda.is_available() else None
+    for t in (*ts, err_flag):
+        if t is None:
+            continue
+        _need(t.is_cuda, "tensors must be CUDA tensors (the library takes device pointers)")
+        _need(t.device.index == dev, f"tensors must be on the current device (cuda:{dev})")
+    _need(err_flag is None or (err_flag.dtype == torch.int32 and err_flag.numel() >= 1),
+          "err_flag must be an int32 tensor of at least one element")
+
+
 # ---------------------------------------------------------------------------
 # decode
 # ---------------------------------------------------------------------------
@@ -209,6 +224,7 @@ def pa_decode(out, q, k_pool, v_pool, block_tables, seq_lens, scale, workspace=N
     _need(seq_lens.dtype == torch.int32 and seq_lens.numel() == q.shape[0], "seq_lens int32 [B]")
     for t in (out, q, k_pool, v_pool, block_tables, seq_lens):
         _need(t.is_contiguous(), "tensors must be contiguous")
+    _on_device(out, q, k_pool, v_pool, block_tables, seq_lens, workspace, err_flag=err_flag)
     _need(q.dtype == out.dtype == k_pool.dtype == v_pool.dtype, "q, out and pools share a dtype")
     B, Hq, D = q.shape
     NB, bs, Hkv, D2 = k_pool.shape
@@ -240,6 +256,8 @@ def pa_decode_append(out, q, k_new, v_new, k_pool, v_pool, block_tables, seq_len
     _need(k_new.shape == (B, Hkv, D) and v_new.shape == k_new.shape, "k_new/v_new must be [B, Hkv, D]")
     for t in (out, q, k_new, v_new, k_pool, v_pool, block_tables, seq_lens):
         _need(t.is_contiguous(), "tensors must be contiguous")
+    _on_device(out, q, k_new, v_new, k_pool, v_pool, block_tables, seq_lens, workspace,
+               err_flag=err_flag)
     _need(q.dtype == out.dtype == k_new.dtype == v_new.dtype == k_pool.dtype == v_pool.dtype,
           "q, out, new K/V and pools share a dtype")
     wbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
@@ -269,6 +287,8 @@ def decode_append_args(out, q, k_new, v_new, k_pool, v_pool, block_tables, seq_l
     _need(k_new.shape == (B, Hkv, D) and v_new.shape == k_new.shape, "k_new/v_new must be [B, Hkv, D]")
     for t in (out, q, k_new, v_new, k_pool, v_pool, block_tables, seq_lens):
         _need(t.is_contiguous(), "tensors must be contiguous")
+    _on_device(out, q, k_new, v_new, k_pool, v_pool, block_tables, seq_lens, workspace,
+               err_flag=err_flag)
     _need(q.dtype == out.dtype == k_new.dtype == v_new.dtype == k_pool.dtype == v_pool.dtype,
           "q, out, new K/V and pools share a dtype")
     wbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
@@ -299,6 +319,7 @@ def pa_decode_no_alloc(out, q, k_pool, v_pool, block_tables, seq_lens, scale, er
     _need(seq_lens.dtype == torch.int32 and seq_lens.numel() == q.shape[0], "seq_lens int32 [B]")
     for t in (out, q, k_pool, v_pool, block_tables, seq_lens):
         _need(t.is_contiguous(), "tensors must be contiguous")
+    _on_device(out, q, k_pool, v_pool, block_tables, seq_lens, err_flag=err_flag)
     _need(q.dtype == out.dtype == k_pool.dtype == v_pool.dtype, "q, out and pools share a dtype")
     B, Hq, D = q.shape
     NB, bs, Hkv, D2 = k_pool.shape
@@ -328,13 +349,19 @@ def pa_decode_shared_prefix(out, q, k_pool, v_pool, block_tables, seq_lens, scal
     import torch
     _need(q.dim() == 3 and out.shape == q.shape, "q/out must be [B, Hq, D]")
     _need(k_pool.dim() == 4 and v_pool.shape == k_pool.shape, "pools must be [NB, bs, Hkv, D]")
-    _need(block_tables.dtype == torch.int32 and seq_lens.dtype == torch.int32, "int32 tables/lens")
+    _need(block_tables.dim() == 2 and block_tables.dtype == torch.int32, "block_tables int32 [B, MB]")
+    _need(seq_lens.dtype == torch.int32 and seq_lens.numel() == q.shape[0], "seq_lens int32 [B]")
     _need(group_of.dtype == torch.int32 and group_of.numel() == q.shape[0], "group_of int32 [B]")
+    _need(group_prefix.dtype == torch.int32, "group_prefix int32 [ngroups]")
     _need(group_members.dim() == 2 and group_members.dtype == torch.int32, "members int32 [ng, m]")
     for t in (out, q, k_pool, v_pool, block_tables, seq_lens, group_of, group_prefix, group_members):
         _need(t.is_contiguous(), "tensors must be contiguous")
+    _on_device(out, q, k_pool, v_pool, block_tables, seq_lens, group_of, group_prefix,
+               group_members, workspace, err_flag=err_flag)
+    _need(q.dtype == out.dtype == k_pool.dtype == v_pool.dtype, "q, out and pools share a dtype")
     B, Hq, D = q.shape
-    NB, bs, Hkv, _ = k_pool.shape
+    NB, bs, Hkv, D2 = k_pool.shape
+    _need(D2 == D and block_tables.shape[0] == B, "shape mismatch")
     ng, maxm = group_members.shape
     _need(group_prefix.numel() >= ng, "group_prefix [ngroups]")
     wbytes = workspace.numel() * workspace.element_size()
@@ -354,8 +381,10 @@ def pa_reshape_and_cache(key, value, k_pool, v_pool, slot_mapping, err_flag=None
     _need(slot_mapping.dtype == torch.int64 and slot_mapping.numel() == key.shape[0],
           "slot_mapping int64 [T]")
     _need(key.dtype == value.dtype == k_pool.dtype == v_pool.dtype, "dtype mismatch")
+    _need(k_pool.dim() == 4 and v_pool.shape == k_pool.shape, "pools must be [NB, bs, Hkv, D]")
     for t in (key, value, k_pool, v_pool, slot_mapping):
         _need(t.is_contiguous(), "tensors must be contiguous")
+    _on_device(key, value, k_pool, v_pool, slot_mapping, err_flag=err_flag)
     NB, bs, Hkv, D = k_pool.shape
     _need(key.shape[1:] == (Hkv, D), "key rows must be [Hkv, D] of the pool")
     st = lib.pa_reshape_and_cache(_ptr(key), _ptr(value), _ptr(k_pool), _ptr(v_pool),
@@ -369,8 +398,11 @@ def pa_copy_blocks(k_pool, v_pool, pairs, err_flag=None, stream=None):
     import torch
     _need(pairs.dtype == torch.int32 and (pairs.numel() == 0 or pairs.shape[-1] == 2),
           "pairs int32 [n, 2]")
+    _need(k_pool.dim() == 4 and v_pool.shape == k_pool.shape and v_pool.dtype == k_pool.dtype,
+          "pools must be [NB, bs, Hkv, D] of one dtype")
     _need(pairs.is_contiguous() and k_pool.is_contiguous() and v_pool.is_contiguous(),
           "tensors must be contiguous")
+    _on_device(k_pool, v_pool, pairs, err_flag=err_flag)
     NB, bs, Hkv, D = k_pool.shape
     n = pairs.numel() // 2
     st = lib.pa_copy_blocks(_ptr(k_pool), _ptr(v_pool), _ptr(pairs), n, bs, Hkv, D, NB,
@@ -380,6 +412,8 @@ def pa_copy_blocks(k_pool, v_pool, pairs, err_flag=None, stream=None):
 
 def pa_selftest_bounded_wait(err_flag, limit_us, stream=None):
     """Run the bounded-wait self-test (see include/pa.h): err_flag gets PA_DEVERR_TIMEOUT."""
+    _need(err_flag is not None, "err_flag is required")
+    _on_device(err_flag=err_flag)
     _check(lib.pa_selftest_bounded_wait(_ptr(err_flag), int(limit_us), _stream(stream)),
            "pa_selftest_bounded_wait")
 

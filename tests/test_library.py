@@ -176,3 +176,37 @@ def test_shared_prefix_argument_errors_are_reported_before_any_launch():
     # no groups: the group arrays other than group_of may be NULL
     assert _call_shared_prefix(ng=0, gpre=0, gmem=0, out=8) == b.PA_ERR_INVALID_ARG
     assert b.pa_decode_shared_prefix_workspace_size(2, 8, 2, 128, 16, 1) > 0
+
+
+def test_binding_rejects_host_tensors_before_the_c_call():
+    """The library takes raw device pointers: a host tensor must never reach a kernel."""
+    import torch
+    from paged_kv_cache_350_b200 import binding as b
+    q = torch.zeros(2, 8, 128, dtype=torch.bfloat16)
+    kp = torch.zeros(4, 16, 2, 128, dtype=torch.bfloat16)
+    tab = torch.zeros(2, 4, dtype=torch.int32)
+    lens = torch.ones(2, dtype=torch.int32)
+    kn = torch.zeros(2, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        b.pa_decode(q.clone(), q, kp, kp.clone(), tab, lens, 0.1)
+    with pytest.raises(ValueError, match="CUDA"):
+        b.pa_decode_append(q.clone(), q, kn, kn.clone(), kp, kp.clone(), tab, lens, 0.1)
+    with pytest.raises(ValueError, match="CUDA"):
+        b.pa_decode_no_alloc(q.clone(), q, kp, kp.clone(), tab, lens, 0.1)
+    with pytest.raises(ValueError, match="CUDA"):
+        b.pa_reshape_and_cache(kn, kn.clone(), kp, kp.clone(), torch.zeros(2, dtype=torch.int64))
+    with pytest.raises(ValueError, match="CUDA"):
+        b.pa_copy_blocks(kp, kp.clone(), torch.zeros(1, 2, dtype=torch.int32))
+    with pytest.raises(ValueError, match="CUDA"):
+        b.pa_decode_shared_prefix(q.clone(), q, kp, kp.clone(), tab, lens, 0.1,
+                                  torch.zeros(2, dtype=torch.int32), torch.zeros(1, dtype=torch.int32),
+                                  torch.zeros(1, 2, dtype=torch.int32), torch.zeros(256, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="err_flag is required"):
+        b.pa_selftest_bounded_wait(None, 1000)
+    # shape and dtype errors come first, with their own messages
+    with pytest.raises(ValueError, match="group_prefix int32"):
+        b.pa_decode_shared_prefix(q.clone(), q, kp, kp.clone(), tab, lens, 0.1,
+                                  torch.zeros(2, dtype=torch.int32), torch.zeros(1, dtype=torch.int64),
+                                  torch.zeros(1, 2, dtype=torch.int32), torch.zeros(256, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="pools must be"):
+        b.pa_copy_blocks(kp, kp[:2], torch.zeros(1, 2, dtype=torch.int32))
