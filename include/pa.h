@@ -81,7 +81,8 @@ typedef enum pa_status {
   PA_ERR_BAD_SEQ_LEN = 8,    /* device flag: seq_lens[b] outside [0, max_blocks*block_size] */
   PA_ERR_BAD_SLOT = 9,       /* device flag: slot >= num_blocks*block_size */
   PA_ERR_TIMEOUT = 10,       /* device flag: a bounded pipeline wait gave up */
-  PA_ERR_SCRATCH_LIMIT = 11  /* pa_decode_no_alloc: the shape needs more than its static scratch */
+  PA_ERR_SCRATCH_LIMIT = 11, /* pa_decode_no_alloc: the shape needs more than its static scratch */
+  PA_ERR_HOST_MEMORY = 12    /* allocator: a host allocation failed; state unchanged */
 } pa_status;
 
 typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
@@ -295,7 +296,9 @@ pa_status pa_copy_blocks(void* k_pool, void* v_pool, const int32_t* pairs, int n
  * full (or absent); when the last block is partial and shared (refcount > 1) the
  * append copies on write: it takes a fresh block dst, reports (src, dst), decrements
  * refcount(src) and points the table at dst.  Freed blocks are pushed in table order
- * when their refcount reaches 0.  A failing call changes no state.  Not thread-safe.
+ * when their refcount reaches 0.  A failing call changes no state, including one that
+ * runs out of host memory (PA_ERR_HOST_MEMORY: every allocation a call needs is made
+ * before it changes anything).  Not thread-safe.
  * ------------------------------------------------------------------------- */
 
 typedef struct pa_allocator pa_allocator;

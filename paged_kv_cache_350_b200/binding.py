@@ -31,6 +31,7 @@ PA_ERR_BAD_SEQ_LEN = 8
 PA_ERR_BAD_SLOT = 9
 PA_ERR_TIMEOUT = 10
 PA_ERR_SCRATCH_LIMIT = 11
+PA_ERR_HOST_MEMORY = 12
 
 # pa_dtype
 PA_F32 = 0

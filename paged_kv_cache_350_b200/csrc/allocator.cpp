@@ -7,11 +7,16 @@
 // is copied (copy on write) so the sibling's prefix stays intact ("深入解析
 // PagedAttention", 核心创新 / 多序列共享; concept card, 实现要点).  The exact policy
 // (LIFO free list, splitmix64 Fisher-Yates shuffle, when a copy happens) is stated in
-// include/pa.h.  Every failing call leaves the state unchanged.
+// include/pa.h.  Every failing call leaves the state unchanged, a failed host allocation
+// included: each entry point allocates (reserves) all it needs before it changes
+// anything, and returns PA_ERR_HOST_MEMORY instead of letting std::bad_alloc cross the
+// C ABI.
 
 #include <algorithm>
 #include <cstring>
+#include <memory>
 #include <new>
+#include <stdexcept>
 #include <unordered_map>
 #include <unordered_set>
 #include <vector>
@@ -64,12 +69,20 @@ bool init_from_order(pa_allocator* a, int num_blocks, int block_size,
   return true;
 }
 
-}  // namespace
+// The entry points' bodies: a failed host allocation (std::bad_alloc, or a size the
+// containers cannot hold) becomes PA_ERR_HOST_MEMORY instead of crossing the C ABI.
+template <class F>
+pa_status guarded(F&& body) {
+  try {
+    return body();
+  } catch (const std::bad_alloc&) {
+    return PA_ERR_HOST_MEMORY;
+  } catch (const std::length_error&) {
+    return PA_ERR_HOST_MEMORY;
+  }
+}
 
-extern "C" {
-
-pa_status pa_alloc_create(int num_blocks, int block_size, uint64_t shuffle_seed,
-                          pa_allocator** out) {
+pa_status create_impl(int num_blocks, int block_size, uint64_t shuffle_seed, pa_allocator** out) {
   if (!out || num_blocks <= 0 || block_size <= 0) return PA_ERR_INVALID_ARG;
   std::vector<int32_t> order(num_blocks);
   for (int i = 0; i < num_blocks; ++i) order[i] = i;
@@ -80,15 +93,14 @@ pa_status pa_alloc_create(int num_blocks, int block_size, uint64_t shuffle_seed,
       std::swap(order[i], order[j]);
     }
   }
-  pa_allocator* a = new (std::nothrow) pa_allocator();
-  if (!a) return PA_ERR_INVALID_ARG;
-  init_from_order(a, num_blocks, block_size, order);
-  *out = a;
+  std::unique_ptr<pa_allocator> a(new pa_allocator());
+  init_from_order(a.get(), num_blocks, block_size, order);
+  *out = a.release();
   return PA_OK;
 }
 
-pa_status pa_alloc_create_ordered(int num_blocks, int block_size, const int32_t* pop_order,
-                                  pa_allocator** out) {
+pa_status create_ordered_impl(int num_blocks, int block_size, const int32_t* pop_order,
+                              pa_allocator** out) {
   if (!out || !pop_order || num_blocks <= 0 || block_size <= 0) return PA_ERR_INVALID_ARG;
   std::vector<int32_t> order(pop_order, pop_order + num_blocks);
   std::vector<char> seen(num_blocks, 0);
@@ -96,40 +108,45 @@ pa_status pa_alloc_create_ordered(int num_blocks, int block_size, const int32_t*
     if (b < 0 || b >= num_blocks || seen[b]) return PA_ERR_INVALID_ARG;
     seen[b] = 1;
   }
-  pa_allocator* a = new (std::nothrow) pa_allocator();
-  if (!a) return PA_ERR_INVALID_ARG;
-  init_from_order(a, num_blocks, block_size, order);
-  *out = a;
+  std::unique_ptr<pa_allocator> a(new pa_allocator());
+  init_from_order(a.get(), num_blocks, block_size, order);
+  *out = a.release();
   return PA_OK;
 }
 
-void pa_alloc_destroy(pa_allocator* a) { delete a; }
-
-pa_status pa_alloc_add_seq(pa_allocator* a, int64_t seq_id, int num_tokens) {
+pa_status add_seq_impl(pa_allocator* a, int64_t seq_id, int num_tokens) {
   if (!a || num_tokens < 0) return PA_ERR_INVALID_ARG;
   if (a->seqs.count(seq_id)) return PA_ERR_EXISTS;
   int64_t need = (static_cast<int64_t>(num_tokens) + a->block_size - 1) / a->block_size;
   if (need > static_cast<int64_t>(a->free_stack.size())) return PA_ERR_OUT_OF_BLOCKS;
-  Seq s;
-  s.table.reserve(need + 1);
+  // allocate the map node and the table first; only then take blocks
+  auto ins = a->seqs.emplace(seq_id, Seq());
+  Seq& s = ins.first->second;
+  try {
+    s.table.reserve(need + 1);
+  } catch (...) {
+    a->seqs.erase(ins.first);
+    throw;
+  }
   for (int64_t i = 0; i < need; ++i) s.table.push_back(a->pop());
   s.ntok = num_tokens;
-  a->seqs.emplace(seq_id, std::move(s));
   return PA_OK;
 }
 
-pa_status pa_alloc_fork(pa_allocator* a, int64_t parent_id, int64_t child_id) {
+pa_status fork_impl(pa_allocator* a, int64_t parent_id, int64_t child_id) {
   if (!a) return PA_ERR_INVALID_ARG;
   auto it = a->seqs.find(parent_id);
   if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
   if (a->seqs.count(child_id)) return PA_ERR_EXISTS;
   Seq child = it->second;  // copy before emplace (rehash may move the parent)
-  for (int32_t b : child.table) a->ref[b] += 1;
-  a->seqs.emplace(child_id, std::move(child));
+  auto ins = a->seqs.emplace(child_id, std::move(child));
+  for (int32_t b : ins.first->second.table) a->ref[b] += 1;
   return PA_OK;
 }
 
-static void append_one(pa_allocator* a, Seq& s, int64_t* slot, int32_t* src, int32_t* dst) {
+// The table must have room for one more entry (reserved by the caller), so nothing here
+// allocates.
+void append_one(pa_allocator* a, Seq& s, int64_t* slot, int32_t* src, int32_t* dst) {
   const int bs = a->block_size;
   const int off = static_cast<int>(s.ntok % bs);
   int32_t phys;
@@ -154,8 +171,8 @@ static void append_one(pa_allocator* a, Seq& s, int64_t* slot, int32_t* src, int
   *slot = static_cast<int64_t>(phys) * bs + off;
 }
 
-pa_status pa_alloc_append_slot(pa_allocator* a, int64_t seq_id, int64_t* slot,
-                               int32_t* cow_src, int32_t* cow_dst) {
+pa_status append_slot_impl(pa_allocator* a, int64_t seq_id, int64_t* slot, int32_t* cow_src,
+                           int32_t* cow_dst) {
   if (!a || !slot || !cow_src || !cow_dst) return PA_ERR_INVALID_ARG;
   auto it = a->seqs.find(seq_id);
   if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
@@ -163,12 +180,13 @@ pa_status pa_alloc_append_slot(pa_allocator* a, int64_t seq_id, int64_t* slot,
   const bool needs_block =
       (s.ntok % a->block_size == 0) || (a->ref[s.table.back()] > 1);
   if (needs_block && a->free_stack.empty()) return PA_ERR_OUT_OF_BLOCKS;
+  s.table.reserve(s.table.size() + 1);
   append_one(a, s, slot, cow_src, cow_dst);
   return PA_OK;
 }
 
-pa_status pa_alloc_append_slots(pa_allocator* a, const int64_t* seq_ids, int n,
-                                int64_t* slot_mapping, int32_t* cow_pairs, int* n_pairs) {
+pa_status append_slots_impl(pa_allocator* a, const int64_t* seq_ids, int n,
+                            int64_t* slot_mapping, int32_t* cow_pairs, int* n_pairs) {
   if (!a || n < 0 || (n > 0 && (!seq_ids || !slot_mapping || !cow_pairs)) || !n_pairs)
     return PA_ERR_INVALID_ARG;
   // Dry run: resolve every sequence, reject duplicates, and count the fresh blocks the
@@ -197,6 +215,7 @@ pa_status pa_alloc_append_slots(pa_allocator* a, const int64_t* seq_ids, int n,
     }
   }
   if (need > static_cast<int64_t>(a->free_stack.size())) return PA_ERR_OUT_OF_BLOCKS;
+  for (Seq* s : rows) s->table.reserve(s->table.size() + 1);  // capacity only: no state
   int np = 0;
   for (int i = 0; i < n; ++i) {
     int32_t src, dst;
@@ -211,7 +230,9 @@ pa_status pa_alloc_append_slots(pa_allocator* a, const int64_t* seq_ids, int n,
   return PA_OK;
 }
 
-pa_status pa_alloc_free_seq(pa_allocator* a, int64_t seq_id) {
+// free_stack holds every block at creation, so its capacity covers all pushes: freeing
+// never allocates.
+pa_status free_seq_impl(pa_allocator* a, int64_t seq_id) {
   if (!a) return PA_ERR_INVALID_ARG;
   auto it = a->seqs.find(seq_id);
   if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
@@ -222,7 +243,7 @@ pa_status pa_alloc_free_seq(pa_allocator* a, int64_t seq_id) {
   return PA_OK;
 }
 
-pa_status pa_alloc_truncate(pa_allocator* a, int64_t seq_id, int num_tokens) {
+pa_status truncate_impl(pa_allocator* a, int64_t seq_id, int num_tokens) {
   if (!a || num_tokens < 0) return PA_ERR_INVALID_ARG;
   auto it = a->seqs.find(seq_id);
   if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
@@ -238,8 +259,8 @@ pa_status pa_alloc_truncate(pa_allocator* a, int64_t seq_id, int num_tokens) {
   return PA_OK;
 }
 
-pa_status pa_alloc_beam_select(pa_allocator* a, const int64_t* seq_ids, const int32_t* parent_idx,
-                               int n) {
+pa_status beam_select_impl(pa_allocator* a, const int64_t* seq_ids, const int32_t* parent_idx,
+                           int n) {
   if (!a || n < 0 || (n > 0 && (!seq_ids || !parent_idx))) return PA_ERR_INVALID_ARG;
   std::vector<Seq*> rows(n);
   std::unordered_set<int64_t> seen;
@@ -251,16 +272,126 @@ pa_status pa_alloc_beam_select(pa_allocator* a, const int64_t* seq_ids, const in
     rows[i] = &it->second;
   }
   std::vector<Seq> next(n);
-  for (int i = 0; i < n; ++i) {
-    next[i] = *rows[parent_idx[i]];
+  for (int i = 0; i < n; ++i) next[i] = *rows[parent_idx[i]];  // every copy before any change
+  for (int i = 0; i < n; ++i)
     for (int32_t b : next[i].table) a->ref[b] += 1;
-  }
   for (int i = 0; i < n; ++i) {
     for (int32_t b : rows[i]->table)
       if (--a->ref[b] == 0) a->free_stack.push_back(b);
   }
   for (int i = 0; i < n; ++i) *rows[i] = std::move(next[i]);
   return PA_OK;
+}
+
+pa_status prefix_groups_impl(const pa_allocator* a, const int64_t* seq_ids, int n,
+                             int max_members, int align_tokens, int32_t* group_of,
+                             int32_t* group_prefix, int32_t* group_members, int* ngroups) {
+  if (!a || n < 0 || max_members < 1 || align_tokens < 1 || !ngroups ||
+      (n > 0 && (!seq_ids || !group_of || !group_prefix || !group_members)))
+    return PA_ERR_INVALID_ARG;
+  std::vector<const Seq*> rows(n);
+  for (int i = 0; i < n; ++i) {
+    auto it = a->seqs.find(seq_ids[i]);
+    if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
+    rows[i] = &it->second;
+    group_of[i] = -1;
+  }
+  // rows by first block, in batch order (first-appearance order of the blocks)
+  std::vector<int32_t> firsts;
+  std::unordered_map<int32_t, std::vector<int>> buckets;
+  for (int i = 0; i < n; ++i) {
+    if (rows[i]->table.empty()) continue;
+    const int32_t f = rows[i]->table[0];
+    auto& v = buckets[f];
+    if (v.empty()) firsts.push_back(f);
+    v.push_back(i);
+  }
+  int ng = 0;
+  for (int32_t f : firsts) {
+    const std::vector<int>& v = buckets[f];
+    for (size_t c0 = 0; c0 < v.size(); c0 += max_members) {
+      const size_t c1 = std::min(v.size(), c0 + static_cast<size_t>(max_members));
+      if (c1 - c0 < 2) continue;
+      size_t k = rows[v[c0]]->table.size();
+      int64_t shortest = rows[v[c0]]->ntok;
+      for (size_t m = c0 + 1; m < c1; ++m) {
+        const Seq& s = *rows[v[m]];
+        size_t j = 0;
+        while (j < k && j < s.table.size() && s.table[j] == rows[v[c0]]->table[j]) ++j;
+        k = j;
+        shortest = std::min<int64_t>(shortest, s.ntok);
+      }
+      int64_t prefix = std::min<int64_t>(static_cast<int64_t>(k) * a->block_size, shortest);
+      prefix -= prefix % align_tokens;
+      if (prefix <= 0) continue;
+      group_prefix[ng] = static_cast<int32_t>(prefix);
+      for (int m = 0; m < max_members; ++m) {
+        const size_t idx = c0 + m;
+        group_members[static_cast<size_t>(ng) * max_members + m] = idx < c1 ? v[idx] : -1;
+        if (idx < c1) group_of[v[idx]] = ng;
+      }
+      ++ng;
+    }
+  }
+  *ngroups = ng;
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_alloc_create(int num_blocks, int block_size, uint64_t shuffle_seed,
+                          pa_allocator** out) {
+  return guarded([&] { return create_impl(num_blocks, block_size, shuffle_seed, out); });
+}
+
+pa_status pa_alloc_create_ordered(int num_blocks, int block_size, const int32_t* pop_order,
+                                  pa_allocator** out) {
+  return guarded([&] { return create_ordered_impl(num_blocks, block_size, pop_order, out); });
+}
+
+void pa_alloc_destroy(pa_allocator* a) { delete a; }
+
+pa_status pa_alloc_add_seq(pa_allocator* a, int64_t seq_id, int num_tokens) {
+  return guarded([&] { return add_seq_impl(a, seq_id, num_tokens); });
+}
+
+pa_status pa_alloc_fork(pa_allocator* a, int64_t parent_id, int64_t child_id) {
+  return guarded([&] { return fork_impl(a, parent_id, child_id); });
+}
+
+pa_status pa_alloc_append_slot(pa_allocator* a, int64_t seq_id, int64_t* slot,
+                               int32_t* cow_src, int32_t* cow_dst) {
+  return guarded([&] { return append_slot_impl(a, seq_id, slot, cow_src, cow_dst); });
+}
+
+pa_status pa_alloc_append_slots(pa_allocator* a, const int64_t* seq_ids, int n,
+                                int64_t* slot_mapping, int32_t* cow_pairs, int* n_pairs) {
+  return guarded(
+      [&] { return append_slots_impl(a, seq_ids, n, slot_mapping, cow_pairs, n_pairs); });
+}
+
+pa_status pa_alloc_free_seq(pa_allocator* a, int64_t seq_id) {
+  return guarded([&] { return free_seq_impl(a, seq_id); });
+}
+
+pa_status pa_alloc_truncate(pa_allocator* a, int64_t seq_id, int num_tokens) {
+  return guarded([&] { return truncate_impl(a, seq_id, num_tokens); });
+}
+
+pa_status pa_alloc_beam_select(pa_allocator* a, const int64_t* seq_ids, const int32_t* parent_idx,
+                               int n) {
+  return guarded([&] { return beam_select_impl(a, seq_ids, parent_idx, n); });
+}
+
+pa_status pa_alloc_prefix_groups(const pa_allocator* a, const int64_t* seq_ids, int n,
+                                 int max_members, int align_tokens, int32_t* group_of,
+                                 int32_t* group_prefix, int32_t* group_members, int* ngroups) {
+  return guarded([&] {
+    return prefix_groups_impl(a, seq_ids, n, max_members, align_tokens, group_of, group_prefix,
+                              group_members, ngroups);
+  });
 }
 
 pa_status pa_alloc_block_table(const pa_allocator* a, int64_t seq_id, int32_t* out, int cap,
@@ -310,60 +441,6 @@ pa_status pa_alloc_seq_slots(const pa_allocator* a, int64_t seq_id, int64_t* slo
   for (int t = 0; t < m; ++t)
     slots[t] = static_cast<int64_t>(s.table[t / bs]) * bs + t % bs;
   *n = ntok;
-  return PA_OK;
-}
-
-pa_status pa_alloc_prefix_groups(const pa_allocator* a, const int64_t* seq_ids, int n,
-                                 int max_members, int align_tokens, int32_t* group_of,
-                                 int32_t* group_prefix, int32_t* group_members, int* ngroups) {
-  if (!a || n < 0 || max_members < 1 || align_tokens < 1 || !ngroups ||
-      (n > 0 && (!seq_ids || !group_of || !group_prefix || !group_members)))
-    return PA_ERR_INVALID_ARG;
-  std::vector<const Seq*> rows(n);
-  for (int i = 0; i < n; ++i) {
-    auto it = a->seqs.find(seq_ids[i]);
-    if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
-    rows[i] = &it->second;
-    group_of[i] = -1;
-  }
-  // rows by first block, in batch order (first-appearance order of the blocks)
-  std::vector<int32_t> firsts;
-  std::unordered_map<int32_t, std::vector<int>> buckets;
-  for (int i = 0; i < n; ++i) {
-    if (rows[i]->table.empty()) continue;
-    const int32_t f = rows[i]->table[0];
-    auto& v = buckets[f];
-    if (v.empty()) firsts.push_back(f);
-    v.push_back(i);
-  }
-  int ng = 0;
-  for (int32_t f : firsts) {
-    const std::vector<int>& v = buckets[f];
-    for (size_t c0 = 0; c0 < v.size(); c0 += max_members) {
-      const size_t c1 = std::min(v.size(), c0 + static_cast<size_t>(max_members));
-      if (c1 - c0 < 2) continue;
-      size_t k = rows[v[c0]]->table.size();
-      int64_t shortest = rows[v[c0]]->ntok;
-      for (size_t m = c0 + 1; m < c1; ++m) {
-        const Seq& s = *rows[v[m]];
-        size_t j = 0;
-        while (j < k && j < s.table.size() && s.table[j] == rows[v[c0]]->table[j]) ++j;
-        k = j;
-        shortest = std::min<int64_t>(shortest, s.ntok);
-      }
-      int64_t prefix = std::min<int64_t>(static_cast<int64_t>(k) * a->block_size, shortest);
-      prefix -= prefix % align_tokens;
-      if (prefix <= 0) continue;
-      group_prefix[ng] = static_cast<int32_t>(prefix);
-      for (int m = 0; m < max_members; ++m) {
-        const size_t idx = c0 + m;
-        group_members[static_cast<size_t>(ng) * max_members + m] = idx < c1 ? v[idx] : -1;
-        if (idx < c1) group_of[v[idx]] = ng;
-      }
-      ++ng;
-    }
-  }
-  *ngroups = ng;
   return PA_OK;
 }
 

@@ -62,6 +62,7 @@ const char* pa_status_string(pa_status s) {
     case PA_ERR_BAD_SLOT: return "slot outside the pool";
     case PA_ERR_TIMEOUT: return "a bounded device wait expired";
     case PA_ERR_SCRATCH_LIMIT: return "shape needs more scratch than the static no-alloc buffer";
+    case PA_ERR_HOST_MEMORY: return "out of host memory";
   }
   return "unknown status";
 }

@@ -27,8 +27,10 @@ def test_every_declared_symbol_is_exported():
 
 def test_status_strings_and_flag_mapping():
     from paged_kv_cache_350_b200 import binding as b
-    for s in range(11):
-        assert b.lib.pa_status_string(s)
+    for s in range(13):
+        assert b.lib.pa_status_string(s) != b"unknown status"
+    assert b.lib.pa_status_string(b.PA_ERR_HOST_MEMORY) == b"out of host memory"
+    assert b.lib.pa_status_string(99) == b"unknown status"
     assert b.lib.pa_status_from_device_flag(0) == b.PA_OK
     assert b.lib.pa_status_from_device_flag(b.PA_DEVERR_BAD_BLOCK_ID | 8) == b.PA_ERR_BAD_BLOCK_ID
     assert b.lib.pa_status_from_device_flag(b.PA_DEVERR_TIMEOUT) == b.PA_ERR_TIMEOUT
