@@ -212,3 +212,24 @@ def test_binding_rejects_host_tensors_before_the_c_call():
                                   torch.zeros(1, 2, dtype=torch.int32), torch.zeros(256, dtype=torch.uint8))
     with pytest.raises(ValueError, match="pools must be"):
         b.pa_copy_blocks(kp, kp[:2], torch.zeros(1, 2, dtype=torch.int32))
+
+
+def test_header_compiles_as_c_and_the_allocator_runs_from_plain_c(tmp_path):
+    """include/pa.h is a C header (strict C11) and the library serves a C client: the
+    allocator's copy-on-write story run from tests/c/alloc_abi.c, no Python in the path."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    from paged_kv_cache_350_b200 import binding
+    libdir = os.path.dirname(binding._LIB_PATH)
+    libname = os.path.basename(binding._LIB_PATH)
+    if libname != "libpagedattn.so":
+        pytest.skip("a renamed build of the library is loaded")
+    exe = str(tmp_path / "alloc_abi")
+    subprocess.run([cc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "c", "alloc_abi.c"),
+                    "-L", libdir, "-lpagedattn", f"-Wl,-rpath,{libdir}", "-o", exe], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stdout + r.stderr
