@@ -18,7 +18,6 @@
 #include <new>
 #include <stdexcept>
 #include <unordered_map>
-#include <unordered_set>
 #include <vector>
 
 #include "pa.h"
@@ -28,7 +27,15 @@ namespace {
 struct Seq {
   std::vector<int32_t> table;
   int64_t ntok = 0;
+  uint64_t mark = 0;  // epoch of the batch call that last listed it (duplicate check)
 };
+
+// Room for one more table entry, grown geometrically.  Capacity only: no allocator
+// state changes, so a call may do this before it knows it will succeed.
+void reserve_one(Seq& s) {
+  if (s.table.size() == s.table.capacity())
+    s.table.reserve(s.table.size() < 8 ? 8 : 2 * s.table.size());
+}
 
 // splitmix64 (Steele, Lea & Flood, OOPSLA 2014).
 struct SplitMix64 {
@@ -49,6 +56,7 @@ struct pa_allocator {
   std::vector<int32_t> free_stack;  // back() is popped first
   std::vector<int32_t> ref;
   std::unordered_map<int64_t, Seq> seqs;
+  uint64_t epoch = 0;  // one per batch call: marks the sequences it has listed
 
   int32_t pop() {
     int32_t b = free_stack.back();
@@ -180,7 +188,7 @@ pa_status append_slot_impl(pa_allocator* a, int64_t seq_id, int64_t* slot, int32
   const bool needs_block =
       (s.ntok % a->block_size == 0) || (a->ref[s.table.back()] > 1);
   if (needs_block && a->free_stack.empty()) return PA_ERR_OUT_OF_BLOCKS;
-  s.table.reserve(s.table.size() + 1);
+  if (s.ntok % a->block_size == 0) reserve_one(s);
   append_one(a, s, slot, cow_src, cow_dst);
   return PA_OK;
 }
@@ -192,18 +200,19 @@ pa_status append_slots_impl(pa_allocator* a, const int64_t* seq_ids, int n,
   // Dry run: resolve every sequence, reject duplicates, and count the fresh blocks the
   // batch takes, replaying the refcount drops of earlier copies in the same batch.
   std::vector<Seq*> rows(n);
-  std::unordered_set<int64_t> seen;
-  seen.reserve(static_cast<size_t>(n) * 2);
   std::unordered_map<int32_t, int> dropped;
+  const uint64_t epoch = ++a->epoch;
   int64_t need = 0;
   for (int i = 0; i < n; ++i) {
     auto it = a->seqs.find(seq_ids[i]);
     if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
-    if (!seen.insert(seq_ids[i]).second) return PA_ERR_INVALID_ARG;
     Seq& s = it->second;
+    if (s.mark == epoch) return PA_ERR_INVALID_ARG;  // listed twice
+    s.mark = epoch;
     rows[i] = &s;
     if (s.ntok % a->block_size == 0) {
       need += 1;
+      reserve_one(s);
     } else {
       int32_t last = s.table.back();
       auto d = dropped.find(last);
@@ -215,7 +224,6 @@ pa_status append_slots_impl(pa_allocator* a, const int64_t* seq_ids, int n,
     }
   }
   if (need > static_cast<int64_t>(a->free_stack.size())) return PA_ERR_OUT_OF_BLOCKS;
-  for (Seq* s : rows) s->table.reserve(s->table.size() + 1);  // capacity only: no state
   int np = 0;
   for (int i = 0; i < n; ++i) {
     int32_t src, dst;
@@ -263,11 +271,12 @@ pa_status beam_select_impl(pa_allocator* a, const int64_t* seq_ids, const int32_
                            int n) {
   if (!a || n < 0 || (n > 0 && (!seq_ids || !parent_idx))) return PA_ERR_INVALID_ARG;
   std::vector<Seq*> rows(n);
-  std::unordered_set<int64_t> seen;
+  const uint64_t epoch = ++a->epoch;
   for (int i = 0; i < n; ++i) {
     auto it = a->seqs.find(seq_ids[i]);
     if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
-    if (!seen.insert(seq_ids[i]).second) return PA_ERR_INVALID_ARG;
+    if (it->second.mark == epoch) return PA_ERR_INVALID_ARG;  // listed twice
+    it->second.mark = epoch;
     if (parent_idx[i] < 0 || parent_idx[i] >= n) return PA_ERR_INVALID_ARG;
     rows[i] = &it->second;
   }
@@ -410,23 +419,27 @@ pa_status pa_alloc_block_table(const pa_allocator* a, int64_t seq_id, int32_t* o
 
 pa_status pa_alloc_block_tables(const pa_allocator* a, const int64_t* seq_ids, int n,
                                 int32_t* block_tables, int max_blocks, int32_t* seq_lens) {
-  if (!a || n < 0 || max_blocks <= 0 ||
-      (n > 0 && (!seq_ids || !block_tables || !seq_lens)))
-    return PA_ERR_INVALID_ARG;
-  for (int i = 0; i < n; ++i) {
-    auto it = a->seqs.find(seq_ids[i]);
-    if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
-    if (static_cast<int>(it->second.table.size()) > max_blocks) return PA_ERR_INVALID_ARG;
-  }
-  for (int i = 0; i < n; ++i) {
-    const Seq& s = a->seqs.find(seq_ids[i])->second;
-    int32_t* row = block_tables + static_cast<int64_t>(i) * max_blocks;
-    int len = static_cast<int>(s.table.size());
-    if (len) std::memcpy(row, s.table.data(), sizeof(int32_t) * len);
-    for (int j = len; j < max_blocks; ++j) row[j] = -1;
-    seq_lens[i] = static_cast<int32_t>(s.ntok);
-  }
-  return PA_OK;
+  return guarded([&]() -> pa_status {
+    if (!a || n < 0 || max_blocks <= 0 ||
+        (n > 0 && (!seq_ids || !block_tables || !seq_lens)))
+      return PA_ERR_INVALID_ARG;
+    std::vector<const Seq*> rows(n);
+    for (int i = 0; i < n; ++i) {
+      auto it = a->seqs.find(seq_ids[i]);
+      if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
+      if (static_cast<int>(it->second.table.size()) > max_blocks) return PA_ERR_INVALID_ARG;
+      rows[i] = &it->second;
+    }
+    for (int i = 0; i < n; ++i) {
+      const Seq& s = *rows[i];
+      int32_t* row = block_tables + static_cast<int64_t>(i) * max_blocks;
+      int len = static_cast<int>(s.table.size());
+      if (len) std::memcpy(row, s.table.data(), sizeof(int32_t) * len);
+      for (int j = len; j < max_blocks; ++j) row[j] = -1;
+      seq_lens[i] = static_cast<int32_t>(s.ntok);
+    }
+    return PA_OK;
+  });
 }
 
 pa_status pa_alloc_seq_slots(const pa_allocator* a, int64_t seq_id, int64_t* slots, int cap,
