@@ -483,8 +483,8 @@ __global__ void __launch_bounds__(kThreads, kMinCtas)
     const int jend = t.j + (pend - gpos);
     for (int j = t.j; j < jend; ++j, ++i) {
       const int stage = warp * SPW + i % SPW;
-      if (!mbar_wait(smem_addr(&full_bar[stage]), (i / SPW) & 1, p.err)) {
-        ok = false;
+      if (!mbar_wait_warp(smem_addr(&full_bar[stage]), (i / SPW) & 1, p.err)) {
+        ok = false;  // the same in every lane: the warp leaves the loop together
         break;
       }
       int valid, row_lo = 0, row_hi = kRows;

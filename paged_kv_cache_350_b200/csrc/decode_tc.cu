@@ -174,7 +174,8 @@ __global__ void __launch_bounds__(C::THREADS)
 
   for (int tile = warp; tile < ntiles; tile += NCW) {
     const int stage = tile % NSTAGE;
-    if (!mbar_wait(smem_addr(&full_bar[stage]), (tile / NSTAGE) & 1, p.err)) break;
+    // one verdict per warp: no lane goes on alone into the tile's ldmatrix / mma.sync
+    if (!mbar_wait_warp(smem_addr(&full_bar[stage]), (tile / NSTAGE) & 1, p.err)) break;
     uint8_t* st_ptr = smem + stage * C::STAGE_BYTES;
     const int valid = min(TILE_T, tok1 - (tok0 + tile * TILE_T));
     if (valid < TILE_T) zero_tail_rows<C>(st_ptr, valid, lane);

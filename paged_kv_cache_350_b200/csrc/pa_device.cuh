@@ -83,6 +83,17 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t
   }
 }
 
+// mbar_wait for a whole warp, with one verdict for all 32 lanes: every lane waits
+// (bounded), then the lanes agree, so the phase counts as complete only if it did for
+// every lane.  A warp that gives up therefore leaves its loop as a whole, and no lane
+// goes on alone into warp-collective code (ldmatrix, mma.sync, full-mask shuffles),
+// which would never complete.  Call from all 32 lanes, converged.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, int32_t* err,
+                                               uint64_t limit_ns = kWaitLimitNs) {
+  const bool got = mbar_wait(bar, parity, err, limit_ns);
+  return __all_sync(0xffffffffu, got) != 0;
+}
+
 // Order this thread's generic-proxy shared-memory writes before later async-proxy
 // (TMA) accesses of the same bytes.
 __device__ __forceinline__ void fence_proxy_async_smem() {
