@@ -12,9 +12,19 @@ import torch
 import workloads
 from oracle import RefAllocator, ref_copy_blocks, ref_decode, ref_reshape_and_cache
 
-BF16_ABS = 1e-2   # bf16: max |gpu - oracle|, or one bf16 ulp of the oracle value if larger
-BF16_REL = 2e-2   # bf16: max over (b, h) rows of max|gpu - oracle| / max|oracle|
-F32_ABS = 1e-4    # fp32 inputs: max |gpu - oracle|
+# Tolerances of the bf16 attention outputs: max-abs-error <= 1e-2 and max-rel-error <= 2e-2
+# against the float64 oracle; <= 1e-4 abs for fp32 inputs.
+BF16_ABS = 1e-2     # elementwise |g - r|, where the bf16 output format can hold it (below)
+BF16_REL = 2e-2     # elementwise |g - r| / max(|r|, REL_FLOOR)
+REL_FLOOR = 1e-3    # so that outputs near zero do not turn rounding noise into a ratio
+F32_ABS = 1e-4      # fp32 inputs: max |g - r|
+# What the bf16 path may differ from the exact value by before its one final rounding to
+# bf16.  It computes in fp32; the largest term is P entering the P.V product as two bf16
+# parts, hi = rn(p) and lo = rn(p - hi), so |p - hi - lo| <= 2^-18 p and the output moves
+# by at most 2^-18 * sum_t p_t |v_t| <= 2^-18 * max|v| (< 8 for N(0,1) draws): 3.1e-5.
+# exp2, the fp32 sums and the tensor cores' fp32 accumulation add orders of magnitude
+# less at these logit sizes.  The slack is about three times that bound.
+F32_SLACK = 1e-4
 
 
 def torch_dtype(w):
@@ -101,36 +111,76 @@ def bf16_ulp(x):
     return np.exp2(np.floor(np.log2(ax)) - 7)
 
 
-def errors(gpu_out, ref_out, bf16=False):
-    """(max abs error, max row-normwise relative error) of gpu vs oracle outputs.
+def abs_bar(r, exact_ref=True):
+    """Elementwise bound on |g - r| for a bf16 output g.
 
-    With ``bf16`` the absolute error is measured in excess of the output
-    format's resolution: elementwise ``|g - r|`` where one bf16 ulp of ``r`` is
-    at most 1e-2, and ``|g - r| * 1e-2 / ulp(r)`` where it is larger (|r| >= 2),
-    so the bar 1e-2 means "within 1e-2, or within one bf16 ulp of the exact
-    value when 1e-2 is finer than the format"."""
-    g = gpu_out.float().cpu().numpy().astype(np.float64)
+    The literal 1e-2, except where bf16 cannot resolve it: a kernel that computes in fp32
+    and rounds once to nearest lands within half a bf16 ulp of its fp32 value, which is
+    within F32_SLACK of the exact value, so the bound is max(1e-2, ulp(r)/2 + F32_SLACK).
+    Half an ulp exceeds 1e-2 only for |r| >= 4 (ulp 2^-5 there).  With ``exact_ref`` False
+    the reference r is itself a rounded GPU output (two GPU paths compared): both lie
+    within that bound of the exact value, so they may differ by twice it."""
+    r = np.asarray(r, dtype=np.float64)
+    k = 1.0 if exact_ref else 2.0
+    return np.maximum(BF16_ABS, k * (0.5 * bf16_ulp(r) + F32_SLACK))
+
+
+def errors(gpu_out, ref_out, bf16=False, exact_ref=True):
+    """Parity figures of gpu vs reference outputs (``[..., D]``), as a dict:
+
+    abs       max |g - r|
+    abs_bar   max |g - r| / abs_bar(r)  (bf16; <= 1 passes)
+    rel       max elementwise |g - r| / max(|r|, REL_FLOOR)  (the asserted relative error)
+    rel_unfloored  max elementwise |g - r| / |r| over r != 0  (reported only)
+    rel_row   max over rows of max_d |g - r| / max_d |r|     (reported only)
+    """
+    g = gpu_out.float().cpu().numpy().astype(np.float64) if hasattr(gpu_out, "cpu") \
+        else np.asarray(gpu_out, dtype=np.float64)
     r = np.asarray(ref_out, dtype=np.float64)
     diff = np.abs(g - r)
-    scaled = diff
+    res = {"abs": float(diff.max()) if diff.size else 0.0, "abs_bar": 0.0, "rel": 0.0,
+           "rel_unfloored": 0.0, "rel_row": 0.0, "n": int(diff.size)}
+    if not diff.size:
+        return res
     if bf16:
-        ulp = bf16_ulp(r)
-        scaled = np.where(ulp > BF16_ABS, diff * BF16_ABS / ulp, diff)
-    abs_err = float(scaled.max()) if diff.size else 0.0
-    scale = np.abs(r).max(axis=-1)
+        res["abs_bar"] = float((diff / abs_bar(r, exact_ref)).max())
+    ar = np.abs(r)
+    res["rel"] = float((diff / np.maximum(ar, REL_FLOOR)).max())
+    nz = ar > 0
+    res["rel_unfloored"] = float((diff[nz] / ar[nz]).max()) if nz.any() else 0.0
+    scale = ar.max(axis=-1)
     row_err = diff.max(axis=-1)
-    nz = scale > 0
-    rel = float((row_err[nz] / scale[nz]).max()) if nz.any() else 0.0
+    rows = scale > 0
+    res["rel_row"] = float((row_err[rows] / scale[rows]).max()) if rows.any() else 0.0
     # rows whose reference is exactly zero (empty sequences) must be exactly zero
-    if (~nz).any():
-        assert float(row_err[~nz].max()) == 0.0
-    return abs_err, rel
+    if (~rows).any():
+        assert float(row_err[~rows].max()) == 0.0, "a zero reference row is not zero"
+    return res
 
 
-def assert_close(w, gpu_out, ref_out):
-    a, r = errors(gpu_out, ref_out, bf16=(w.dtype == "bf16"))
-    if w.dtype == "bf16":
-        assert a <= BF16_ABS and r <= BF16_REL, (a, r)
+def _log(w, res, exact_ref):
+    """Append the figures to the file named by PA_PARITY_LOG (when set), one JSON line per
+    comparison, so that a GPU run leaves a record of the errors it saw."""
+    import json
+    import os
+    path = os.environ.get("PA_PARITY_LOG")
+    if not path:
+        return
+    rec = {"test": os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0], "workload": w.name,
+           "dtype": w.dtype, "exact_ref": exact_ref, **res}
+    with open(path, "a") as f:
+        f.write(json.dumps(rec) + "\n")
+
+
+def assert_close(w, gpu_out, ref_out, exact_ref=True):
+    """Assert the tolerances: bf16, elementwise |g - r| <= abs_bar(r) and
+    |g - r| / max(|r|, 1e-3) <= 2e-2; fp32, |g - r| <= 1e-4.  ``exact_ref``: the reference
+    is the float64 oracle (False: another GPU path's bf16 output).  Returns the figures."""
+    bf16 = w.dtype == "bf16"
+    res = errors(gpu_out, ref_out, bf16=bf16, exact_ref=exact_ref)
+    _log(w, res, exact_ref)
+    if bf16:
+        assert res["abs_bar"] <= 1.0 and res["rel"] <= BF16_REL, res
     else:
-        assert a <= F32_ABS, a
-    return a, r
+        assert res["abs"] <= F32_ABS, res
+    return res

@@ -1,48 +1,61 @@
 """GPU parity at the full serving sizes, in the launch configuration bench.py times
 (automatic path and partitioning, workspace from pa_decode_workspace_size).
 
-The oracle computes a sample of batch rows one by one; the remaining rows are
-checked for the properties that hold at any size (finite, and each output row
-inside the convex hull bound max|v| of its values)."""
+Every output row of every serving batch is compared with the float64 oracle.  The oracle
+runs on all host cores (tests/_oracle_pool.py), once per batch, and serves both the fused
+step (pa_decode_append, the call bench.py times) and the unfused one (pa_reshape_and_cache
++ pa_decode).  The pools after the fused step are compared bit for bit with the oracle's
+pools after copy_blocks and reshape_and_cache.
+"""
 
 import numpy as np
 import pytest
 import torch
 
 import workloads
-from _parity import assert_close, gpu_step, oracle_step
+from _oracle_pool import decode_all_rows
+from _parity import assert_close, gpu_step, oracle_bits, pool_bits
+from oracle import RefAllocator, ref_copy_blocks, ref_reshape_and_cache
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
 FULL = {
-    "gqa": (workloads.gqa, [0, 1, 77, 128, 255]),
-    "mha": (workloads.mha, [0, 31, 63]),
-    "long": (workloads.long_context, [0, 5]),
-    "prefix": (workloads.prefix, [0, 9, 255]),
-    "prefix_cow": (workloads.prefix_cow, [0, 7, 8, 250]),
+    "gqa": workloads.gqa,
+    "mha": workloads.mha,
+    "long": workloads.long_context,
+    "prefix": workloads.prefix,
+    "prefix_cow": workloads.prefix_cow,
 }
 
 
-@pytest.mark.parametrize("fused", [True, False])
+def _oracle_every_row(w):
+    """The oracle side of one workload step, with the decode over every row on all cores."""
+    alloc = RefAllocator(w.num_blocks, w.block_size, shuffle_seed=w.alloc_seed, pop_order=w.pop_order)
+    setup_pairs = workloads.run_setup(w, alloc)
+    slots, pairs, tables, lens = workloads.run_step_allocation(w, alloc)
+    kp, vp = ref_copy_blocks(w.k_pool(), w.v_pool(), setup_pairs)
+    kp, vp = ref_copy_blocks(kp, vp, [tuple(p) for p in pairs])
+    kp, vp = ref_reshape_and_cache(w.new_k(), w.new_v(), kp, vp, slots)
+    out = decode_all_rows(w.q(), kp, vp, tables, lens, w.scale)
+    return {"out": out, "slots": slots, "pairs": pairs, "tables": tables, "lens": lens,
+            "k_pool": kp, "v_pool": vp}
+
+
 @pytest.mark.parametrize("name", sorted(FULL))
-def test_full_size_sampled_rows(name, fused):
-    """fused: pa_decode_append, the call bench.py times; else reshape_and_cache + pa_decode."""
-    build, rows = FULL[name]
-    w = build()
-    g = gpu_step(w, fused=fused, keep=fused)
-    assert g["err"] == 0
-    if fused:
-        # every row's new K/V sits in the slot the allocator reserved for it
-        slots = torch.from_numpy(g["slots"]).cuda()
-        for pool, new in ((g["k_pool"], g["nk"]), (g["v_pool"], g["nv"])):
-            rows_at = pool.view(-1, w.Hkv, w.D)[slots]
-            assert torch.equal(rows_at, new)
-    out = g["out"].float()
-    assert torch.isfinite(out).all()
-    # |o| <= max |v| for a convex combination: a property of every row
-    assert float(out.abs().max()) <= 6.0
-    r = oracle_step(w, rows=rows)
-    np.testing.assert_array_equal(g["slots"], r["slots"])
-    np.testing.assert_array_equal(g["pairs"], r["pairs"])
-    np.testing.assert_array_equal(g["tables"], r["tables"])
-    assert_close(w, g["out"][torch.as_tensor(rows)], r["out"])
+def test_full_size_every_row(name):
+    w = FULL[name]()
+    r = _oracle_every_row(w)
+    for fused in (True, False):
+        g = gpu_step(w, fused=fused, keep=fused)
+        assert g["err"] == 0
+        np.testing.assert_array_equal(g["slots"], r["slots"])
+        np.testing.assert_array_equal(g["pairs"], r["pairs"])
+        np.testing.assert_array_equal(g["tables"], r["tables"])
+        np.testing.assert_array_equal(g["lens"], r["lens"])
+        assert_close(w, g["out"], r["out"])
+        if fused:
+            # the decode kernel wrote every row's new K/V into its slot, and nothing else
+            for pool, ref in ((g["k_pool"], r["k_pool"]), (g["v_pool"], r["v_pool"])):
+                assert np.array_equal(pool_bits(pool), oracle_bits(ref, w))
+        del g
+        torch.cuda.empty_cache()

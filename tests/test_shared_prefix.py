@@ -84,7 +84,7 @@ def test_shared_prefix_matches_oracle_and_pa_decode(name):
         assert ng > 0
     r = oracle_step(w)
     assert_close(w, out, r["out"])
-    assert_close(w, out, g["out"].float().cpu().numpy())
+    assert_close(w, out, g["out"].float().cpu().numpy(), exact_ref=False)
 
 
 @pytest.mark.gpu

@@ -3,9 +3,9 @@
 It serves callers that cannot allocate device memory (a runtime that owns every
 device buffer through its own pool, or a caller that cannot afford cudaMalloc),
 so it takes no workspace and uses the library's static device scratch instead.
-Its output must match pa_decode's (same inputs, workspace supplied) within the
-parity tolerance, on two calls in a row with different batches, so that
-whatever the first call left in the shared scratch cannot leak into the second.
+Its output must match the float64 oracle's and pa_decode's (same inputs, workspace
+supplied) within the parity tolerance, on two calls in a row with different batches, so
+that whatever the first call left in the shared scratch cannot leak into the second.
 
 This file is collected last on purpose: it runs after every other test in a
 full session, and must also pass alone in a fresh process.
@@ -17,15 +17,21 @@ import torch
 
 import workloads
 from _parity import assert_close, to_device
+from oracle import ref_decode
 
 pytestmark = pytest.mark.gpu
 
 
-def _inputs(w):
+def _host_tables(w):
     import paged_kv_cache_350_b200 as pa
     alloc = pa.Allocator(w.num_blocks, w.block_size, shuffle_seed=w.alloc_seed, pop_order=w.pop_order)
     workloads.run_setup(w, alloc)
     _, _, tables, lens = workloads.run_step_allocation(w, alloc)
+    return tables, lens
+
+
+def _inputs(w):
+    tables, lens = _host_tables(w)
     return (to_device(w.q(), w), to_device(w.k_pool(), w), to_device(w.v_pool(), w),
             torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda())
 
@@ -40,7 +46,7 @@ def _reference(w, q, kp, vp, tables, lens):
     return out
 
 
-def test_no_alloc_matches_pa_decode_on_two_calls_in_a_row():
+def test_no_alloc_matches_oracle_and_pa_decode_on_two_calls_in_a_row():
     import paged_kv_cache_350_b200 as pa
     cases = [workloads.gqa(B=40, median=300, lo=1, hi=1200, seed=5100),
              workloads.long_context(B=3, lo=2000, hi=9000, Hq=32, seed=5101)]
@@ -53,7 +59,9 @@ def test_no_alloc_matches_pa_decode_on_two_calls_in_a_row():
         torch.cuda.synchronize()
         assert int(err.item()) == 0
         assert torch.isfinite(out.float()).all()
-        assert_close(w, out, ref.float().cpu().numpy())
+        tables, lens = _host_tables(w)
+        assert_close(w, out, ref_decode(w.q(), w.k_pool(), w.v_pool(), tables, lens, w.scale))
+        assert_close(w, out, ref.float().cpu().numpy(), exact_ref=False)
 
 
 def test_no_alloc_rejects_what_it_does_not_take():
