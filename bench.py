@@ -80,6 +80,9 @@ def parse_args(argv=None):
                     help="decode with pa_decode_shared_prefix (fork groups read shared blocks once)")
     ap.add_argument("--block-size", type=int, default=0,
                     help="override the workload's block size (8, 16 or 32) for a sweep")
+    ap.add_argument("--long", type=int, default=1,
+                    help="with the gqa config, also time the long-context batch in the same run "
+                         "(reported under \"long\"; 0: off)")
     ap.add_argument("--unfused", action="store_true",
                     help="pa_reshape_and_cache + pa_decode as two calls (default: pa_decode_append)")
     return ap.parse_args(argv)
@@ -395,19 +398,11 @@ def to_device(arr, w, device):
     return torch.from_numpy(np.ascontiguousarray(arr)).to(device)
 
 
-def run_ours(args):
+def prepare(args, pa, device, config, block_size=0):
+    """Inputs of one config resident on the device, and the step closure that runs the hot
+    path over them (the allocator's output for the step computed on the host first)."""
     import torch
-    rank, local_rank, world = dist_env()
-    device = torch.device("cuda", local_rank)
-    torch.cuda.set_device(device)
-    dist = init_dist(world, local_rank)
-    if rank == 0:
-        from paged_kv_cache_350_b200.build import build
-        build()
-    barrier(dist, device)
-    import paged_kv_cache_350_b200 as pa
-
-    w = workloads.build(args.config, **({"bs": args.block_size} if args.block_size else {}))
+    w = workloads.build(config, **({"bs": block_size} if block_size else {}))
     esize = 2 if w.dtype == "bf16" else 4
     dtype_pa = pa.PA_BF16 if w.dtype == "bf16" else pa.PA_F32
 
@@ -440,13 +435,14 @@ def run_ours(args):
     append_launch = 1 if (not fused or plan["kernel"] != pa.binding.PA_KERNEL_TC_STREAM) else 0
     launches_per_step = plan["launches"] + append_launch + (1 if npairs else 0)
     unique_kv = None
+    sp = None
     if args.shared_prefix:
         maxm = max(1, 16 // (w.Hq // w.Hkv))
         gof, gpre, gmem = alloc.prefix_groups(w.step_seqs, maxm, pa.binding.PA_SHARED_PREFIX_ALIGN)
         ng = len(gpre)
-        gof_d = torch.from_numpy(np.ascontiguousarray(gof)).to(device)
-        gpre_d = torch.from_numpy(np.ascontiguousarray(gpre) if ng else np.zeros(1, np.int32)).to(device)
-        gmem_d = torch.from_numpy(np.ascontiguousarray(gmem).reshape(ng, maxm)).to(device)
+        sp = {"gof": torch.from_numpy(np.ascontiguousarray(gof)).to(device),
+              "gpre": torch.from_numpy(np.ascontiguousarray(gpre) if ng else np.zeros(1, np.int32)).to(device),
+              "gmem": torch.from_numpy(np.ascontiguousarray(gmem).reshape(ng, maxm)).to(device)}
         nws = pa.pa_decode_shared_prefix_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.block_size, ng)
         ws = torch.empty(max(nws, 1), dtype=torch.uint8, device=device)
         pre_of = np.where(gof >= 0, np.asarray(gpre, dtype=np.int64)[np.maximum(gof, 0)] if ng else 0, 0)
@@ -470,21 +466,40 @@ def run_ours(args):
         if ev is not None:
             ev[0].record(stream)
         if args.shared_prefix:
-            pa.pa_decode_shared_prefix(out, q, kp, vp, tables_d, lens_d, w.scale, gof_d, gpre_d,
-                                       gmem_d, ws, err_flag=err, stream=stream)
+            pa.pa_decode_shared_prefix(out, q, kp, vp, tables_d, lens_d, w.scale, sp["gof"],
+                                       sp["gpre"], sp["gmem"], ws, err_flag=err, stream=stream)
         else:
             pa.pa_decode(out, q, kp, vp, tables_d, lens_d, w.scale, workspace=ws, err_flag=err,
                          stream=stream)
         if ev is not None:
             ev[1].record(stream)
 
-    for _ in range(args.warmup):
+    alg_bytes, kv_bytes = decode_bytes(lens, w.B, w.Hq, w.Hkv, w.D, w.block_size, esize)
+    # bytes that must cross HBM: with shared prefixes, each group's shared tokens once
+    roof_bytes = alg_bytes if unique_kv is None else alg_bytes - kv_bytes + unique_kv
+    # the fused call also writes each row's new K/V to its slot (its read replaces the
+    # read of that slot, already counted in the decode bytes)
+    append_bytes = 2 * w.B * w.Hkv * w.D * esize if fused else 0
+    roof_bytes += append_bytes
+    return {"w": w, "config": config, "esize": esize, "alloc": alloc, "slots": slots,
+            "pairs": pairs, "tables": tables, "lens": lens, "MB": MB, "kp": kp, "vp": vp,
+            "q": q, "nk": nk, "nv": nv, "err": err, "plan": plan, "npairs": npairs,
+            "stream": stream, "fused": fused, "launches_per_step": launches_per_step,
+            "unique_kv": unique_kv, "step": step, "alg_bytes": alg_bytes, "kv_bytes": kv_bytes,
+            "roof_bytes": roof_bytes, "append_bytes": append_bytes}
+
+
+def time_steps(st, K, W, dist, device):
+    """W untimed steps, then K steps bracketed by a barrier and a synchronize on both sides,
+    timed with CUDA events on the launching stream (whole region, and each decode call);
+    the clocks are sampled during the timed region.  Times are the max over ranks."""
+    import torch
+    step, err, stream = st["step"], st["err"], st["stream"]
+    for _ in range(W):
         step()
     torch.cuda.synchronize()
     if int(err.item()) != 0:
         raise RuntimeError(f"device error flag {int(err.item())} during warm-up")
-
-    K = args.steps
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(device.index)
@@ -499,22 +514,53 @@ def run_ours(args):
     clocks.stop()
     barrier(dist, device)
     elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), dist, device)
-    dec_ms = [a.elapsed_time(b) for a, b in evs]
-    dec_avg_ms = max_over_ranks(statistics.fmean(dec_ms), dist, device)
+    dec_avg_ms = max_over_ranks(statistics.fmean(a.elapsed_time(b) for a, b in evs), dist, device)
     if int(err.item()) != 0:
         raise RuntimeError(f"device error flag {int(err.item())} during timing")
+    return elapsed_ms, dec_avg_ms, clocks.summary()
 
-    alg_bytes, kv_bytes = decode_bytes(lens, w.B, w.Hq, w.Hkv, w.D, w.block_size, esize)
+
+def roofline(st, dec_avg_ms, config):
+    """The decode call of one step against the measured HBM copy bandwidth."""
+    peak, peak_src = measured_peak()
+    achieved = st["roof_bytes"] / (dec_avg_ms / 1e3) / 1e9
+    fused = st["fused"]
+    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak,
+            "traffic": recorded_traffic(config, "pa_decode_append" if fused else "pa_decode"),
+            "kernel": ("pa_decode_append call (decode kernel with the fused cache write + its "
+                       "reduce)" if fused else
+                       "pa_decode_shared_prefix call (main kernel + its cut reduce)"
+                       if st["unique_kv"] is not None else
+                       "pa_decode call (main kernel + its reduce)") + ", CUDA events per call",
+            "append_bytes_per_call": st["append_bytes"],
+            "peak_source": f"{peak_src} HBM copy bandwidth (burst)"}
+
+
+def run_ours(args):
+    import torch
+    rank, local_rank, world = dist_env()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    dist = init_dist(world, local_rank)
+    if rank == 0:
+        from paged_kv_cache_350_b200.build import build
+        build()
+    barrier(dist, device)
+    import paged_kv_cache_350_b200 as pa
+
+    st = prepare(args, pa, device, args.config, args.block_size)
+    w, esize, alloc = st["w"], st["esize"], st["alloc"]
+    tables, lens, MB = st["tables"], st["lens"], st["MB"]
+    kp, vp, q, nk, nv = st["kp"], st["vp"], st["q"], st["nk"], st["nv"]
+    plan, npairs, stream, fused = st["plan"], st["npairs"], st["stream"], st["fused"]
+    unique_kv, alg_bytes, kv_bytes = st["unique_kv"], st["alg_bytes"], st["kv_bytes"]
+
+    K = args.steps
+    elapsed_ms, dec_avg_ms, clock_summary = time_steps(st, K, args.warmup, dist, device)
     value = alg_bytes * K * world / (elapsed_ms / 1e3) / 1e9
     tokens_per_s = w.B * K * world / (elapsed_ms / 1e3)
-    peak, peak_src = measured_peak()
-    # bytes that must cross HBM: with shared prefixes, each group's shared tokens once
-    roof_bytes = alg_bytes if unique_kv is None else alg_bytes - kv_bytes + unique_kv
-    # the fused call also writes each row's new K/V to its slot (its read replaces the
-    # read of that slot, already counted in the decode bytes)
-    append_bytes = 2 * w.B * w.Hkv * w.D * esize if fused else 0
-    roof_bytes += append_bytes
-    achieved = roof_bytes / (dec_avg_ms / 1e3) / 1e9
+    roof = roofline(st, dec_avg_ms, args.config)
 
     # ---- end to end through the public API with host buffers -------------------------
     # PagedKVCache.pipeline: every step runs the C allocator, one host->device copy of the
@@ -567,6 +613,32 @@ def run_ours(args):
                              "device->host copy of the output (read two steps later); steps queued "
                              "back to back over three staging slots"}
 
+    # ---- the long-context batch, timed in the same run ---------------------------------
+    # The decode must hold its bandwidth on both serving shapes: the GQA batch above and
+    # long contexts (B=8, 32K-128K tokens), where every unit is split over many streams.
+    long_line = None
+    gpu_launches = st["launches_per_step"] * K
+    if args.config == "gqa" and args.long and not args.shared_prefix and not args.block_size:
+        sl = prepare(args, pa, device, "long")
+        l_ms, l_dec_ms, l_clocks = time_steps(sl, K, args.warmup, dist, device)
+        wl = sl["w"]
+        long_line = {
+            "workload": CONFIG_TEXT["long"], "name": "long", "B": wl.B, "Hq": wl.Hq,
+            "Hkv": wl.Hkv, "head_dim": wl.D, "block_size": wl.block_size,
+            "mean_seq_len": float(np.mean(sl["lens"])), "steps": K, "warmup": args.warmup,
+            "value": sl["alg_bytes"] * K * world / (l_ms / 1e3) / 1e9, "unit": UNIT,
+            "ms_per_step": l_ms / K,
+            "decode_tokens_per_s": wl.B * K * world / (l_ms / 1e3),
+            "alg_bytes_per_step": sl["alg_bytes"], "decode_plan": sl["plan"],
+            "step_calls": "pa_decode_append" if sl["fused"] else "pa_reshape_and_cache + pa_decode",
+            "roofline": roofline(sl, l_dec_ms, "long"),
+            "clocks": l_clocks,
+            "l2": "inputs larger than L2 (K/V pools of %.2f GB vs 126 MB L2); not flushed"
+                  % (2 * sl["kp"].numel() * sl["esize"] / 1e9),
+        }
+        gpu_launches += sl["launches_per_step"] * K
+        del sl
+
     # ---- CPU oracle baseline (rank 0, one GPU only) --------------------------------
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -575,8 +647,8 @@ def run_ours(args):
         if args.cpu_all_cores:
             try:
                 need = 2 * w.k_pool().nbytes + w.q().nbytes
-                st = os.statvfs("/dev/shm")
-                if st.f_bavail * st.f_frsize < 1.2 * need:
+                fs = os.statvfs("/dev/shm")
+                if fs.f_bavail * fs.f_frsize < 1.2 * need:
                     raise RuntimeError(f"/dev/shm has less than {1.2 * need / 1e9:.1f} GB free")
                 rate_n, procs, desc_n = oracle_rate_all_cores(w, tables, lens, args.cpu_seconds / 2)
                 cpu["all_cores"] = {"value": rate_n, "unit": UNIT, "cores": procs, "sample": desc_n}
@@ -610,20 +682,14 @@ def run_ours(args):
         },
         "decode_tokens_per_s": tokens_per_s,
         "kernel_kv_gbs": alg_bytes / (dec_avg_ms / 1e3) / 1e9,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak,
-                     "traffic": recorded_traffic(args.config, "pa_decode_append" if fused
-                                                 else "pa_decode"),
-                     "kernel": ("pa_decode_append call (decode kernel with the fused cache "
-                                "write + its reduce)" if fused else "pa_decode call (main kernel "
-                                "+ its reduce)") + ", CUDA events per call",
-                     "append_bytes_per_call": append_bytes,
-                     "peak_source": f"{peak_src} HBM copy bandwidth (burst)"},
+        "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": launches_per_step * K,
-        "clocks": clocks.summary(),
+        "gpu_launches": gpu_launches,
+        "clocks": clock_summary,
     }
+    if long_line is not None:
+        line["long"] = long_line
     print(json.dumps(line), flush=True)
     return 0
 

@@ -236,9 +236,15 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_pool,
  * tensor-core kernel with its scratch in a static device array of the library
  * (PA_NO_ALLOC_SCRATCH_BYTES per device that loads the library, held until exit); it
  * calls no cudaMalloc, cudaFree or allocating library routine.
+ *   - The array is device memory reserved when the library's module loads on a device:
+ *     at context creation under CUDA_MODULE_LOADING=EAGER (then even by processes that
+ *     never call this function), or inside the first call under lazy loading (the
+ *     default).
  *   - The first call on each device looks up the array's address (cudaGetSymbolAddress
- *     with that device current) and caches it: make that first call before any stream
- *     capture.
+ *     with that device current) and caches it for the current context; a new context on
+ *     the device (e.g. after cudaDeviceReset) is detected and the address looked up
+ *     again.  Make that first call before any stream capture, so that neither the module
+ *     load nor the lookup happens inside one.
  *   - All calls on a device share the array, which keeps the last call's contents;
  *     nothing in it has to start at zero.  Calls whose kernels overlap on the GPU race
  *     on the array: order them (e.g. one stream).

@@ -12,9 +12,14 @@
 // Properties:
 //   * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.  The
 //     scratch array exists once per device that loads the library, until exit.
+//   * The array is device memory of the library's module: it is reserved when the module
+//     loads, at context creation under CUDA_MODULE_LOADING=EAGER, or in the first call
+//     on the device under lazy loading (the default).
 //   * The first call on each device looks up the array's device address with
-//     cudaGetSymbolAddress (with that device current) and caches it; make that first
-//     call before any stream capture.
+//     cudaGetSymbolAddress (with that device current) and caches it for the current
+//     context (looked up again if the context changes, e.g. after cudaDeviceReset); make
+//     that first call before any stream capture, so that neither the module load nor
+//     the lookup happens inside one.
 //   * Every call on a device uses the same array and leaves its contents behind.  The
 //     stream kernel writes every metadata slot and partial it later reads within the
 //     same call, so nothing has to start at zero.  Two calls whose kernels overlap on
@@ -23,6 +28,8 @@
 //   * A shape whose one-wave schedule needs more than kScratchBytes is rejected with
 //     PA_ERR_SCRATCH_LIMIT before anything is queued; shapes the stream kernel does not
 //     take (fp32, block size 4, G > 16, B > 8192) get PA_ERR_UNSUPPORTED.
+
+#include <cuda.h>
 
 #include <cmath>
 #include <mutex>
@@ -39,20 +46,55 @@ constexpr int kStreamMaxB = 8192;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 std::mutex g_mu;
+// Per device: the context the address was looked up in, and the address.  A device reset
+// (cudaDeviceReset) destroys the device's primary context, and the array of the next
+// context on that device has another address, so a cached address holds only while the
+// current context is the one it came from.
+CUcontext g_ctx[kMaxDevices] = {};
 void* g_addr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (looked up once per device).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// cuCtxGetCurrent through the runtime's driver entry point (the library links only the
+// runtime); null if unavailable.
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+  });
+  return fn;
+}
+
+CUcontext current_context() {
+  CUcontext c = nullptr;
+  const CtxGetCurrentFn fn = ctx_get_current();
+  if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// Device address of the scratch array in the current context.  The first call on a
+// device (and the first after its context changed) looks it up with cudaGetSymbolAddress,
+// with that device current; later calls reuse it.  The lookup allocates nothing: the
+// array is part of the library's module, reserved when the module loads.
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_addr[dev]) {
+  CUcontext ctx = current_context();
+  if (!g_addr[dev] || !ctx || ctx != g_ctx[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
     if (!p) return cudaErrorInvalidSymbol;
+    // the lookup made the device's context current if none was
+    g_ctx[dev] = ctx ? ctx : current_context();
     g_addr[dev] = p;
   }
   *out = g_addr[dev];
