@@ -349,6 +349,10 @@ pa_status pa_alloc_block_table(const pa_allocator* a, int64_t seq_id, int32_t* o
 /* Fill block_tables[n][max_blocks] (padded with -1) and seq_lens[n] for n sequences. */
 pa_status pa_alloc_block_tables(const pa_allocator* a, const int64_t* seq_ids, int n,
                                 int32_t* block_tables, int max_blocks, int32_t* seq_lens);
+/* PA_OK if every listed sequence exists (else PA_ERR_NOT_FOUND) and its table would still
+ * fit max_blocks entries after one more token (else PA_ERR_INVALID_ARG).  Changes nothing. */
+pa_status pa_alloc_check_append_fits(const pa_allocator* a, const int64_t* seq_ids, int n,
+                                     int max_blocks);
 /* Slots of all tokens of a sequence, token t at
  * table[t / block_size] * block_size + t % block_size (up to cap); *n = its token count.
  * Used to write a prompt's K/V (prefill) with pa_reshape_and_cache. */
@@ -369,6 +373,72 @@ int pa_alloc_num_free(const pa_allocator* a);
 int64_t pa_alloc_internal_waste_slots(const pa_allocator* a);
 /* Free stack bottom-to-top into out (up to cap); returns its length. */
 int pa_alloc_free_list(const pa_allocator* a, int32_t* out, int cap);
+
+/* ---------------------------------------------------------------------------
+ * Decode-step pipeline: one call per step of a serving loop
+ *
+ * Each step: the allocator reserves every sequence's next slot (pa_alloc_append_slots;
+ * copy-on-write pairs for partial blocks still shared) and writes the padded tables and
+ * lengths (pa_alloc_block_tables) into a pinned host input slot behind the step's q / new
+ * K / new V, which the caller wrote there; one host->device copy moves the slot; then
+ * pa_copy_blocks (if the step has pairs) and pa_decode_append run, and the output is
+ * copied back to a pinned host output slot.  Copies run on their own streams and steps
+ * are queued back to back over `depth` slots, so the host prepares step t+1 and the copy
+ * engines move neighbouring steps' data while the GPU decodes step t ("深入解析
+ * PagedAttention", 核心创新: blocks are allocated on demand as each sequence grows;
+ * "什么是 LLM 中的分页注意力", 使用分页注意力: each new token fills the next slot of the
+ * sequence's current block).
+ *
+ * Ownership: every buffer and stream is the caller's; the pipeline creates only CUDA
+ * events (no device memory).  The allocator is borrowed: it must outlive the pipeline and
+ * not be used by another thread during a call.  Not thread-safe.
+ * ------------------------------------------------------------------------- */
+
+typedef struct pa_pipeline pa_pipeline;
+
+typedef struct pa_pipeline_desc {
+  int B, Hq, Hkv, D, block_size, max_blocks, num_blocks;  /* the batch shape, fixed */
+  pa_dtype dtype;
+  int depth;                  /* staging slots, 1 .. 64 */
+  void* k_pool;               /* device pools [num_blocks][block_size][Hkv][D] */
+  void* v_pool;
+  void* workspace;            /* device, pa_decode_workspace_size bytes (may be NULL) */
+  size_t workspace_bytes;
+  int32_t* dev_err_flag;      /* device, nullable */
+  void* const* host_in;       /* [depth] pinned host, pa_pipeline_input_bytes each */
+  void* const* dev_in;        /* [depth] device, pa_pipeline_input_bytes each, 256-B aligned */
+  void* const* host_out;      /* [depth] pinned host [B][Hq][D] */
+  void* const* dev_out;       /* [depth] device [B][Hq][D], 16-B aligned */
+  pa_stream_t compute;        /* kernels */
+  pa_stream_t copy_in;        /* host->device copies */
+  pa_stream_t copy_out;       /* device->host copies */
+} pa_pipeline_desc;
+
+/* Bytes of one input slot; offsets[6] (nullable) receives the byte offsets of its
+ * sections: q [B][Hq][D], k_new [B][Hkv][D], v_new [B][Hkv][D] (written by the caller),
+ * block_tables [B][max_blocks] int32, seq_lens [B] int32 and copy pairs [B][2] int32
+ * (written by the pipeline).  0 for invalid arguments. */
+size_t pa_pipeline_input_bytes(int B, int Hq, int Hkv, int D, int max_blocks, pa_dtype dtype,
+                               size_t* offsets);
+/* The descriptor's arrays are copied.  PA_ERR_INVALID_ARG for a bad descriptor. */
+pa_status pa_pipeline_create(pa_allocator* alloc, const pa_pipeline_desc* desc,
+                             pa_pipeline** out);
+/* Waits for every queued step, then frees the pipeline (not the caller's buffers). */
+void pa_pipeline_destroy(pa_pipeline* p);
+/* *slot = the input slot of the next step, once its previous host->device copy has
+ * finished: the caller then writes q, k_new and v_new there and calls submit. */
+pa_status pa_pipeline_next_slot(pa_pipeline* p, int* slot);
+/* Queue one step for seq_ids[B] (distinct live sequences; the batch order of q/k/v).
+ * *step (nullable) = its index (0, 1, ...), *h2d_bytes (nullable) = bytes copied in.
+ * Returns once the step is queued.  An allocator error (e.g. PA_ERR_OUT_OF_BLOCKS) leaves
+ * everything unchanged; after PA_ERR_CUDA the pipeline should be destroyed. */
+pa_status pa_pipeline_submit(pa_pipeline* p, const int64_t* seq_ids, float scale,
+                             int64_t* step, size_t* h2d_bytes);
+/* Waits for step's output copy; *slot = the host_out slot holding it, valid until step +
+ * depth is submitted.  PA_ERR_INVALID_ARG for a step not yet queued or no longer held. */
+pa_status pa_pipeline_result(pa_pipeline* p, int64_t step, int* slot);
+/* Waits for every queued step. */
+pa_status pa_pipeline_sync(pa_pipeline* p);
 
 #ifdef __cplusplus
 }

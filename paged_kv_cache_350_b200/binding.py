@@ -73,6 +73,21 @@ class pa_decode_plan_info(ctypes.Structure):
                 ("max_parts", ctypes.c_int), ("grid", ctypes.c_int), ("launches", ctypes.c_int)]
 
 
+class pa_pipeline_desc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+                ("D", ctypes.c_int), ("block_size", ctypes.c_int), ("max_blocks", ctypes.c_int),
+                ("num_blocks", ctypes.c_int), ("dtype", ctypes.c_int), ("depth", ctypes.c_int),
+                ("k_pool", ctypes.c_void_p), ("v_pool", ctypes.c_void_p),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+                ("dev_err_flag", ctypes.c_void_p),
+                ("host_in", ctypes.POINTER(ctypes.c_void_p)),
+                ("dev_in", ctypes.POINTER(ctypes.c_void_p)),
+                ("host_out", ctypes.POINTER(ctypes.c_void_p)),
+                ("dev_out", ctypes.POINTER(ctypes.c_void_p)),
+                ("compute", ctypes.c_void_p), ("copy_in", ctypes.c_void_p),
+                ("copy_out", ctypes.c_void_p)]
+
+
 def _load():
     if not os.path.exists(_LIB_PATH):
         raise ImportError(
@@ -123,6 +138,14 @@ def _load():
         "pa_alloc_num_free": (i32, [vp]),
         "pa_alloc_internal_waste_slots": (i64, [vp]),
         "pa_alloc_free_list": (i32, [vp, pi32, i32]),
+        "pa_alloc_check_append_fits": (i32, [vp, pi64, i32, i32]),
+        "pa_pipeline_input_bytes": (sz, [i32, i32, i32, i32, i32, i32, ctypes.POINTER(sz)]),
+        "pa_pipeline_create": (i32, [vp, ctypes.POINTER(pa_pipeline_desc), ctypes.POINTER(vp)]),
+        "pa_pipeline_destroy": (None, [vp]),
+        "pa_pipeline_next_slot": (i32, [vp, pint]),
+        "pa_pipeline_submit": (i32, [vp, pi64, f32, pi64, ctypes.POINTER(sz)]),
+        "pa_pipeline_result": (i32, [vp, i64, pint]),
+        "pa_pipeline_sync": (i32, [vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -144,7 +167,9 @@ EXPORTED = (
     "pa_alloc_append_slot", "pa_alloc_append_slots", "pa_alloc_free_seq", "pa_alloc_truncate",
     "pa_alloc_beam_select", "pa_alloc_block_table",
     "pa_alloc_block_tables", "pa_alloc_seq_slots", "pa_alloc_refcount", "pa_alloc_num_free",
-    "pa_alloc_internal_waste_slots", "pa_alloc_free_list",
+    "pa_alloc_internal_waste_slots", "pa_alloc_free_list", "pa_alloc_check_append_fits",
+    "pa_pipeline_input_bytes", "pa_pipeline_create", "pa_pipeline_destroy",
+    "pa_pipeline_next_slot", "pa_pipeline_submit", "pa_pipeline_result", "pa_pipeline_sync",
 )
 
 

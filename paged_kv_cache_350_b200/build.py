@@ -26,7 +26,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpagedattn.so")
 
 SOURCES = ["api.cu", "decode_tc.cu", "decode_stream.cu", "decode_generic.cu", "cache_ops.cu", "allocator.cpp",
-           "decode_noalloc.cu", "decode_prefix.cu", "selftest.cu"]
+           "decode_noalloc.cu", "decode_prefix.cu", "selftest.cu", "pipeline.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]
 

@@ -21,9 +21,10 @@ caller writes the step's q / new K / new V straight into the cache's pinned
 input buffer, the allocator writes slots, tables and lengths behind them, and a
 single copy moves the whole step input.
 
-``pipeline`` (``StepPipeline``) queues such steps back to back: double-buffered
-staging, the copies on their own streams, so the host and the copy engines work on
-neighbouring steps while the GPU decodes the current one.
+``pipeline`` (``StepPipeline``, the C ``pa_pipeline_*`` calls) queues such steps back to
+back, one C call per step: staging in several slots, the copies on their own streams, so
+the host and the copy engines work on neighbouring steps while the GPU decodes the
+current one.
 """
 
 from __future__ import annotations
@@ -236,18 +237,17 @@ class PagedKVCache:
 
 
 class StepPipeline:
-    """Decode steps of a fixed batch shape queued back to back, host and device overlapped.
+    """Decode steps of a fixed batch shape queued back to back: ``pa_pipeline_*`` (C).
 
     Each step is the same work as ``PagedKVCache.step_staged``: the allocator reserves a
     slot per sequence, one host->device copy moves the step's q / new K / new V, tables,
     lengths and copy pairs, ``pa_copy_blocks`` + ``pa_decode_append`` run, and the output
-    is copied back to pinned host memory.  Here the step input and output buffers come in
-    ``depth`` slots, the copies run on their own streams, and ``submit`` returns once the
-    step is queued.  So the host prepares step t+1 and the copy engines move its input
-    and step t-1's output while the GPU decodes step t.  Events order every reuse of a
-    slot: a host input buffer is rewritten only after its copy has finished, a device
-    input buffer only after the kernels that read it, a device output buffer only after
-    its copy to the host.
+    is copied back to pinned host memory.  The whole step is one C call
+    (``pa_pipeline_submit``), which returns once the step is queued.  The step input and
+    output buffers come in ``depth`` slots and the copies run on their own streams, so
+    the host prepares step t+1 and the copy engines move its input and step t-1's output
+    while the GPU decodes step t; events order every reuse of a slot.  This class owns
+    the buffers and streams (PyTorch memory) and marshals the calls.
 
         pipe = cache.pipeline(B, Hq, max_blocks)
         q, k, v = pipe.inputs()        # pinned views of the next step's input slot
@@ -259,106 +259,89 @@ class StepPipeline:
     """
 
     def __init__(self, cache, B, Hq, max_blocks, depth=2, stream=None):
+        import ctypes
         assert depth >= 1
         self.cache, self.B, self.Hq, self.max_blocks, self.depth = cache, B, Hq, max_blocks, depth
         self.dev = cache.device
         self.stream = stream or torch.cuda.current_stream(self.dev)
         self.copy_in = torch.cuda.Stream(self.dev)
         self.copy_out = torch.cuda.Stream(self.dev)
-        self.lay, total = cache._layout(B, Hq, max_blocks)
-        n_out = B * Hq * cache.D
+        D, Hkv, dt = cache.D, cache.Hkv, cache.dtype
+        pdt = _b.PA_BF16 if dt == torch.bfloat16 else _b.PA_F32
+        offs = (ctypes.c_size_t * 6)()
+        total = _b.lib.pa_pipeline_input_bytes(B, Hq, Hkv, D, max_blocks, pdt, offs)
+        if total == 0:
+            raise _b.PAError(_b.PA_ERR_INVALID_ARG, "pa_pipeline_input_bytes")
+        self.offsets = list(offs)
+        n_out = B * Hq * D
         self.h_in = [torch.empty(total, dtype=torch.uint8, pin_memory=True) for _ in range(depth)]
         self.d_in = [torch.empty(total, dtype=torch.uint8, device=self.dev) for _ in range(depth)]
-        self.h_out = [torch.empty(n_out, dtype=cache.dtype, pin_memory=True).view(B, Hq, cache.D)
+        self.h_out = [torch.empty(n_out, dtype=dt, pin_memory=True).view(B, Hq, D)
                       for _ in range(depth)]
-        self.d_out = [torch.empty(n_out, dtype=cache.dtype, device=self.dev).view(B, Hq, cache.D)
+        self.d_out = [torch.empty(n_out, dtype=dt, device=self.dev).view(B, Hq, D)
                       for _ in range(depth)]
-        ev = lambda: [torch.cuda.Event() for _ in range(depth)]  # noqa: E731
-        self.h2d_done, self.kern_done, self.d2h_done = ev(), ev(), ev()
-        self.used = [False] * depth   # slot has a step in flight (its events are recorded)
-        self.next = 0                 # index of the next step to submit
-        self.bytes_in = self.bytes_out = 0
         self.ws = cache.workspace(B, Hq, max_blocks)
-        # Per slot, built once (the per-step host work is the allocator and the queueing):
-        # the allocator's output views in the pinned input, the device views the kernels
-        # read, and the argument list of the pa_decode_append call.
-        D, Hkv, dt = cache.D, cache.Hkv, cache.dtype
-        self.h_views, self.d_pairs, self.decode_args = [], [], []
-        for k in range(depth):
-            h, d = self.h_in[k], self.d_in[k]
-            self.h_views.append((self._view(h, "slots", (B,), torch.int64).numpy(),
-                                 self._view(h, "pairs", (B, 2), torch.int32).numpy(),
-                                 self._view(h, "tables", (B, max_blocks), torch.int32).numpy(),
-                                 self._view(h, "lens", (B,), torch.int32).numpy()))
-            self.d_pairs.append(self._view(d, "pairs", (B, 2), torch.int32))
-            self.decode_args.append(_b.decode_append_args(
-                self.d_out[k], self._view(d, "q", (B, Hq, D), dt), self._view(d, "k", (B, Hkv, D), dt),
-                self._view(d, "v", (B, Hkv, D), dt), cache.k_pool, cache.v_pool,
-                self._view(d, "tables", (B, max_blocks), torch.int32),
-                self._view(d, "lens", (B,), torch.int32), workspace=self.ws, err_flag=cache.err,
-                stream=self.stream))
+        esz = self.h_out[0].element_size()
+        sec = [B * Hq * D * esz, B * Hkv * D * esz, B * Hkv * D * esz]
+        self._in_views = [tuple(h[o:o + n].view(dt).view(shape) for o, n, shape in
+                                zip(self.offsets[:3], sec, ((B, Hq, D), (B, Hkv, D), (B, Hkv, D))))
+                          for h in self.h_in]
+        arr = lambda ts: (ctypes.c_void_p * depth)(*[t.data_ptr() for t in ts])  # noqa: E731
+        self._arrays = (arr(self.h_in), arr(self.d_in), arr(self.h_out), arr(self.d_out))
+        desc = _b.pa_pipeline_desc(
+            B, Hq, Hkv, D, cache.block_size, max_blocks, cache.k_pool.shape[0], pdt, depth,
+            cache.k_pool.data_ptr(), cache.v_pool.data_ptr(),
+            self.ws.data_ptr() if self.ws is not None else None,
+            self.ws.numel() if self.ws is not None else 0, cache.err.data_ptr(), *self._arrays,
+            self.stream.cuda_stream, self.copy_in.cuda_stream, self.copy_out.cuda_stream)
+        h = ctypes.c_void_p()
+        _b._check(_b.lib.pa_pipeline_create(cache.alloc._h, ctypes.byref(desc), ctypes.byref(h)),
+                  "pa_pipeline_create")
+        self._h = h
+        self._slot = ctypes.c_int()
+        self._step = ctypes.c_int64()
+        self._h2d = ctypes.c_size_t()
+        self.next = 0
+        self.bytes_in = 0
+        self.bytes_out = n_out * esz
 
-    def _view(self, buf, name, shape, dtype):
-        off, n = self.lay[name]
-        return buf[off:off + n].view(dtype).view(shape)
+    def close(self):
+        if getattr(self, "_h", None):
+            _b.lib.pa_pipeline_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
     def inputs(self):
         """Pinned host (q, k, v) of the next step's slot, once its previous copy is done."""
-        k = self.next % self.depth
-        if self.used[k]:
-            self.h2d_done[k].synchronize()
-        c, h = self.cache, self.h_in[k]
-        return (self._view(h, "q", (self.B, self.Hq, c.D), c.dtype),
-                self._view(h, "k", (self.B, c.Hkv, c.D), c.dtype),
-                self._view(h, "v", (self.B, c.Hkv, c.D), c.dtype))
+        import ctypes
+        _b._check(_b.lib.pa_pipeline_next_slot(self._h, ctypes.byref(self._slot)),
+                  "pa_pipeline_next_slot")
+        return self._in_views[self._slot.value]
 
     def submit(self, seq_ids, scale):
         """Queue one decode step for seq_ids (the inputs() of this step must be written)."""
-        c, B = self.cache, self.B
+        import ctypes
         ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
-        assert ids.size == B, "the batch shape is fixed per pipeline"
-        t, k = self.next, self.next % self.depth
-        h, d = self.h_in[k], self.d_in[k]
-        slots_h, pairs_h, tables_h, lens_h = self.h_views[k]
-        if self.used[k]:
-            self.h2d_done[k].synchronize()   # normally long done: the copy of step t - depth
-        _, pairs = c.alloc.append_slots(ids, slot_out=slots_h, pairs_out=pairs_h)
-        c.alloc.block_tables(ids, self.max_blocks, tables_out=tables_h, lens_out=lens_h)
-        npairs = pairs.shape[0]
-        used = self.lay["pairs"][0] + npairs * 8 if npairs else self.lay["lens"][0] + B * 4
-        if self.used[k]:
-            self.copy_in.wait_event(self.kern_done[k])     # step t - depth has read d_in[k]
-        with torch.cuda.stream(self.copy_in):
-            d[:used].copy_(h[:used], non_blocking=True)
-        self.h2d_done[k].record(self.copy_in)
-        s = self.stream
-        s.wait_event(self.h2d_done[k])
-        if self.used[k]:
-            s.wait_event(self.d2h_done[k])                 # d_out[k] was copied out
-        if npairs:
-            _b.pa_copy_blocks(c.k_pool, c.v_pool, self.d_pairs[k][:npairs], err_flag=c.err,
-                              stream=s)
-        _b.decode_append_call(self.decode_args[k], scale)
-        self.kern_done[k].record(s)
-        self.copy_out.wait_event(self.kern_done[k])
-        with torch.cuda.stream(self.copy_out):
-            self.h_out[k].copy_(self.d_out[k], non_blocking=True)
-        self.d2h_done[k].record(self.copy_out)
-        self.used[k] = True
-        self.bytes_in = used
-        self.bytes_out = self.h_out[k].numel() * self.h_out[k].element_size()
-        self.next = t + 1
-        return t
+        assert ids.size == self.B, "the batch shape is fixed per pipeline"
+        _b._check(_b.lib.pa_pipeline_submit(self._h, _b._i64p(ids), float(scale),
+                                            ctypes.byref(self._step), ctypes.byref(self._h2d)),
+                  "pa_pipeline_submit")
+        self.bytes_in = self._h2d.value
+        self.next = self._step.value + 1
+        return self._step.value
 
     def result(self, t):
         """Pinned host output [B, Hq, D] of step t (waits for its copy)."""
-        assert self.next - self.depth <= t < self.next, "step no longer (or not yet) held"
-        k = t % self.depth
-        self.d2h_done[k].synchronize()
-        return self.h_out[k]
+        import ctypes
+        _b._check(_b.lib.pa_pipeline_result(self._h, int(t), ctypes.byref(self._slot)),
+                  "pa_pipeline_result")
+        return self.h_out[self._slot.value]
 
     def sync(self):
         """Wait for every queued step."""
-        for k in range(self.depth):
-            if self.used[k]:
-                self.d2h_done[k].synchronize()
+        _b._check(_b.lib.pa_pipeline_sync(self._h), "pa_pipeline_sync")

@@ -442,6 +442,21 @@ pa_status pa_alloc_block_tables(const pa_allocator* a, const int64_t* seq_ids, i
   });
 }
 
+// Whether every listed sequence exists and still has a table of at most max_blocks entries
+// after one more token (the decode-step pipeline checks this before it appends, so that a
+// step it cannot describe changes no state).
+pa_status pa_alloc_check_append_fits(const pa_allocator* a, const int64_t* seq_ids, int n,
+                                     int max_blocks) {
+  if (!a || n < 0 || max_blocks <= 0 || (n > 0 && !seq_ids)) return PA_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    auto it = a->seqs.find(seq_ids[i]);
+    if (it == a->seqs.end()) return PA_ERR_NOT_FOUND;
+    const int64_t blocks = (it->second.ntok + 1 + a->block_size - 1) / a->block_size;
+    if (blocks > max_blocks) return PA_ERR_INVALID_ARG;
+  }
+  return PA_OK;
+}
+
 pa_status pa_alloc_seq_slots(const pa_allocator* a, int64_t seq_id, int64_t* slots, int cap,
                              int* n) {
   if (!a || !n || cap < 0 || (cap > 0 && !slots)) return PA_ERR_INVALID_ARG;

@@ -162,7 +162,8 @@ def test_shared_prefix_argument_errors_are_reported_before_any_launch():
     assert _call_shared_prefix(maxm=0) == b.PA_ERR_INVALID_ARG
     assert _call_shared_prefix(ng=-1) == b.PA_ERR_INVALID_ARG
     assert _call_shared_prefix(scale=float("inf")) == b.PA_ERR_INVALID_ARG
-    assert _call_shared_prefix(maxm=5) == b.PA_ERR_UNSUPPORTED    # 5 members x 4 heads > 16 rows
+    assert _call_shared_prefix(maxm=17) == b.PA_ERR_UNSUPPORTED   # 17 members x 4 heads > 64 rows
+    assert _call_shared_prefix(maxm=33, Hq=4, Hkv=4) == b.PA_ERR_UNSUPPORTED  # > 32 members
     assert _call_shared_prefix(dtype=b.PA_F32) == b.PA_ERR_UNSUPPORTED
     assert _call_shared_prefix(D=96) == b.PA_ERR_UNSUPPORTED
     assert _call_shared_prefix(B=8000, ng=500) == b.PA_ERR_UNSUPPORTED  # more rows than the kernel takes
@@ -233,3 +234,42 @@ def test_header_compiles_as_c_and_the_allocator_runs_from_plain_c(tmp_path):
                     "-L", libdir, "-lpagedattn", f"-Wl,-rpath,{libdir}", "-o", exe], check=True)
     r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0 and r.stdout.strip() == "ok", r.stdout + r.stderr
+
+
+def test_pipeline_layout_and_argument_errors_before_any_cuda_call():
+    """pa_pipeline_*: the input-slot layout, descriptors rejected on the host, and the
+    allocator check that keeps a step that cannot be described from changing state."""
+    from paged_kv_cache_350_b200 import binding as b
+    import numpy as np
+    offs = (ctypes.c_size_t * 6)()
+    total = b.lib.pa_pipeline_input_bytes(3, 8, 2, 128, 5, b.PA_BF16, offs)
+    sizes = [3 * 8 * 128 * 2, 3 * 2 * 128 * 2, 3 * 2 * 128 * 2, 3 * 5 * 4, 3 * 4, 3 * 8]
+    up = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    assert list(offs) == [sum(up(s) for s in sizes[:i]) for i in range(6)]
+    assert total == sum(up(s) for s in sizes)
+    assert b.lib.pa_pipeline_input_bytes(0, 8, 2, 128, 5, b.PA_BF16, None) == 0
+    assert b.lib.pa_pipeline_input_bytes(3, 8, 2, 128, 5, 7, None) == 0
+
+    a = b.Allocator(8, 4)
+    h = ctypes.c_void_p()
+    desc = b.pa_pipeline_desc()  # all zero: B = 0, no buffers
+    assert b.lib.pa_pipeline_create(a._h, ctypes.byref(desc), ctypes.byref(h)) == b.PA_ERR_INVALID_ARG
+    assert not h.value
+    assert b.lib.pa_pipeline_create(None, ctypes.byref(desc), ctypes.byref(h)) == b.PA_ERR_INVALID_ARG
+    slot = ctypes.c_int()
+    assert b.lib.pa_pipeline_next_slot(None, ctypes.byref(slot)) == b.PA_ERR_INVALID_ARG
+    assert b.lib.pa_pipeline_result(None, 0, ctypes.byref(slot)) == b.PA_ERR_INVALID_ARG
+    assert b.lib.pa_pipeline_sync(None) == b.PA_ERR_INVALID_ARG
+    b.lib.pa_pipeline_destroy(None)
+
+    # the append check: sequence 1 holds 8 tokens = 2 full blocks of 4
+    a.add_seq(0, 3)
+    a.add_seq(1, 8)
+    ids = np.array([0, 1], dtype=np.int64)
+    chk = lambda i, mb: b.lib.pa_alloc_check_append_fits(a._h, b._i64p(i), i.size, mb)  # noqa: E731
+    assert chk(ids, 3) == b.PA_OK
+    assert chk(ids, 2) == b.PA_ERR_INVALID_ARG           # token 9 needs a third block
+    assert chk(np.array([0], dtype=np.int64), 1) == b.PA_OK
+    assert chk(np.array([5], dtype=np.int64), 3) == b.PA_ERR_NOT_FOUND
+    free = a.num_free()
+    assert free == 8 - 1 - 2 and a.block_table(1)[1] == 8   # the checks changed nothing
