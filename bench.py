@@ -437,7 +437,7 @@ def prepare(args, pa, device, config, block_size=0):
     unique_kv = None
     sp = None
     if args.shared_prefix:
-        maxm = max(1, 16 // (w.Hq // w.Hkv))
+        maxm = max(1, min(32, 64 // (w.Hq // w.Hkv)))
         gof, gpre, gmem = alloc.prefix_groups(w.step_seqs, maxm, pa.binding.PA_SHARED_PREFIX_ALIGN)
         ng = len(gpre)
         sp = {"gof": torch.from_numpy(np.ascontiguousarray(gof)).to(device),
@@ -563,11 +563,12 @@ def run_ours(args):
     roof = roofline(st, dec_avg_ms, args.config)
 
     # ---- end to end through the public API with host buffers -------------------------
-    # PagedKVCache.pipeline: every step runs the C allocator, one host->device copy of the
-    # step input (q, new K/V, tables, lengths, copy pairs), pa_copy_blocks +
-    # pa_decode_append and a device->host copy of the output; steps are queued back to
-    # back over three staging slots, and each step's output is read two steps later (so
-    # the host and the copies of neighbouring steps stay off the GPU's critical path).
+    # PagedKVCache.pipeline: every step is one C call (pa_pipeline_submit) that runs the
+    # allocator, one host->device copy of the step input (q, new K/V, tables, lengths, copy
+    # pairs), pa_copy_blocks + pa_decode_append and a device->host copy of the output; steps
+    # are queued back to back over three staging slots, and each step's output is read two
+    # steps later (so the host and the copies of neighbouring steps stay off the GPU's
+    # critical path).
     e2e = None
     if not args.no_e2e and args.e2e_steps > 0 and not args.shared_prefix:
         cache = pa.PagedKVCache(w.num_blocks, w.block_size, w.Hkv, w.D, dtype=kp.dtype, device=device,
@@ -579,6 +580,7 @@ def run_ours(args):
         ids = np.asarray(w.step_seqs, dtype=np.int64)
         warm = max(2, pipe.depth)
         nbytes = []
+        host_s = []
         cur = lens.astype(np.int64).copy()
         t0 = None
         done = 0
@@ -591,7 +593,10 @@ def run_ours(args):
                 barrier(dist, device)
                 t0 = time.perf_counter()
             try:
+                h0 = time.perf_counter()
                 pipe.submit(ids, w.scale)
+                if i >= warm:
+                    host_s.append(time.perf_counter() - h0)
             except pa.PAError:  # the pool ran out of blocks for more appends
                 break
             if i >= lag:
@@ -608,10 +613,12 @@ def run_ours(args):
             e2e = {"value": sum(nbytes) * world / dt / 1e9, "unit": UNIT,
                    "h2d_bytes_per_step": int(pipe.bytes_in), "d2h_bytes_per_step": int(pipe.bytes_out),
                    "ms_per_step": 1e3 * dt / done, "steps": done,
-                   "timing": "host perf_counter over the steps of PagedKVCache.pipeline: per step the C "
-                             "allocator, one host->device copy of the step input, kernels, a "
-                             "device->host copy of the output (read two steps later); steps queued "
-                             "back to back over three staging slots"}
+                   "host_us_per_submit": 1e6 * statistics.median(host_s) if host_s else None,
+                   "timing": "host perf_counter over the steps of PagedKVCache.pipeline: per step "
+                             "one C call (pa_pipeline_submit: the allocator, one host->device copy "
+                             "of the step input, the kernels, a device->host copy of the output, "
+                             "read two steps later); steps queued back to back over three staging "
+                             "slots"}
 
     # ---- the long-context batch, timed in the same run ---------------------------------
     # The decode must hold its bandwidth on both serving shapes: the GQA batch above and

@@ -202,8 +202,9 @@ pa_status pa_decode_append(void* out, const void* q, const void* k_new, const vo
  * forked from one prompt, or requests with a common system prompt ("深入解析 PagedAttention",
  * 多序列共享; "什么是 LLM 中的分页注意力", 跨请求的内存共享).  Same result as pa_decode, but each
  * group's shared tokens are read from HBM once for the whole group: the members' query heads
- * are stacked as one tile (members x Hq/Hkv <= 16 rows) that streams the shared tokens and
- * then each member's own tokens with the other members' rows masked out of the softmax.
+ * are stacked as the rows of one tensor-core tile (members x Hq/Hkv <= 64 rows) that streams
+ * the shared tokens and then each member's own tokens with the other members' rows masked
+ * out of the softmax.
  *   group_of      [B] device int32: group of batch row b, or -1
  *   group_prefix  [ngroups] device int32: shared tokens of the group, a multiple of
  *                 PA_SHARED_PREFIX_ALIGN and <= every member's length; members' tables must
@@ -211,7 +212,8 @@ pa_status pa_decode_append(void* out, const void* q, const void* k_new, const vo
  *                 shares no tokens; its members' own tokens are still read as one unit)
  *   group_members [ngroups][max_members] device int32: the group's batch rows, -1 padded
  * pa_alloc_prefix_groups builds these from the allocator.  bf16 tensor-core shapes only
- * (PA_ERR_UNSUPPORTED otherwise); max_members * (Hq/Hkv) <= 16; B + ngroups <= 8192.
+ * (PA_ERR_UNSUPPORTED otherwise); max_members <= 32, max_members * (Hq/Hkv) <= 64;
+ * B + ngroups <= 8192.
  * Workspace: pa_decode_shared_prefix_workspace_size (on the current device). */
 #define PA_SHARED_PREFIX_ALIGN 32
 size_t pa_decode_shared_prefix_workspace_size(int B, int Hq, int Hkv, int D, int block_size,

@@ -310,7 +310,8 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_pool,
     return PA_ERR_INVALID_ARG;
   const int G = Hq / Hkv;
   if (!pa::tc_eligible(G, D, block_size, dtype)) return PA_ERR_UNSUPPORTED;
-  if (G * max_members > 16 || B + ngroups > kStreamMaxB) return PA_ERR_UNSUPPORTED;
+  if (max_members > 32 || G * max_members > 64 || B + ngroups > kStreamMaxB)
+    return PA_ERR_UNSUPPORTED;
   const int64_t max_seq = static_cast<int64_t>(max_blocks) * block_size;
   if (max_seq > 0x7fffffffLL) return PA_ERR_INVALID_ARG;
   if (static_cast<int64_t>(B + ngroups) * Hkv * ceil_div(max_seq, PA_SHARED_PREFIX_ALIGN) >=

@@ -59,3 +59,27 @@ def test_full_size_every_row(name):
                 assert np.array_equal(pool_bits(pool), oracle_bits(ref, w))
         del g
         torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", ["prefix", "prefix_cow"])
+def test_full_size_shared_prefix_every_row(name):
+    """pa_decode_shared_prefix in the grouping bench.py times (whole fork families of
+    8 samples x 4 heads as one unit), every row against the oracle."""
+    import paged_kv_cache_350_b200 as pa
+    w = FULL[name]()
+    r = _oracle_every_row(w)
+    g = gpu_step(w, keep=True)
+    maxm = min(32, 64 // (w.Hq // w.Hkv))
+    gof, gpre, gmem = g["alloc"].prefix_groups(w.step_seqs, maxm, pa.binding.PA_SHARED_PREFIX_ALIGN)
+    assert len(gpre) == w.meta["prompts"]
+    n = pa.pa_decode_shared_prefix_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.block_size, len(gpre))
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    out = torch.full_like(g["q"], float("nan"))
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.pa_decode_shared_prefix(out, g["q"], g["k_pool"], g["v_pool"], g["t_d"], g["l_d"], w.scale,
+                               torch.from_numpy(gof).cuda(), torch.from_numpy(gpre).cuda(),
+                               torch.from_numpy(np.ascontiguousarray(gmem)).cuda(), ws,
+                               err_flag=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert_close(w, out, r["out"])

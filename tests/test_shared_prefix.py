@@ -71,6 +71,21 @@ CASES = {
     "prefix_bs32_d64": (lambda: workloads.prefix(prompts=2, n=4, prompt_len=130, max_private=50,
                                                  bs=32, D=64), 4),
     "mixed_no_groups": (lambda: workloads.gqa(B=5, median=100, lo=1, hi=200), 4),
+    # whole fork families as one unit: 32 and 64 stacked rows
+    "prefix_g4_m8": (lambda: workloads.prefix(prompts=3, n=8, prompt_len=150, max_private=60), 8),
+    "prefix_g4_m16": (lambda: workloads.prefix(prompts=2, n=16, prompt_len=130, max_private=70), 16),
+    "prefix_g8_m8": (lambda: workloads.prefix(prompts=2, n=8, prompt_len=200, max_private=30,
+                                              Hq=16, Hkv=2), 8),
+    "cow_g4_m8": (lambda: workloads.prefix_cow(prompts=2, n=8, prompt_len=100), 8),
+    "prefix_g1_m32": (lambda: workloads.prefix(prompts=1, n=32, prompt_len=64, max_private=40,
+                                               Hq=4, Hkv=4), 32),
+    "prefix_bs8_m8": (lambda: workloads.prefix(prompts=2, n=8, prompt_len=70, max_private=50,
+                                               bs=8), 8),
+    "prefix_bs32_d64_m8": (lambda: workloads.prefix(prompts=2, n=8, prompt_len=130,
+                                                    max_private=50, bs=32, D=64), 8),
+    # long prompts: units span several CTAs, so cut units are merged by the reduce
+    "long_prompt_m8": (lambda: workloads.prefix(prompts=4, n=8, prompt_len=2000,
+                                                max_private=300), 8),
 }
 
 
