@@ -491,8 +491,11 @@ def prepare(args, pa, device, config, block_size=0):
 
 def time_steps(st, K, W, dist, device):
     """W untimed steps, then K steps bracketed by a barrier and a synchronize on both sides,
-    timed with CUDA events on the launching stream (whole region, and each decode call);
-    the clocks are sampled during the timed region.  Times are the max over ranks."""
+    timed with CUDA events on the launching stream; then the same K steps again with an
+    event pair around each decode call (the kernel's own time: an event between two
+    kernels stops the second from launching while the first drains, so the whole-region
+    figure is taken without them).  The clocks are sampled during both.  Times are the max
+    over ranks."""
     import torch
     step, err, stream = st["step"], st["err"], st["stream"]
     for _ in range(W):
@@ -508,8 +511,11 @@ def time_steps(st, K, W, dist, device):
     clocks.start()
     t_start.record(stream)
     for i in range(K):
-        step(evs[i])
+        step()
     t_end.record(stream)
+    torch.cuda.synchronize()
+    for i in range(K):
+        step(evs[i])
     torch.cuda.synchronize()
     clocks.stop()
     barrier(dist, device)

@@ -276,6 +276,21 @@ bool make_pool_map(CUtensorMap* map, const void* pool, int NB, int BS, int Hkv, 
   return r == CUDA_SUCCESS;
 }
 
+bool make_q_map(CUtensorMap* map, const void* q, int B, int Hq, int D, int G) {
+  auto encode = get_encode_fn();
+  if (!encode || G < 1 || G > 256) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hq),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(Hq) * D * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(G), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims,
+                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 namespace {
 
 template <class C>

@@ -59,8 +59,10 @@ struct PrefixParams {
   int ngroups, max_members;
   int streams;
   int32_t* meta;   // [streams][4] cut-unit slot metadata
-  float* pml;      // [streams][2][16][2]
-  float* pacc;     // [streams][2][16][D]
+  float* pml;      // [streams][2][64][2]: (max, sum) of cut-unit pieces, base 2
+  float* pacc;     // [streams][2][64][D]: unnormalised outputs of those pieces
+  float* pxch;     // [streams][2][2][64][2]: per piece parity and column group, the
+                   // (max, sum) the two softmax column groups exchange
 };
 int prefix_grid(int D, int block_size, int R);
 int prefix_warps_per_cta();
@@ -72,6 +74,9 @@ cudaError_t launch_decode_prefix(const PrefixParams& pp, int grid, cudaStream_t 
 // block starting at a row coordinate) x 64 columns of one head.
 bool make_pool_map(CUtensorMap* map, const void* pool, int NB, int BS, int Hkv, int D,
                    int box_rows);
+// Tensor map over q viewed as [B][Hq][D] (bf16): boxes of 64 columns x G heads of one
+// batch row, 128-byte swizzled.
+bool make_q_map(CUtensorMap* map, const void* q, int B, int Hq, int D, int G);
 
 // Launch the bf16 tensor-core decode kernel (+ reduce when max_parts > 1).
 cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t stream);
