@@ -448,8 +448,8 @@ def prepare(args, pa, device, config, block_size=0):
         pre_of = np.where(gof >= 0, np.asarray(gpre, dtype=np.int64)[np.maximum(gof, 0)] if ng else 0, 0)
         tok_unique = int(np.asarray(gpre, dtype=np.int64).sum()) + int((lens - pre_of).sum())
         unique_kv = 2 * tok_unique * w.Hkv * w.D * esize
-        plan = {"kernel": "shared_prefix", "groups": ng, "max_members": maxm, "launches": 2}
-        launches_per_step = 2 + 1 + (1 if npairs else 0)
+        plan = {"kernel": "shared_prefix", "groups": ng, "max_members": maxm, "launches": 1}
+        launches_per_step = 1 + 1 + (1 if npairs else 0)
 
     def step(ev=None):
         if npairs:
@@ -536,7 +536,7 @@ def roofline(st, dec_avg_ms, config):
             "traffic": recorded_traffic(config, "pa_decode_append" if fused else "pa_decode"),
             "kernel": ("pa_decode_append call (decode kernel with the fused cache write + its "
                        "reduce)" if fused else
-                       "pa_decode_shared_prefix call (main kernel + its cut reduce)"
+                       "pa_decode_shared_prefix call (one kernel; cut units merged inside it)"
                        if st["unique_kv"] is not None else
                        "pa_decode call (main kernel + its reduce)") + ", CUDA events per call",
             "append_bytes_per_call": st["append_bytes"],

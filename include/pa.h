@@ -214,7 +214,12 @@ pa_status pa_decode_append(void* out, const void* q, const void* k_new, const vo
  * pa_alloc_prefix_groups builds these from the allocator.  bf16 tensor-core shapes only
  * (PA_ERR_UNSUPPORTED otherwise); max_members <= 32, max_members * (Hq/Hkv) <= 64;
  * B + ngroups <= 8192.
- * Workspace: pa_decode_shared_prefix_workspace_size (on the current device). */
+ * One launch: a persistent kernel with one CTA per SM.  A unit split between CTAs is
+ * merged by the CTA that finishes its last piece (the pieces' partials and a per-call
+ * tagged counter live in the workspace; no CTA waits for another).
+ * Workspace: pa_decode_shared_prefix_workspace_size (on the current device); its contents
+ * need no initialisation, and calls whose kernels may overlap on the GPU must not share
+ * one. */
 #define PA_SHARED_PREFIX_ALIGN 32
 size_t pa_decode_shared_prefix_workspace_size(int B, int Hq, int Hkv, int D, int block_size,
                                               int ngroups);

@@ -356,6 +356,7 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* k_pool,
   pp.ngroups = ngroups;
   pp.max_members = max_members;
   pa::prefix_carve(&pp, workspace, rows);
+  pp.epoch = pa::prefix_epoch();
   const cudaError_t e = pa::launch_decode_prefix(pp, grid, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

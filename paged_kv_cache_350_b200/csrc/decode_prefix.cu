@@ -19,7 +19,7 @@
 // walks its range in tiles of up to four chunks (128 tokens) of one unit; a tile may hold
 // several members' own chunks (each row masks the chunks that are not its own).  A unit
 // cut by a range boundary leaves a partial (max, sum, unnormalised output) per row, which
-// the cut reduce merges by log-sum-exp.
+// the CTA completing the unit merges by log-sum-exp.
 //
 // Per CTA, warp-specialised:
 //   warps 0, 1  producers, taking turns tile by tile: resolve block ids through the
@@ -55,6 +55,7 @@
 
 #include <atomic>
 #include <climits>
+#include <random>
 
 #include "pa_device.cuh"
 #include "pa_internal.h"
@@ -95,7 +96,7 @@ struct TileInfo {
   int nch;        // chunks in this tile (1..4)
   int flags;
   int piece;      // index of the piece (unit part) within this CTA
-  int slot;       // partial slot of a cut piece (0: the CTA's first piece, 1: last)
+  int ubeg, uend; // the unit's chunk range (for the merge of a cut unit)
   int mem[kCPT];  // per chunk: member (-1: shared tokens, every row)
   int nv[kCPT];   // per chunk: valid tokens (1..32)
 };
@@ -282,6 +283,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // (max, sum) in the CTA's exchange slots i (i = piece parity, so a post never meets an
   // unread one); the slots are in global memory, as shared memory is full
   __shared__ __align__(8) uint64_t xch_bar[2][4];
+  // cut_bar[0]: the softmax threads have written a cut piece's partial; cut_bar[1]: the
+  // partials the owner of a cut unit merges have been published
+  __shared__ __align__(8) uint64_t cut_bar[2];
   __shared__ TileInfo info[kMaxStages];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int warp_sum[kWarps];
@@ -301,6 +305,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(smem_addr(&pfull_bar[0]), kSoftThreads);
     mbar_init(smem_addr(&pfull_bar[1]), kSoftThreads);
     for (int i = 0; i < 8; ++i) mbar_init(smem_addr(&xch_bar[i >> 2][i & 3]), 64);
+    mbar_init(smem_addr(&cut_bar[0]), kSoftThreads);
+    mbar_init(smem_addr(&cut_bar[1]), 1);
     mbar_init(smem_addr(&pvdone_bar[0]), 1);
     mbar_init(smem_addr(&pvdone_bar[1]), 1);
     mbar_init(smem_addr(&drain_bar), 1);
@@ -385,7 +391,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int cta = static_cast<int>(blockIdx.x);
   const int beg = min(T, cta * per);
   const int end = min(T, beg + per);
-  // Let the cut reduce be launched now; it waits for this grid to complete.
+  // Let the next kernel on the stream be launched now; it waits for this grid to complete
+  // before it touches memory.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const float sl2 = p.scale_log2;
 
@@ -529,7 +536,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     };
 
-    int own_u = -1, own_slot = 0, own_n = 0, own_rows = 0;
     int q_loads = 0;  // Q loads issued (pieces 0 .. q_loads - 1)
     int t = 0, piece = 0;
     bool ok = beg < end;
@@ -552,14 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // stage) before either loads a tile
     asm volatile("bar.sync 1, 64;" ::: "memory");
     while (ok) {
-      const int slot = pc.g == beg ? 0 : 1;
       const bool complete = pc.g == pc.ubeg && pc.pend == pc.uend;
-      if (!complete && pc.ubeg >= beg) {  // the unit starts here: it is this CTA's to merge
-        own_u = pc.r * Hkv + pc.kvh;
-        own_slot = slot;
-        own_n = (pc.uend - 1) / per - cta + 1;
-        own_rows = pc.rows;
-      }
       const bool has_next = pc.pend < end;
       // steps of the next piece's preparation done (4: all; producer 1 has no Q step)
       int prep = has_next ? 0 : 4;
@@ -597,7 +596,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ti->rows = pc.rows;
             ti->nch = nch;
             ti->piece = piece;
-            ti->slot = slot;
+            ti->ubeg = pc.ubeg;
+            ti->uend = pc.uend;
             ti->flags = (c0 == pc.g ? kFirstOfPiece : 0) | (last_of_piece ? kLastOfPiece : 0) |
                         (last_of_piece && !has_next ? kLastOfCta : 0) |
                         (complete ? kCompleteUnit : 0);
@@ -688,10 +688,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(smem_addr(&kfull_bar[k % nst]), (k / nst) & 1, nullptr, kWaitLimitNs);
         mbar_wait(smem_addr(&vfull_bar[k % nst]), (k / nst) & 1, nullptr, kWaitLimitNs);
       }
-    }
-    if (pw == 0 && lane == 0) {
-      const int4 m = make_int4(abort_flag ? -1 : own_u, own_slot, own_n, own_rows);
-      *reinterpret_cast<int4*>(pp.meta + cta * 4) = m;
     }
   } else if (warp == 2) {
     // spare: no work after the prologue
@@ -847,6 +843,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tid_g = (warp & 3) * 32 + lane;   // 0..127 within the group
     float m_ref = -INFINITY, lsum = 0.f;        // lsum: this thread's part of the row sum
     int b_row = -1;  // the row's batch row, loaded at the piece's first tile, used at its end
+    int pub_uses = 0, own_uses = 0;  // phases of cut_bar[0] and cut_bar[1]
+    // A unit cut by CTA range boundaries: its first piece is the last piece of the CTA c0
+    // holding its first chunk (the owner), each other piece the first piece of a later
+    // CTA.  A later CTA writes its piece's partial (max, sum, unnormalised output per row)
+    // and publishes it with an epoch-tagged flag; the owner, at its piece's end, takes
+    // those partials and merges them with its own piece by log-sum-exp as it writes the
+    // rows' output.  The other pieces are at the start of their CTAs' ranges, so the
+    // owner's wait (bounded) has normally ended before it begins; every CTA of the grid is
+    // resident before any later kernel can be (a dependent grid launches only once each
+    // CTA has passed the prologue's trigger), so the CTAs it waits for do run.
+    auto publish_partial = [&](int use) -> bool {
+      mbar_arrive(smem_addr(&cut_bar[0]));  // release: this thread's partial first
+      if (threadIdx.x == 4 * 32) {
+        if (!wait_or_abort(smem_addr(&cut_bar[0]), use & 1, p.err, &abort_flag)) return false;
+        st_release_gpu(pp.cut_flag + cta, pp.epoch);
+      }
+      return true;
+    };
+    // The owner: wait for the flags of CTAs c0 + 1 .. c0 + n - 1 (one thread), then let
+    // every softmax thread read the partials.
+    auto await_partials = [&](int n, int use) -> bool {
+      if (threadIdx.x == 4 * 32) {
+        const uint64_t t0 = global_timer_ns();
+        for (int i = 1; i < n && !abort_flag; ++i) {
+          while (ld_acquire_gpu(pp.cut_flag + cta + i) != pp.epoch) {
+            if (abort_flag) break;
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+              flag_error(p.err, PA_DEVERR_TIMEOUT);
+              abort_flag = 1;
+              break;
+            }
+          }
+        }
+        mbar_arrive(smem_addr(&cut_bar[1]));  // release: the acquired flags come first
+      }
+      return wait_warp(smem_addr(&cut_bar[1]), use & 1, p.err, &abort_flag) && !abort_flag;
+    };
     bool ok = beg < end;
     for (int t = 0; ok; ++t) {
       const int s = t % nst;
@@ -980,8 +1013,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kvh = ti.unit % Hkv;
         const int b = b_row;
         const bool complete = (ti.flags & kCompleteUnit) != 0;
-        const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
-        const size_t prow = (static_cast<size_t>(cta) * 2 + ti.slot) * kRows + r;
+        const bool owner = !complete && ti.ubeg >= beg;  // the unit's first chunk is here
+        const int n = owner ? (ti.uend - 1) / per - cta + 1 : 1;  // pieces of the unit
+        // the owner merges the partials of the unit's other pieces (those of CTAs
+        // cta + 1 .. cta + n - 1) with its own: the row's max, its own weight, the sum
+        float M = mx, e_own = 1.f, L = ltot;
+        if (n > 1) {
+          if (!await_partials(n, own_uses++)) break;
+          for (int i = 1; i < n; ++i)
+            M = fmaxf(M, __ldcg(reinterpret_cast<const float2*>(pp.pml) +
+                                static_cast<size_t>(cta + i) * kRows + r).x);
+          e_own = mx == -INFINITY ? 0.f : ex2_approx(mx - M);
+          L = e_own * ltot;
+          for (int i = 1; i < n; ++i) {
+            const float2 ml = __ldcg(reinterpret_cast<const float2*>(pp.pml) +
+                                     static_cast<size_t>(cta + i) * kRows + r);
+            L += ml.x == -INFINITY ? 0.f : ex2_approx(ml.x - M) * ml.y;
+          }
+        }
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        const size_t prow = static_cast<size_t>(cta) * kRows + r;  // this CTA's partial row
         // group g writes output columns [g * D / 2, (g + 1) * D / 2); each thread reads its
         // own lane (O hi or O lo) of both accumulators, and the pair adds the two
 #pragma unroll
@@ -1002,10 +1053,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int col = c + 16 * h;  // this thread's 16 of the 32 columns
           float vv[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) vv[j] = h ? v[16 + j] : v[j];
-          if (complete) {
+          for (int j = 0; j < 16; ++j) vv[j] = (h ? v[16 + j] : v[j]) * e_own;
+          for (int i = 1; i < n; ++i) {  // the other pieces' partials (the owner of a cut unit)
+            const size_t pr = static_cast<size_t>(cta + i) * kRows + r;
+            const float2 ml = __ldcg(reinterpret_cast<const float2*>(pp.pml) + pr);
+            if (ml.x == -INFINITY) continue;
+            const float wi = ex2_approx(ml.x - M);
+            const float4* src = reinterpret_cast<const float4*>(pp.pacc + pr * D + col);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float4 a = __ldcg(src + j);
+              vv[4 * j] += wi * a.x;
+              vv[4 * j + 1] += wi * a.y;
+              vv[4 * j + 2] += wi * a.z;
+              vv[4 * j + 3] += wi * a.w;
+            }
+          }
+          if (complete || owner) {
             // a row without output (length 0) is left to the prologue's zero fill
-            if (b >= 0 && b < B && ltot > 0.f) {
+            if (b >= 0 && b < B && L > 0.f) {
               uint4* o = reinterpret_cast<uint4*>(
                   out + (static_cast<size_t>(b) * p.Hq + kvh * G + r % G) * D + col);
 #pragma unroll
@@ -1015,16 +1081,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   pack_bf16x2(vv[8 * j + 4] * inv, vv[8 * j + 5] * inv),
                                   pack_bf16x2(vv[8 * j + 6] * inv, vv[8 * j + 7] * inv));
             }
-          } else {
+          } else {  // a later piece of a cut unit: its partial, for the owner
             float4* o = reinterpret_cast<float4*>(pp.pacc + prow * D + col);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               o[j] = make_float4(vv[4 * j], vv[4 * j + 1], vv[4 * j + 2], vv[4 * j + 3]);
           }
         }
-        // a row with no token here has max -inf, sum 0
-        if (active && !complete && grp == 0 && h == 0)
-          *reinterpret_cast<float2*>(pp.pml + prow * 2) = make_float2(mx, ltot);
+        if (!complete && !owner) {
+          // a row with no token here has max -inf, sum 0
+          if (active && grp == 0 && h == 0)
+            *reinterpret_cast<float2*>(pp.pml + prow * 2) = make_float2(mx, ltot);
+          if (!publish_partial(pub_uses++)) break;
+        }
       }
       if (ti.flags & kLastOfCta) break;
     }
@@ -1035,51 +1104,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc05::fence_after_sync();
   if (warp == kMmaWarp) tc05::dealloc(tmem, kTmemCols);
-}
-
-// Merge the pieces of units cut by a CTA boundary and write the outputs of their rows.
-// Piece i of the unit CTA s owns is slot 0 of CTA s + i, except the first, which is in the
-// slot CTA s recorded.  A piece that holds no token of a row has max -inf and is skipped
-// for that row.
-template <int D>
-__global__ void __launch_bounds__(256) group_cut_reduce_kernel(const PrefixParams pp) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const DecodeParams& p = pp.d;
-  const int s = blockIdx.x;
-  const int4 m = *reinterpret_cast<const int4*>(pp.meta + static_cast<size_t>(s) * 4);
-  if (m.x < 0) return;
-  const int u = m.x, slot0 = m.y, n = m.z, nrows = m.w;
-  const int ur = u / p.Hkv, kvh = u - ur * p.Hkv;
-  const int G = p.G;
-  constexpr int TPR = D / 4;  // threads per row
-  for (int idx = threadIdx.x; idx < nrows * TPR; idx += blockDim.x) {
-    const int row = idx / TPR;
-    const int c = (idx % TPR) * 4;
-    const int b = ur < pp.ngroups ? member_of(pp, ur, row / G) : ur - pp.ngroups;
-    float M = -INFINITY, l = 0.f, a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 4
-    for (int i = 0; i < n; ++i) {
-      const size_t pr = (static_cast<size_t>(s + i) * 2 + (i == 0 ? slot0 : 0)) * kRows + row;
-      const float2 ml = *reinterpret_cast<const float2*>(pp.pml + pr * 2);
-      const float4 a = *reinterpret_cast<const float4*>(pp.pacc + pr * D + c);
-      const float Mn = fmaxf(M, ml.x);
-      const float so = M == -INFINITY ? 0.f : exp2f(M - Mn);
-      const float sn = ml.x == -INFINITY ? 0.f : exp2f(ml.x - Mn);
-      l = l * so + ml.y * sn;
-      a0 = a0 * so + a.x * sn;
-      a1 = a1 * so + a.y * sn;
-      a2 = a2 * so + a.z * sn;
-      a3 = a3 * so + a.w * sn;
-      M = Mn;
-    }
-    if (b < 0 || b >= p.B || !(l > 0.f)) continue;  // no output row, or one left to the zero fill
-    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) +
-                       (static_cast<size_t>(b) * p.Hq + kvh * G + row % G) * D + c;
-    const float inv = 1.f / l;
-    *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf16x2(a0 * inv, a1 * inv),
-                                              pack_bf16x2(a2 * inv, a3 * inv));
-  }
 }
 
 // Per device: the opt-in shared memory per block and the SM count, read once; per kernel
@@ -1156,9 +1180,7 @@ cudaError_t launch_group_cfg(PrefixParams pp, int grid, cudaStream_t stream) {
   if (nst == 0) return cudaErrorInvalidValue;
   const size_t smem = group_smem_bytes<C>(nst, R);
   if (!grant_smem<C>(dev, smem)) return cudaErrorInvalidValue;
-  cudaError_t e;
-  // the main kernel as a programmatic dependent of the previous kernel on the stream,
-  // the cut reduce as one of the main kernel
+  // a programmatic dependent of the previous kernel on the stream
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -1169,12 +1191,7 @@ cudaError_t launch_group_cfg(PrefixParams pp, int grid, cudaStream_t stream) {
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
-  if ((e = cudaLaunchKernelEx(&cfg, decode_group_kernel<C>, tmk, tmv, tmq, pp, nst)) != cudaSuccess)
-    return e;
-  cfg.gridDim = dim3(static_cast<unsigned>(pp.streams));
-  cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = 0;
-  return cudaLaunchKernelEx(&cfg, group_cut_reduce_kernel<C::D>, pp);
+  return cudaLaunchKernelEx(&cfg, decode_group_kernel<C>, tmk, tmv, tmq, pp, nst);
 }
 
 }  // namespace
@@ -1196,22 +1213,32 @@ int prefix_warps_per_cta() { return 1; }  // one partial-slot owner per CTA
 size_t prefix_workspace_bytes(int streams, int rows, int D) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   (void)rows;
-  return up(static_cast<size_t>(streams) * 16) + up(static_cast<size_t>(streams) * 2 * kRows * 8) +
-         up(static_cast<size_t>(streams) * 2 * kRows * D * 4) +
+  return up(static_cast<size_t>(streams) * 8) + up(static_cast<size_t>(streams) * kRows * 8) +
+         up(static_cast<size_t>(streams) * kRows * D * 4) +
          static_cast<size_t>(streams) * 2 * 2 * kRows * 8;
 }
 
 void prefix_carve(PrefixParams* pp, void* workspace, int rows) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   char* w = static_cast<char*>(workspace);
-  pp->meta = reinterpret_cast<int32_t*>(w);
-  w += up(static_cast<size_t>(pp->streams) * 16);
+  pp->cut_flag = reinterpret_cast<unsigned long long*>(w);
+  w += up(static_cast<size_t>(pp->streams) * 8);
   pp->pml = reinterpret_cast<float*>(w);
-  w += up(static_cast<size_t>(pp->streams) * 2 * kRows * 8);
+  w += up(static_cast<size_t>(pp->streams) * kRows * 8);
   pp->pacc = reinterpret_cast<float*>(w);
-  w += up(static_cast<size_t>(pp->streams) * 2 * kRows * pp->d.D * 4);
+  w += up(static_cast<size_t>(pp->streams) * kRows * pp->d.D * 4);
   pp->pxch = reinterpret_cast<float*>(w);
   (void)rows;
+}
+
+uint64_t prefix_epoch() {
+  // a 64-bit tag per call for the cut-unit flags: a flag left by another call, or never
+  // written, holds another value
+  static std::atomic<uint64_t> next{[] {
+    std::random_device rd;
+    return (static_cast<uint64_t>(rd()) << 32) ^ rd();
+  }()};
+  return next.fetch_add(1, std::memory_order_relaxed);
 }
 
 cudaError_t launch_decode_prefix(const PrefixParams& pp, int grid, cudaStream_t stream) {

@@ -58,9 +58,11 @@ struct PrefixParams {
   const int32_t* group_members;  // [ngroups][max_members] batch rows, -1 padded
   int ngroups, max_members;
   int streams;
-  int32_t* meta;   // [streams][4] cut-unit slot metadata
-  float* pml;      // [streams][2][64][2]: (max, sum) of cut-unit pieces, base 2
-  float* pacc;     // [streams][2][64][D]: unnormalised outputs of those pieces
+  uint64_t epoch;  // this call's tag for the cut-unit flags
+  unsigned long long* cut_flag;  // [streams]: = epoch once CTA s has published the partial
+                                 // of its first piece (a later piece of a cut unit)
+  float* pml;      // [streams][64][2]: (max, sum) of that piece per row, base 2
+  float* pacc;     // [streams][64][D]: its unnormalised output per row
   float* pxch;     // [streams][2][2][64][2]: per piece parity and column group, the
                    // (max, sum) the two softmax column groups exchange
 };
@@ -68,6 +70,8 @@ int prefix_grid(int D, int block_size, int R);
 int prefix_warps_per_cta();
 size_t prefix_workspace_bytes(int streams, int rows, int D);
 void prefix_carve(PrefixParams* pp, void* workspace, int rows);
+// A fresh tag for one shared-prefix call.
+uint64_t prefix_epoch();
 cudaError_t launch_decode_prefix(const PrefixParams& pp, int grid, cudaStream_t stream);
 
 // 4-D TMA view of a bf16 pool [NB][BS][Hkv][D]: box = box_rows rows (BS, or a part of a
