@@ -808,9 +808,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          // nothing ready: sleep briefly on the event this step needs first
-          if (!pv_done) mbar_try_wait_for(pb, ppar, 200);
-          else mbar_try_wait_for(kb1, par1, 200);
+          // nothing ready: a short pause, then look at both events again (a wait on one of
+          // them would hold up the other: S of the next tile is due as soon as its K has
+          // landed, P.V of this one as soon as its P is written)
+          __nanosleep(32);
         }
         if (!more) break;
       }
