@@ -8,7 +8,8 @@
 // query head).
 //
 // Units.  One unit per (group row, KV head): the query heads of that KV head of all the
-// group's members are stacked as the rows of one tile (members x G <= 64 rows).  A unit's
+// group's members are stacked as the rows of one tile (members x G <= 64 rows; member m's
+// G heads are rows m*G .. m*G + G - 1, the order of q).  A unit's
 // tokens are a list of 32-token chunks: first the shared tokens [0, prefix) through the
 // first member's table, which every row attends to, then each member's own tokens
 // [prefix, L_m) through that member's table, which only that member's rows attend to.  An
@@ -17,9 +18,10 @@
 // Schedule.  One persistent CTA per SM; the chunks of all units laid end to end are split
 // into equal contiguous ranges, one per CTA, so the work is balanced to one chunk.  A CTA
 // walks its range in tiles of up to four chunks (128 tokens) of one unit; a tile may hold
-// several members' own chunks (each row masks the chunks that are not its own).  A unit
-// cut by a range boundary leaves a partial (max, sum, unnormalised output) per row, which
-// the CTA completing the unit merges by log-sum-exp.
+// several members' own chunks (each row masks the chunks that are not its own).  The
+// pieces of a unit cut by range boundaries are merged by log-sum-exp in the same launch:
+// the later CTAs publish per-row partials (max, sum, unnormalised output), which the CTA
+// holding the unit's first chunk folds into its own rows' output.
 //
 // Per CTA, warp-specialised:
 //   warps 0, 1  producers, taking turns tile by tile: resolve block ids through the
@@ -116,7 +118,7 @@ struct GroupCfg {
   static_assert(BS == 8 || BS == 16 || BS == 32, "block size");
 };
 
-// Static shared memory of the kernel is below this (barriers, tile records: ~530 B).
+// Static shared memory of the kernel is below this (barriers, tile records: ~560 B).
 constexpr size_t kStaticSmemBound = 640;
 
 template <class C>
