@@ -1091,6 +1091,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               o[j] = make_float4(vv[4 * j], vv[4 * j + 1], vv[4 * j + 2], vv[4 * j + 3]);
           }
         }
+        if (n > 1 && threadIdx.x == 4 * 32) {
+          // consumed: clear the flags, so that a replay of this same launch (a CUDA graph
+          // keeps its tag) waits for fresh partials
+          for (int i = 1; i < n; ++i) pp.cut_flag[cta + i] = 0ull;
+        }
         if (!complete && !owner) {
           // a row with no token here has max -inf, sum 0
           if (active && grp == 0 && h == 0)
@@ -1236,7 +1241,8 @@ void prefix_carve(PrefixParams* pp, void* workspace, int rows) {
 
 uint64_t prefix_epoch() {
   // a 64-bit tag per call for the cut-unit flags: a flag left by another call, or never
-  // written, holds another value
+  // written, holds another value (the owner clears the flags it consumed, for replays of
+  // a captured launch, which keep their tag)
   static std::atomic<uint64_t> next{[] {
     std::random_device rd;
     return (static_cast<uint64_t>(rd()) << 32) ^ rd();

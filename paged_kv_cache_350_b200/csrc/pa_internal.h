@@ -70,7 +70,7 @@ int prefix_grid(int D, int block_size, int R);
 int prefix_warps_per_cta();
 size_t prefix_workspace_bytes(int streams, int rows, int D);
 void prefix_carve(PrefixParams* pp, void* workspace, int rows);
-// A fresh tag for one shared-prefix call.
+// A fresh tag for one shared-prefix call (its cut-unit flags).
 uint64_t prefix_epoch();
 cudaError_t launch_decode_prefix(const PrefixParams& pp, int grid, cudaStream_t stream);
 

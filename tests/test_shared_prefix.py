@@ -83,7 +83,7 @@ CASES = {
                                                bs=8), 8),
     "prefix_bs32_d64_m8": (lambda: workloads.prefix(prompts=2, n=8, prompt_len=130,
                                                     max_private=50, bs=32, D=64), 8),
-    # long prompts: units span several CTAs, so cut units are merged by the reduce
+    # long prompts: units span several CTAs, so cut units are merged across CTAs
     "long_prompt_m8": (lambda: workloads.prefix(prompts=4, n=8, prompt_len=2000,
                                                 max_private=300), 8),
 }
@@ -163,3 +163,58 @@ def test_group_with_no_shared_tokens(all_empty):
     for b in np.flatnonzero(lens == 0):
         assert (got[b] == 0).all()
     assert_close(workloads.independent([1]), out, ref)
+
+
+@pytest.mark.gpu
+def test_shared_prefix_replayed_from_a_cuda_graph():
+    """The shared-prefix call captured in a CUDA graph and replayed, on a batch whose units
+    span several CTAs (cut units merged across CTAs, through flags tagged per call): a
+    replay keeps the call's tag, so the flags must be cleared once consumed.  After a call
+    no flag is left set (the flags lead the workspace, one 8-byte word per CTA), and every
+    replay, each with new queries, matches an eager call on the same inputs bit for bit."""
+    import paged_kv_cache_350_b200 as pa
+    w = workloads.prefix(prompts=4, n=8, prompt_len=2000, max_private=300)
+    maxm = 8
+    _, g, _ = _shared_prefix_gpu(w, maxm)
+    gof, gpre, gmem = g["alloc"].prefix_groups(w.step_seqs, maxm, pa.binding.PA_SHARED_PREFIX_ALIGN)
+    n = pa.pa_decode_shared_prefix_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.block_size, len(gpre))
+    gof_d = torch.from_numpy(gof).cuda()
+    gpre_d = torch.from_numpy(np.ascontiguousarray(gpre)).cuda()
+    gmem_d = torch.from_numpy(np.ascontiguousarray(gmem).reshape(len(gpre), maxm)).cuda()
+    q = g["q"].clone()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def call(out, ws, stream=None):
+        pa.pa_decode_shared_prefix(out, q, g["k_pool"], g["v_pool"], g["t_d"], g["l_d"], w.scale,
+                                   gof_d, gpre_d, gmem_d, ws, err_flag=err, stream=stream)
+
+    # flags: zero before, zero after (each one set by a later piece is cleared by its owner)
+    ws_eager = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    ref = torch.empty_like(q)
+    call(ref, ws_eager)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    ctas = torch.cuda.get_device_properties(0).multi_processor_count
+    assert int(ws_eager[: ctas * 8].count_nonzero()) == 0
+
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(q)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):  # warm-up on the capture stream (first-call setup)
+        call(out, ws, stream=s)
+    s.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        call(out, ws, stream=s)
+    gen = torch.Generator(device="cuda").manual_seed(7700)
+    for _ in range(3):
+        q.copy_(torch.randn(q.shape, generator=gen, device="cuda", dtype=torch.float32).to(q.dtype))
+        out.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        call(ref, ws_eager)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+    del graph
