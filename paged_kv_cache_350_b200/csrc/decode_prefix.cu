@@ -30,10 +30,10 @@
 //               Q rows (one box per member) into one of two Q buffers;
 //   warp 3      MMA: one thread issues, per tile, S = Q.K^T (M = 64 rows, N = tile
 //               tokens, K = head dim; A = Q, B = K, both K-major in shared memory) into
-//               one of two S accumulators in tensor memory, and O += P.V (M = 128: the
-//               rows' P hi and P lo parts stacked, A = P from tensor memory, B = V,
-//               MN-major in shared memory); S of the next tile is issued as soon as its K
-//               has landed, so that it overlaps this tile's softmax;
+//               one of two S accumulators in tensor memory, and O += P.V (M = 64, once
+//               for the P hi parts and once for the P lo parts; A = P from tensor memory,
+//               B = V, MN-major in shared memory); S of the next tile is issued as soon as
+//               its K has landed, so that it overlaps this tile's softmax;
 //   warps 4-11  softmax, two column groups of four warps: group g takes chunks 2g and
 //               2g + 1 of every tile, with its own online softmax (fp32, base 2, a lazy
 //               rescale: the reference max moves only when a tile's max passes it by more
@@ -697,7 +697,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ============================ MMA issuer ============================
     if (lane == 0 && beg < end) {
       const uint32_t id_s_base = tc05::instr_desc_bf16(kRows, 8, 0) & ~(0x3Fu << 17);
-      const uint32_t id_pv = tc05::instr_desc_bf16(2 * kRows, D, 1);  // P hi and lo rows
+      const uint32_t id_pv = tc05::instr_desc_bf16(kRows, D, 1);
       bool ok = true;
       // The tile records are read from shared memory where they are used (a record stays
       // until its stage is released after the tile's P.V), and every loop below is
@@ -767,8 +767,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 C::KV_CHUNK_BYTES, 1024);
             const uint32_t tp = tmem + ((t & 1) ? kColS1 : kColS0);  // P of tile t
             if (flags & kFirstOfPiece) fresh0 = fresh1 = true;
-            // chunk q's P at S columns 64 * (q / 2) + 16 * (q % 2); chunks 0-1 go into O0,
-            // 2-3 into O1; a chunk's second 16-token step only where it has valid tokens
+            // chunk q's P hi parts at S columns 64 * (q / 2) + 16 * (q % 2), its lo parts 32
+            // columns on; chunks 0-1 go into O0, 2-3 into O1 (hi, then lo, accumulated); a
+            // chunk's second 16-token step only where it has valid tokens
 #pragma unroll
             for (int q = 0; q < kCPT; ++q) {
               if (q < nch) {
@@ -781,9 +782,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t pa = tp + 64 * (q >> 1) + 16 * (q & 1) + 8 * kk;
                     if (q < 2) {
                       tc05::mma_ts(tmem + kColO0, pa, vdesc, id_pv, !fresh0);
+                      tc05::mma_ts(tmem + kColO0, pa + 32, vdesc, id_pv, true);
                       fresh0 = false;
                     } else {
                       tc05::mma_ts(tmem + kColO1, pa, vdesc, id_pv, !fresh1);
+                      tc05::mma_ts(tmem + kColO1, pa + 32, vdesc, id_pv, true);
                       fresh1 = false;
                     }
                   }
@@ -832,10 +835,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // group serves each sub-partition.  Threads t and t + 16 share the row of lane t % 16
     // when reading S (the 16x32bx2 shape): half h = t / 16 takes chunk 2g + h, so a row's
     // max and sum within the group combine by one shuffle.  P goes back over the group's
-    // S columns with one row per lane: thread t < 16 writes the row's hi parts to lane t,
-    // thread t + 16 its lo parts to lane t + 16, so P.V is one M = 128 product per 16
-    // tokens whose accumulator rows follow the same lanes (O hi and O lo, added when the
-    // piece's output is read).
+    // S columns in the same shape, each half writing its own chunk's hi parts and lo
+    // parts in separate column blocks, so P.V is two M = 64 products per 16 tokens (hi,
+    // then lo) into the same accumulator rows, and no lane exchange is needed.
     const int sp = warp & 3;                    // tensor-memory sub-partition
     const int grp = (warp - 4) >> 2;            // column group
     const int h = lane >> 4;                    // chunk within the group's pair
@@ -942,15 +944,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                        &abort_flag))
           break;
         tc05::fence_after_sync();
-        const uint32_t oa = tmem + col_o + lane_addr;  // lane t: O hi (t < 16) or O lo
+        const uint32_t oa = tmem + col_o + lane_addr;  // the row's O (lanes 0-15)
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
+        for (int c = 0; c < D; c += 64) {
           uint32_t v[32];
-          tc05::ld32(oa + c, v);
+          tc05::ld_pair32(oa + c, v);  // this half's 32 of the 64 columns
           tc05::wait_ld();
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
-          tc05::st32(oa + c, v);
+          tc05::st_pair32(oa + c, v);
         }
       }
       lsum *= alpha;
@@ -973,9 +975,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         fence_proxy_async_smem();
-        // P over this group's S columns: lane t (< 16) the row's hi parts, lane t + 16 its
-        // lo parts, packed pairs (chunk 2g at columns 64g .. 64g + 15, 2g + 1 after it)
-        uint32_t w[32];
+        // P over this group's S columns, in the row's lane: the hi parts of chunks 2g and
+        // 2g + 1 (packed pairs) at columns 64g .. 64g + 31, their lo parts at 64g + 32 ..
+        // 64g + 63; each half of the lane pair writes its own chunk (the 16x32bx2 shape)
+        uint32_t whi[16], wlo[16];
         float ls = 0.f;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -983,14 +986,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float p0 = ex2_approx(fmaf(x[2 * j], sl2, -mref));
           const float p1 = ex2_approx(fmaf(x[2 * j + 1], sl2, -mref));
           ls += p0 + p1;
-          uint32_t hi, lo;
-          split_bf16x2(p0, p1, hi, lo);
-          // half 0 keeps its hi parts and sends its lo parts; half 1 the reverse
-          const uint32_t got = __shfl_xor_sync(kFull, h ? hi : lo, 16);
-          w[j] = h ? got : hi;       // chunk 2g: hi (lane t) or lo (lane t + 16)
-          w[16 + j] = h ? lo : got;  // chunk 2g + 1
+          split_bf16x2(p0, p1, whi[j], wlo[j]);
         }
-        tc05::st32(sbuf + 64 * grp, w);
+        tc05::st_pair16(sbuf + 64 * grp, whi);
+        tc05::st_pair16(sbuf + 64 * grp + 32, wlo);
         lsum += ls;
         tc05::wait_st();
       }
@@ -1036,59 +1035,62 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float inv = L > 0.f ? 1.f / L : 0.f;
         const size_t prow = static_cast<size_t>(cta) * kRows + r;  // this CTA's partial row
-        // group g writes output columns [g * D / 2, (g + 1) * D / 2); each thread reads its
-        // own lane (O hi or O lo) of both accumulators, and the pair adds the two
-#pragma unroll
-        for (int c = grp * D / 2; c < (grp + 1) * D / 2; c += 32) {
-          uint32_t a0[32], a1[32];
-          tc05::ld32(tmem + kColO0 + lane_addr + c, a0);
-          tc05::ld32(tmem + kColO1 + lane_addr + c, a1);
+        // group g writes output columns [g * D / 2, (g + 1) * D / 2): each half of the lane
+        // pair reads W = D / 4 of them from both accumulators (the row's lane)
+        {
+          constexpr int W = D / 4;
+          const int c = grp * D / 2;
+          uint32_t a0[W], a1[W];
+          if constexpr (W == 32) {
+            tc05::ld_pair32(tmem + kColO0 + lane_addr + c, a0);
+            tc05::ld_pair32(tmem + kColO1 + lane_addr + c, a1);
+          } else {
+            tc05::ld_pair16(tmem + kColO0 + lane_addr + c, a0);
+            tc05::ld_pair16(tmem + kColO1 + lane_addr + c, a1);
+          }
           tc05::wait_ld();
-          float v[32];
+          const int col = c + W * h;  // this thread's W columns
+          float vv[W];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
+          for (int j = 0; j < W; ++j)
             // an accumulator with weight 0 may never have been written in this piece
-            const float part = (w0 > 0.f ? w0 * __uint_as_float(a0[j]) : 0.f) +
-                               (w1 > 0.f ? w1 * __uint_as_float(a1[j]) : 0.f);
-            v[j] = part + __shfl_xor_sync(kFull, part, 16);
-          }
-          if (!active) continue;
-          const int col = c + 16 * h;  // this thread's 16 of the 32 columns
-          float vv[16];
+            vv[j] = ((w0 > 0.f ? w0 * __uint_as_float(a0[j]) : 0.f) +
+                     (w1 > 0.f ? w1 * __uint_as_float(a1[j]) : 0.f)) * e_own;
+          if (active) {
+            // the other pieces' partials (the owner of a cut unit)
+            for (int i = 1; i < n; ++i) {
+              const size_t pr = static_cast<size_t>(cta + i) * kRows + r;
+              const float2 ml = __ldcg(reinterpret_cast<const float2*>(pp.pml) + pr);
+              if (ml.x == -INFINITY) continue;
+              const float wi = ex2_approx(ml.x - M);
+              const float4* src = reinterpret_cast<const float4*>(pp.pacc + pr * D + col);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) vv[j] = (h ? v[16 + j] : v[j]) * e_own;
-          for (int i = 1; i < n; ++i) {  // the other pieces' partials (the owner of a cut unit)
-            const size_t pr = static_cast<size_t>(cta + i) * kRows + r;
-            const float2 ml = __ldcg(reinterpret_cast<const float2*>(pp.pml) + pr);
-            if (ml.x == -INFINITY) continue;
-            const float wi = ex2_approx(ml.x - M);
-            const float4* src = reinterpret_cast<const float4*>(pp.pacc + pr * D + col);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float4 a = __ldcg(src + j);
-              vv[4 * j] += wi * a.x;
-              vv[4 * j + 1] += wi * a.y;
-              vv[4 * j + 2] += wi * a.z;
-              vv[4 * j + 3] += wi * a.w;
+              for (int j = 0; j < W / 4; ++j) {
+                const float4 a = __ldcg(src + j);
+                vv[4 * j] += wi * a.x;
+                vv[4 * j + 1] += wi * a.y;
+                vv[4 * j + 2] += wi * a.z;
+                vv[4 * j + 3] += wi * a.w;
+              }
             }
-          }
-          if (complete || owner) {
-            // a row without output (length 0) is left to the prologue's zero fill
-            if (b >= 0 && b < B && L > 0.f) {
-              uint4* o = reinterpret_cast<uint4*>(
-                  out + (static_cast<size_t>(b) * p.Hq + kvh * G + r % G) * D + col);
+            if (complete || owner) {
+              // a row without output (length 0) is left to the prologue's zero fill
+              if (b >= 0 && b < B && L > 0.f) {
+                uint4* o = reinterpret_cast<uint4*>(
+                    out + (static_cast<size_t>(b) * p.Hq + kvh * G + r % G) * D + col);
 #pragma unroll
-              for (int j = 0; j < 2; ++j)
-                o[j] = make_uint4(pack_bf16x2(vv[8 * j] * inv, vv[8 * j + 1] * inv),
-                                  pack_bf16x2(vv[8 * j + 2] * inv, vv[8 * j + 3] * inv),
-                                  pack_bf16x2(vv[8 * j + 4] * inv, vv[8 * j + 5] * inv),
-                                  pack_bf16x2(vv[8 * j + 6] * inv, vv[8 * j + 7] * inv));
+                for (int j = 0; j < W / 8; ++j)
+                  o[j] = make_uint4(pack_bf16x2(vv[8 * j] * inv, vv[8 * j + 1] * inv),
+                                    pack_bf16x2(vv[8 * j + 2] * inv, vv[8 * j + 3] * inv),
+                                    pack_bf16x2(vv[8 * j + 4] * inv, vv[8 * j + 5] * inv),
+                                    pack_bf16x2(vv[8 * j + 6] * inv, vv[8 * j + 7] * inv));
+              }
+            } else {  // a later piece of a cut unit: its partial, for the owner
+              float4* o = reinterpret_cast<float4*>(pp.pacc + prow * D + col);
+#pragma unroll
+              for (int j = 0; j < W / 4; ++j)
+                o[j] = make_float4(vv[4 * j], vv[4 * j + 1], vv[4 * j + 2], vv[4 * j + 3]);
             }
-          } else {  // a later piece of a cut unit: its partial, for the owner
-            float4* o = reinterpret_cast<float4*>(pp.pacc + prow * D + col);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              o[j] = make_float4(vv[4 * j], vv[4 * j + 1], vv[4 * j + 2], vv[4 * j + 3]);
           }
         }
         if (n > 1 && threadIdx.x == 4 * 32) {
