@@ -895,6 +895,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool active = r < ti.rows;
       const int my_member = r / G;
       const bool has = ti.nch > 2 * grp;        // the tile reaches this group's chunks
+      // a warp whose 16 rows are all past the unit's rows (a unit of up to 32 rows leaves
+      // sub-partitions 2 and 3 idle) keeps only the barrier protocol and its share of the V
+      // zeroing: the P rows it leaves unwritten only reach accumulator rows never output
+      const bool live = has && 16 * sp < ti.rows;
       if (first) {
         m_ref = -INFINITY;
         lsum = 0.f;
@@ -906,7 +910,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sbuf = tmem + ((t & 1) ? kColS1 : kColS0) + lane_addr;
       float x[32];  // this thread's chunk of raw scores; -inf where masked
       float mt = -INFINITY;
-      if (has) {
+      if (live) {
         uint32_t v[32];
         tc05::ld_pair32(sbuf + 64 * grp, v);
         tc05::wait_ld();
@@ -975,6 +979,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         fence_proxy_async_smem();
+      }
+      if (live) {
         // P over this group's S columns, in the row's lane: the hi parts of chunks 2g and
         // 2g + 1 (packed pairs) at columns 64g .. 64g + 31, their lo parts at 64g + 32 ..
         // 64g + 63; each half of the lane pair writes its own chunk (the 16x32bx2 shape)
