@@ -44,10 +44,11 @@
 //               lo = rn(p - hi), so it keeps ~16 significant bits;
 //   warp 2      spare.
 // Tensor memory: S buffers at columns 0 and 128 (lanes 0-15 of each sub-partition, the
-// M = 64 layout), each overwritten by its P once the softmax has read it (the hi parts of
-// a row in its own lane, the lo parts in the lane 16 above it, packed pairs), so P is
-// double buffered with S; the groups' O accumulators at 256 and 384 (128 lanes: the rows'
-// P hi.V and P lo.V, added when the output is read).
+// M = 64 layout), each overwritten by its P once the softmax has read it (in the row's
+// lane, group g's hi parts at columns 64g .. 64g + 31 and its lo parts at 64g + 32 ..
+// 64g + 63, packed pairs), so P is double buffered with S; the groups' O accumulators at
+// 256 and 384 (the M = 64 layout as well: P hi.V and P lo.V accumulate in the same rows).
+// Softmax warps whose rows are all past a unit's rows skip their score reads and P.
 //
 // Every wait is bounded in time; on expiry the kernel records PA_DEVERR_TIMEOUT, every
 // role stops, the loads and tensor-core operations in flight are drained (bounded), and
