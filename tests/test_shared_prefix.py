@@ -86,6 +86,12 @@ CASES = {
     # long prompts: units span several CTAs, so cut units are merged across CTAs
     "long_prompt_m8": (lambda: workloads.prefix(prompts=4, n=8, prompt_len=2000,
                                                 max_private=300), 8),
+    # units of 64, 36, 24, 12 and 4 rows (and ungrouped sequences) in one launch, so a CTA
+    # moves between units whose rows fill different numbers of sub-partitions
+    "families_mixed_m16": (lambda: workloads.families(), 16),
+    "families_mixed_long_m16": (lambda: workloads.families(seed=1022, sizes=(9, 16, 2, 5),
+                                                           solo=4, prompt_len=1500,
+                                                           max_private=200), 16),
 }
 
 

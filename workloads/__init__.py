@@ -248,6 +248,45 @@ def prefix(seed=1003, prompts=32, n=8, prompt_len=1024, max_private=256, Hq=32, 
     )
 
 
+def families(seed=1021, sizes=(16, 3, 6, 1, 9), solo=3, prompt_len=140, max_private=70,
+             Hq=32, Hkv=8, D=128, bs=16, dtype="bf16"):
+    """Fork families of mixed sizes (each prompt forked into ``sizes[i]`` samples holding
+    U{0..max_private} private tokens) and ``solo`` unforked sequences of U{1..300} tokens,
+    in one batch: units of different row counts meet in one launch."""
+    rng = np.random.default_rng(seed)
+    ops, seqs = [], []
+    need, max_tok, sid = 0, 0, 0
+    for n in sizes:
+        parent = sid
+        ops.append(("add", parent, prompt_len))
+        need += _blocks(prompt_len, bs)
+        for k in range(1, n):
+            ops.append(("fork", parent, parent + k))
+        for k in range(n):
+            priv = int(rng.integers(0, max_private + 1))
+            if priv:
+                ops.append(("append", parent + k, priv))
+            seqs.append(parent + k)
+            total = prompt_len + priv + 1
+            max_tok = max(max_tok, total)
+            need += _blocks(total, bs) - (prompt_len // bs)
+        sid += n
+    for _ in range(solo):
+        L = int(rng.integers(1, 301))
+        ops.append(("add", sid, L - 1))
+        seqs.append(sid)
+        need += _blocks(L, bs)
+        max_tok = max(max_tok, L)
+        sid += 1
+    nb = max(1, math.ceil(1.1 * need))
+    return Workload(
+        name="families", dtype=dtype, B=len(seqs), Hq=Hq, Hkv=Hkv, D=D, block_size=bs,
+        num_blocks=nb, scale=1.0 / math.sqrt(D), alloc_seed=seed, setup_ops=ops,
+        step_seqs=seqs, seed=seed, max_blocks=_blocks(max_tok, bs),
+        meta={"sizes": list(sizes), "solo": solo, "prompt_len": prompt_len},
+    )
+
+
 def prefix_cow(seed=1013, prompts=32, n=8, prompt_len=1000, **kw):
     return prefix(seed=seed, prompts=prompts, n=n, prompt_len=prompt_len, first_divergence=True, **kw)
 
