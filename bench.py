@@ -575,12 +575,23 @@ def run_ours(args):
     # are queued back to back over three staging slots, and each step's output is read two
     # steps later (so the host and the copies of neighbouring steps stay off the GPU's
     # critical path).
+    # Shared-prefix runs take the pipeline's shared-prefix steps (fork groups formed in the
+    # same C call; copy_blocks, reshape_and_cache and pa_decode_shared_prefix), on a pool of
+    # their own with room for every step's appends (zeroed blocks: the work does not depend
+    # on the values; the batch's 10 % of free blocks would last a few steps).
     e2e = None
-    if not args.no_e2e and args.e2e_steps > 0 and not args.shared_prefix:
-        cache = pa.PagedKVCache(w.num_blocks, w.block_size, w.Hkv, w.D, dtype=kp.dtype, device=device,
-                                shuffle_seed=w.alloc_seed, pop_order=w.pop_order, k_pool=kp, v_pool=vp)
+    if not args.no_e2e and args.e2e_steps > 0:
+        members = plan["max_members"] if args.shared_prefix else 0
+        if members:
+            nb_e2e = w.num_blocks + w.B * ((args.e2e_steps + 8 + w.block_size - 1) // w.block_size + 1)
+            cache = pa.PagedKVCache(nb_e2e, w.block_size, w.Hkv, w.D, dtype=kp.dtype, device=device,
+                                    shuffle_seed=w.alloc_seed, pop_order=w.pop_order)
+        else:
+            cache = pa.PagedKVCache(w.num_blocks, w.block_size, w.Hkv, w.D, dtype=kp.dtype,
+                                    device=device, shuffle_seed=w.alloc_seed, pop_order=w.pop_order,
+                                    k_pool=kp, v_pool=vp)
         workloads.run_setup(w, cache.alloc)
-        pipe = cache.pipeline(w.B, w.Hq, MB, depth=3, stream=stream)
+        pipe = cache.pipeline(w.B, w.Hq, MB, depth=3, stream=stream, shared_prefix_members=members)
         lag = pipe.depth - 1
         q_c, nk_c, nv_c = q.cpu(), nk.cpu(), nv.cpu()
         ids = np.asarray(w.step_seqs, dtype=np.int64)
@@ -621,10 +632,13 @@ def run_ours(args):
                    "ms_per_step": 1e3 * dt / done, "steps": done,
                    "host_us_per_submit": 1e6 * statistics.median(host_s) if host_s else None,
                    "timing": "host perf_counter over the steps of PagedKVCache.pipeline: per step "
-                             "one C call (pa_pipeline_submit: the allocator, one host->device copy "
-                             "of the step input, the kernels, a device->host copy of the output, "
-                             "read two steps later); steps queued back to back over three staging "
-                             "slots"}
+                             "one C call (pa_pipeline_submit: the allocator%s, one host->device "
+                             "copy of the step input, the kernels, a device->host copy of the "
+                             "output, read two steps later); steps queued back to back over three "
+                             "staging slots%s" % (
+                                 " and the fork grouping" if members else "",
+                                 "; the batch grows a token per step, so only the first step "
+                                 "copies blocks on write" if members else "")}
 
     # ---- the long-context batch, timed in the same run ---------------------------------
     # The decode must hold its bandwidth on both serving shapes: the GQA batch above and

@@ -396,6 +396,13 @@ int pa_alloc_free_list(const pa_allocator* a, int32_t* out, int cap);
  * "什么是 LLM 中的分页注意力", 使用分页注意力: each new token fills the next slot of the
  * sequence's current block).
  *
+ * With shared_prefix_members > 0 a step is the parallel-sampling one ("深入解析
+ * PagedAttention", 多序列共享): after the appends the allocator also groups the rows whose
+ * tables share leading blocks (pa_alloc_prefix_groups, up to shared_prefix_members rows a
+ * group, PA_SHARED_PREFIX_ALIGN) and writes the slot mapping, and the kernels are
+ * pa_copy_blocks, pa_reshape_and_cache and pa_decode_shared_prefix, which reads each
+ * group's shared blocks once.
+ *
  * Ownership: every buffer and stream is the caller's; the pipeline creates only CUDA
  * events (no device memory).  The allocator is borrowed: it must outlive the pipeline and
  * not be used by another thread during a call.  Not thread-safe.
@@ -419,6 +426,9 @@ typedef struct pa_pipeline_desc {
   pa_stream_t compute;        /* kernels */
   pa_stream_t copy_in;        /* host->device copies */
   pa_stream_t copy_out;       /* device->host copies */
+  int shared_prefix_members;  /* 0: pa_decode_append; 1 .. 32 (and * Hq/Hkv <= 64): the
+                                 shared-prefix step, workspace of
+                                 pa_decode_shared_prefix_workspace_size(B, .., B / 2) bytes */
 } pa_pipeline_desc;
 
 /* Bytes of one input slot; offsets[6] (nullable) receives the byte offsets of its
@@ -427,6 +437,13 @@ typedef struct pa_pipeline_desc {
  * (written by the pipeline).  0 for invalid arguments. */
 size_t pa_pipeline_input_bytes(int B, int Hq, int Hkv, int D, int max_blocks, pa_dtype dtype,
                                size_t* offsets);
+/* The same for a pipeline with shared_prefix_members = m: offsets[10] (nullable) adds,
+ * after those six, slot_mapping [B] int64, group_of [B], group_prefix [B] and
+ * group_members [B][m] int32 (all written by the pipeline).  With m = 0 it equals
+ * pa_pipeline_input_bytes.  0 for invalid arguments (m outside 0 .. 32). */
+size_t pa_pipeline_input_bytes_prefix(int B, int Hq, int Hkv, int D, int max_blocks,
+                                      pa_dtype dtype, int shared_prefix_members,
+                                      size_t* offsets);
 /* The descriptor's arrays are copied.  PA_ERR_INVALID_ARG for a bad descriptor. */
 pa_status pa_pipeline_create(pa_allocator* alloc, const pa_pipeline_desc* desc,
                              pa_pipeline** out);
@@ -438,7 +455,9 @@ pa_status pa_pipeline_next_slot(pa_pipeline* p, int* slot);
 /* Queue one step for seq_ids[B] (distinct live sequences; the batch order of q/k/v).
  * *step (nullable) = its index (0, 1, ...), *h2d_bytes (nullable) = bytes copied in.
  * Returns once the step is queued.  An allocator error (e.g. PA_ERR_OUT_OF_BLOCKS) leaves
- * everything unchanged; after PA_ERR_CUDA the pipeline should be destroyed. */
+ * everything unchanged, except that a failure of the shared-prefix grouping (host memory
+ * only) leaves the step's appends made; after PA_ERR_CUDA the pipeline should be
+ * destroyed. */
 pa_status pa_pipeline_submit(pa_pipeline* p, const int64_t* seq_ids, float scale,
                              int64_t* step, size_t* h2d_bytes);
 /* Waits for step's output copy; *slot = the host_out slot holding it, valid until step +

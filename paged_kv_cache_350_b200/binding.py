@@ -85,7 +85,7 @@ class pa_pipeline_desc(ctypes.Structure):
                 ("host_out", ctypes.POINTER(ctypes.c_void_p)),
                 ("dev_out", ctypes.POINTER(ctypes.c_void_p)),
                 ("compute", ctypes.c_void_p), ("copy_in", ctypes.c_void_p),
-                ("copy_out", ctypes.c_void_p)]
+                ("copy_out", ctypes.c_void_p), ("shared_prefix_members", ctypes.c_int)]
 
 
 def _load():
@@ -140,6 +140,8 @@ def _load():
         "pa_alloc_free_list": (i32, [vp, pi32, i32]),
         "pa_alloc_check_append_fits": (i32, [vp, pi64, i32, i32]),
         "pa_pipeline_input_bytes": (sz, [i32, i32, i32, i32, i32, i32, ctypes.POINTER(sz)]),
+        "pa_pipeline_input_bytes_prefix": (sz, [i32, i32, i32, i32, i32, i32, i32,
+                                                ctypes.POINTER(sz)]),
         "pa_pipeline_create": (i32, [vp, ctypes.POINTER(pa_pipeline_desc), ctypes.POINTER(vp)]),
         "pa_pipeline_destroy": (None, [vp]),
         "pa_pipeline_next_slot": (i32, [vp, pint]),
@@ -168,7 +170,8 @@ EXPORTED = (
     "pa_alloc_beam_select", "pa_alloc_block_table",
     "pa_alloc_block_tables", "pa_alloc_seq_slots", "pa_alloc_refcount", "pa_alloc_num_free",
     "pa_alloc_internal_waste_slots", "pa_alloc_free_list", "pa_alloc_check_append_fits",
-    "pa_pipeline_input_bytes", "pa_pipeline_create", "pa_pipeline_destroy",
+    "pa_pipeline_input_bytes", "pa_pipeline_input_bytes_prefix", "pa_pipeline_create",
+    "pa_pipeline_destroy",
     "pa_pipeline_next_slot", "pa_pipeline_submit", "pa_pipeline_result", "pa_pipeline_sync",
 )
 

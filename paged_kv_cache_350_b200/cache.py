@@ -21,6 +21,11 @@ caller writes the step's q / new K / new V straight into the cache's pinned
 input buffer, the allocator writes slots, tables and lengths behind them, and a
 single copy moves the whole step input.
 
+``step_shared_prefix`` is ``step`` for parallel sampling: the sequences that share a
+prompt's blocks are grouped (``pa_alloc_prefix_groups``), the new tokens' K/V go to their
+slots with ``pa_reshape_and_cache``, and ``pa_decode_shared_prefix`` reads each group's
+shared blocks once.
+
 ``pipeline`` (``StepPipeline``, the C ``pa_pipeline_*`` calls) queues such steps back to
 back, one C call per step: staging in several slots, the copies on their own streams, so
 the host and the copy engines work on neighbouring steps while the GPU decodes the
@@ -117,6 +122,81 @@ class PagedKVCache:
         stream.synchronize()
         return h2d, out_host.numel() * out_host.element_size()
 
+    # -- one decode step reading each fork group's shared prompt once ------------------
+    def step_shared_prefix(self, seq_ids, q_host, k_host, v_host, out_host, scale, max_blocks,
+                           max_members, stream=None):
+        """``step`` with the shared-prefix attention.
+
+        Sequences forked from one prompt point at the same physical blocks ("深入解析
+        PagedAttention", 多序列共享); after this step's appends (so that a block copied on
+        write is a member's own), ``pa_alloc_prefix_groups`` groups them, up to
+        ``max_members`` per group, and ``pa_decode_shared_prefix`` reads each group's shared
+        blocks once (``max_members`` <= 32 and ``max_members`` * Hq / Hkv <= 64).  The new
+        tokens' K/V are written to their slots by ``pa_reshape_and_cache`` first.  Same
+        tensors as ``step``; returns (h2d_bytes, d2h_bytes), and ``last_prefix_groups`` is the
+        number of groups formed.
+        """
+        stream = stream or torch.cuda.current_stream(self.device)
+        B, Hq, D = q_host.shape
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        slots_h = self._pinned(("slots",), (B,), torch.int64)
+        pairs_h = self._pinned(("pairs",), (B, 2), torch.int32)
+        tables_h = self._pinned(("tables",), (B, max_blocks), torch.int32)
+        lens_h = self._pinned(("lens",), (B,), torch.int32)
+        _, pairs = self.alloc.append_slots(ids, slot_out=slots_h.numpy(), pairs_out=pairs_h.numpy())
+        self.alloc.block_tables(ids, max_blocks, tables_out=tables_h.numpy(), lens_out=lens_h.numpy())
+        npairs = pairs.shape[0]
+        gof, gpre, gmem = self.alloc.prefix_groups(ids, max_members)
+        ng = len(gpre)
+        self.last_prefix_groups = ng
+        gof_h = self._pinned(("gof",), (B,), torch.int32)
+        gpre_h = self._pinned(("gpre",), (B,), torch.int32)
+        gmem_h = self._pinned(("gmem",), (B, max_members), torch.int32)
+        gof_h.numpy()[:] = gof
+        gpre_h.numpy()[:ng] = gpre
+        gmem_h.numpy()[:ng] = gmem
+
+        with torch.cuda.stream(stream):
+            q = self._dev(("q",), q_host.shape, self.dtype)
+            kn = self._dev(("k",), k_host.shape, self.dtype)
+            vn = self._dev(("v",), v_host.shape, self.dtype)
+            tables = self._dev(("tables",), (B, max_blocks), torch.int32)
+            lens = self._dev(("lens",), (B,), torch.int32)
+            slots = self._dev(("slots",), (B,), torch.int64)
+            gof_d = self._dev(("gof",), (B,), torch.int32)
+            gpre_d = self._dev(("gpre",), (B,), torch.int32)
+            gmem_d = self._dev(("gmem",), (B, max_members), torch.int32)
+            out = self._dev(("out",), q_host.shape, self.dtype)
+            h2d = 0
+            for dst, src in ((q, q_host), (kn, k_host), (vn, v_host), (tables, tables_h),
+                             (lens, lens_h), (slots, slots_h), (gof_d, gof_h)):
+                dst.copy_(src, non_blocking=True)
+                h2d += src.numel() * src.element_size()
+            if ng:
+                gpre_d[:ng].copy_(gpre_h[:ng], non_blocking=True)
+                gmem_d[:ng].copy_(gmem_h[:ng], non_blocking=True)
+                h2d += ng * 4 * (1 + max_members)
+            if npairs:
+                pairs_d = self._dev(("pairs",), (B, 2), torch.int32)
+                pairs_d[:npairs].copy_(pairs_h[:npairs], non_blocking=True)
+                h2d += npairs * 8
+                _b.pa_copy_blocks(self.k_pool, self.v_pool, pairs_d[:npairs], err_flag=self.err,
+                                  stream=stream)
+            _b.pa_reshape_and_cache(kn, vn, self.k_pool, self.v_pool, slots, err_flag=self.err,
+                                    stream=stream)
+            n = _b.pa_decode_shared_prefix_workspace_size(B, Hq, self.Hkv, self.D,
+                                                          self.block_size, ng)
+            ws = getattr(self, "_ws_prefix", None)
+            if ws is None or ws.numel() < max(n, 1):
+                ws = self._ws_prefix = torch.empty(max(n, 1), dtype=torch.uint8,
+                                                   device=self.device)
+            _b.pa_decode_shared_prefix(out, q, self.k_pool, self.v_pool, tables, lens, scale,
+                                       gof_d, gpre_d, gmem_d[:ng], ws, err_flag=self.err,
+                                       stream=stream)
+            out_host.copy_(out, non_blocking=True)
+        stream.synchronize()
+        return h2d, out_host.numel() * out_host.element_size()
+
     # -- one decode step, single staged copy -----------------------------------------
     def _layout(self, B, Hq, max_blocks):
         """Byte offsets of the sections of the step input buffer (256-byte aligned)."""
@@ -193,9 +273,11 @@ class PagedKVCache:
         stream.synchronize()
         return self._out_h, (used, self._out_h.numel() * self._out_h.element_size())
 
-    def pipeline(self, B, Hq, max_blocks, depth=2, stream=None):
-        """A StepPipeline over this cache: decode steps queued back to back."""
-        return StepPipeline(self, B, Hq, max_blocks, depth=depth, stream=stream)
+    def pipeline(self, B, Hq, max_blocks, depth=2, stream=None, shared_prefix_members=0):
+        """A StepPipeline over this cache: decode steps queued back to back (with
+        ``shared_prefix_members`` > 0, the steps of ``step_shared_prefix``)."""
+        return StepPipeline(self, B, Hq, max_blocks, depth=depth, stream=stream,
+                            shared_prefix_members=shared_prefix_members)
 
     # -- sequence management ------------------------------------------------------------
     def admit(self, seq_id, k_host, v_host, stream=None):
@@ -256,9 +338,13 @@ class StepPipeline:
         out = pipe.result(t)           # waits for step t's output copy (pinned [B,Hq,D])
 
     ``result(t)`` stays valid until step t + depth is submitted.
+
+    With ``shared_prefix_members`` > 0 each step is that of ``PagedKVCache.step_shared_prefix``
+    (fork groups formed by the C allocator in the same call; ``pa_copy_blocks``,
+    ``pa_reshape_and_cache`` and ``pa_decode_shared_prefix`` queued).
     """
 
-    def __init__(self, cache, B, Hq, max_blocks, depth=2, stream=None):
+    def __init__(self, cache, B, Hq, max_blocks, depth=2, stream=None, shared_prefix_members=0):
         import ctypes
         assert depth >= 1
         self.cache, self.B, self.Hq, self.max_blocks, self.depth = cache, B, Hq, max_blocks, depth
@@ -268,10 +354,11 @@ class StepPipeline:
         self.copy_out = torch.cuda.Stream(self.dev)
         D, Hkv, dt = cache.D, cache.Hkv, cache.dtype
         pdt = _b.PA_BF16 if dt == torch.bfloat16 else _b.PA_F32
-        offs = (ctypes.c_size_t * 6)()
-        total = _b.lib.pa_pipeline_input_bytes(B, Hq, Hkv, D, max_blocks, pdt, offs)
+        m = int(shared_prefix_members)
+        offs = (ctypes.c_size_t * 10)()
+        total = _b.lib.pa_pipeline_input_bytes_prefix(B, Hq, Hkv, D, max_blocks, pdt, m, offs)
         if total == 0:
-            raise _b.PAError(_b.PA_ERR_INVALID_ARG, "pa_pipeline_input_bytes")
+            raise _b.PAError(_b.PA_ERR_INVALID_ARG, "pa_pipeline_input_bytes_prefix")
         self.offsets = list(offs)
         n_out = B * Hq * D
         self.h_in = [torch.empty(total, dtype=torch.uint8, pin_memory=True) for _ in range(depth)]
@@ -280,7 +367,13 @@ class StepPipeline:
                       for _ in range(depth)]
         self.d_out = [torch.empty(n_out, dtype=dt, device=self.dev).view(B, Hq, D)
                       for _ in range(depth)]
-        self.ws = cache.workspace(B, Hq, max_blocks)
+        if m:
+            # the shared-prefix workspace: its size does not grow with the groups of a step
+            # (at most B / 2: a group has two members or more)
+            n = _b.pa_decode_shared_prefix_workspace_size(B, Hq, Hkv, D, cache.block_size, B // 2)
+            self.ws = torch.empty(max(n, 1), dtype=torch.uint8, device=self.dev)
+        else:
+            self.ws = cache.workspace(B, Hq, max_blocks)
         esz = self.h_out[0].element_size()
         sec = [B * Hq * D * esz, B * Hkv * D * esz, B * Hkv * D * esz]
         self._in_views = [tuple(h[o:o + n].view(dt).view(shape) for o, n, shape in
@@ -293,7 +386,7 @@ class StepPipeline:
             cache.k_pool.data_ptr(), cache.v_pool.data_ptr(),
             self.ws.data_ptr() if self.ws is not None else None,
             self.ws.numel() if self.ws is not None else 0, cache.err.data_ptr(), *self._arrays,
-            self.stream.cuda_stream, self.copy_in.cuda_stream, self.copy_out.cuda_stream)
+            self.stream.cuda_stream, self.copy_in.cuda_stream, self.copy_out.cuda_stream, m)
         h = ctypes.c_void_p()
         _b._check(_b.lib.pa_pipeline_create(cache.alloc._h, ctypes.byref(desc), ctypes.byref(h)),
                   "pa_pipeline_create")

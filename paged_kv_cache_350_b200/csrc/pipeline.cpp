@@ -8,6 +8,11 @@
 // batch of a few hundred sequences.  Here one call does the whole step's host work in C and
 // queues it, so the host prepares step t+1 while the GPU decodes step t.
 //
+// With shared_prefix_members > 0 the step is the parallel-sampling one: the allocator also
+// groups the sequences that share a prompt's blocks (pa_alloc_prefix_groups) and writes the
+// slot mapping, and the kernels are pa_copy_blocks, pa_reshape_and_cache and
+// pa_decode_shared_prefix, which reads each group's shared blocks once.
+//
 // Staging: `depth` slots, each a pinned host input buffer, a device input buffer, a device
 // output and a pinned host output, all caller-owned.  The input copy runs on `copy_in`,
 // the kernels on `compute`, the output copy on `copy_out`; events order every reuse of a
@@ -32,7 +37,9 @@ size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 struct pa_pipeline {
   pa_allocator* alloc = nullptr;
   pa_pipeline_desc d{};
-  size_t off[6] = {};  // q, k_new, v_new, block_tables, seq_lens, pairs
+  // q, k_new, v_new, block_tables, seq_lens, pairs; with shared_prefix_members > 0 also
+  // slot_mapping, group_of, group_prefix, group_members
+  size_t off[10] = {};
   size_t in_bytes = 0, out_bytes = 0;
   std::vector<void*> h_in, d_in, h_out, d_out;
   std::vector<cudaEvent_t> h2d_done, kern_done, d2h_done;
@@ -46,6 +53,7 @@ namespace {
 bool valid_desc(const pa_pipeline_desc* d) {
   return d && d->B > 0 && d->Hq > 0 && d->Hkv > 0 && d->Hq % d->Hkv == 0 && d->D > 0 &&
          d->block_size > 0 && d->max_blocks > 0 && d->num_blocks > 0 && d->depth >= 1 &&
+         d->shared_prefix_members >= 0 && d->shared_prefix_members <= 32 &&
          d->depth <= 64 && (d->dtype == PA_F32 || d->dtype == PA_BF16) && d->k_pool &&
          d->v_pool && d->host_in && d->dev_in && d->host_out && d->dev_out;
 }
@@ -60,22 +68,35 @@ void destroy_events(pa_pipeline* p) {
 
 extern "C" {
 
-size_t pa_pipeline_input_bytes(int B, int Hq, int Hkv, int D, int max_blocks, pa_dtype dtype,
-                               size_t* offsets) {
+size_t pa_pipeline_input_bytes_prefix(int B, int Hq, int Hkv, int D, int max_blocks,
+                                      pa_dtype dtype, int shared_prefix_members,
+                                      size_t* offsets) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || max_blocks <= 0 ||
-      (dtype != PA_F32 && dtype != PA_BF16))
+      (dtype != PA_F32 && dtype != PA_BF16) || shared_prefix_members < 0 ||
+      shared_prefix_members > 32)
     return 0;
   const size_t e = dtype == PA_BF16 ? 2 : 4;
-  const size_t sizes[6] = {static_cast<size_t>(B) * Hq * D * e, static_cast<size_t>(B) * Hkv * D * e,
-                           static_cast<size_t>(B) * Hkv * D * e,
-                           static_cast<size_t>(B) * max_blocks * 4, static_cast<size_t>(B) * 4,
-                           static_cast<size_t>(B) * 8};
+  const size_t b = static_cast<size_t>(B);
+  const bool sp = shared_prefix_members > 0;
+  const size_t sizes[10] = {b * Hq * D * e, b * Hkv * D * e, b * Hkv * D * e,
+                            b * max_blocks * 4, b * 4, b * 8,
+                            sp ? b * 8 : 0, sp ? b * 4 : 0, sp ? b * 4 : 0,
+                            b * static_cast<size_t>(shared_prefix_members) * 4};
   size_t off = 0;
-  for (int i = 0; i < 6; ++i) {
+  for (int i = 0; i < 10; ++i) {
     if (offsets) offsets[i] = off;
     off += up(sizes[i]);
   }
   return off;
+}
+
+size_t pa_pipeline_input_bytes(int B, int Hq, int Hkv, int D, int max_blocks, pa_dtype dtype,
+                               size_t* offsets) {
+  size_t all[10];
+  const size_t n = pa_pipeline_input_bytes_prefix(B, Hq, Hkv, D, max_blocks, dtype, 0, all);
+  if (n && offsets)
+    for (int i = 0; i < 6; ++i) offsets[i] = all[i];
+  return n;
 }
 
 pa_status pa_pipeline_create(pa_allocator* alloc, const pa_pipeline_desc* desc,
@@ -94,8 +115,9 @@ pa_status pa_pipeline_create(pa_allocator* alloc, const pa_pipeline_desc* desc,
   try {
     p->alloc = alloc;
     p->d = *desc;
-    p->in_bytes = pa_pipeline_input_bytes(desc->B, desc->Hq, desc->Hkv, desc->D,
-                                          desc->max_blocks, desc->dtype, p->off);
+    p->in_bytes = pa_pipeline_input_bytes_prefix(desc->B, desc->Hq, desc->Hkv, desc->D,
+                                                 desc->max_blocks, desc->dtype,
+                                                 desc->shared_prefix_members, p->off);
     p->out_bytes = static_cast<size_t>(desc->B) * desc->Hq * desc->D *
                    (desc->dtype == PA_BF16 ? 2 : 4);
     p->h_in.assign(desc->host_in, desc->host_in + depth);
@@ -151,15 +173,27 @@ pa_status pa_pipeline_submit(pa_pipeline* p, const int64_t* seq_ids, float scale
   // so that a step that cannot be described changes no allocator state
   pa_status st = pa_alloc_check_append_fits(p->alloc, seq_ids, d.B, d.max_blocks);
   if (st != PA_OK) return st;
+  const int m = d.shared_prefix_members;
   int npairs = 0;
   int32_t* pairs_h = reinterpret_cast<int32_t*>(h + p->off[5]);
-  st = pa_alloc_append_slots(p->alloc, seq_ids, d.B, p->slots.data(), pairs_h, &npairs);
+  int64_t* slots_h = m ? reinterpret_cast<int64_t*>(h + p->off[6]) : p->slots.data();
+  st = pa_alloc_append_slots(p->alloc, seq_ids, d.B, slots_h, pairs_h, &npairs);
   if (st != PA_OK) return st;
   st = pa_alloc_block_tables(p->alloc, seq_ids, d.B, reinterpret_cast<int32_t*>(h + p->off[3]),
                              d.max_blocks, reinterpret_cast<int32_t*>(h + p->off[4]));
   if (st != PA_OK) return st;
-  const size_t used = npairs ? p->off[5] + static_cast<size_t>(npairs) * 8
-                             : p->off[4] + static_cast<size_t>(d.B) * 4;
+  int ngroups = 0;
+  if (m) {
+    // after this step's appends, so that a block copied on write is a member's own
+    st = pa_alloc_prefix_groups(p->alloc, seq_ids, d.B, m, PA_SHARED_PREFIX_ALIGN,
+                                reinterpret_cast<int32_t*>(h + p->off[7]),
+                                reinterpret_cast<int32_t*>(h + p->off[8]),
+                                reinterpret_cast<int32_t*>(h + p->off[9]), &ngroups);
+    if (st != PA_OK) return st;
+  }
+  const size_t used = m ? p->off[9] + static_cast<size_t>(ngroups) * m * 4
+                      : npairs ? p->off[5] + static_cast<size_t>(npairs) * 8
+                               : p->off[4] + static_cast<size_t>(d.B) * 4;
   cudaStream_t cin = reinterpret_cast<cudaStream_t>(d.copy_in);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(d.compute);
   cudaStream_t cout = reinterpret_cast<cudaStream_t>(d.copy_out);
@@ -178,11 +212,27 @@ pa_status pa_pipeline_submit(pa_pipeline* p, const int64_t* seq_ids, float scale
                         d.compute);
     if (st != PA_OK) return st;
   }
-  st = pa_decode_append(p->d_out[k], dv + p->off[0], dv + p->off[1], dv + p->off[2], d.k_pool,
-                        d.v_pool, reinterpret_cast<const int32_t*>(dv + p->off[3]),
-                        reinterpret_cast<const int32_t*>(dv + p->off[4]), d.B, d.Hq, d.Hkv, d.D,
-                        d.block_size, d.max_blocks, d.num_blocks, scale, d.dtype, d.workspace,
-                        d.workspace_bytes, d.dev_err_flag, d.compute, nullptr);
+  if (m) {
+    st = pa_reshape_and_cache(dv + p->off[1], dv + p->off[2], d.k_pool, d.v_pool,
+                              reinterpret_cast<const int64_t*>(dv + p->off[6]), d.B, d.Hkv, d.D,
+                              d.block_size, d.num_blocks, d.dtype, d.dev_err_flag, d.compute);
+    if (st != PA_OK) return st;
+    st = pa_decode_shared_prefix(
+        p->d_out[k], dv + p->off[0], d.k_pool, d.v_pool,
+        reinterpret_cast<const int32_t*>(dv + p->off[3]),
+        reinterpret_cast<const int32_t*>(dv + p->off[4]), d.B, d.Hq, d.Hkv, d.D, d.block_size,
+        d.max_blocks, d.num_blocks, scale, d.dtype,
+        reinterpret_cast<const int32_t*>(dv + p->off[7]),
+        reinterpret_cast<const int32_t*>(dv + p->off[8]),
+        reinterpret_cast<const int32_t*>(dv + p->off[9]), ngroups, m, d.workspace,
+        d.workspace_bytes, d.dev_err_flag, d.compute);
+  } else {
+    st = pa_decode_append(p->d_out[k], dv + p->off[0], dv + p->off[1], dv + p->off[2], d.k_pool,
+                          d.v_pool, reinterpret_cast<const int32_t*>(dv + p->off[3]),
+                          reinterpret_cast<const int32_t*>(dv + p->off[4]), d.B, d.Hq, d.Hkv,
+                          d.D, d.block_size, d.max_blocks, d.num_blocks, scale, d.dtype,
+                          d.workspace, d.workspace_bytes, d.dev_err_flag, d.compute, nullptr);
+  }
   if (st != PA_OK) return st;
   if (cudaEventRecord(p->kern_done[k], cs) != cudaSuccess ||
       cudaStreamWaitEvent(cout, p->kern_done[k], 0) != cudaSuccess ||

@@ -249,12 +249,24 @@ def test_pipeline_layout_and_argument_errors_before_any_cuda_call():
     assert total == sum(up(s) for s in sizes)
     assert b.lib.pa_pipeline_input_bytes(0, 8, 2, 128, 5, b.PA_BF16, None) == 0
     assert b.lib.pa_pipeline_input_bytes(3, 8, 2, 128, 5, 7, None) == 0
+    # the shared-prefix slot: the same six sections, then slot_mapping, group_of,
+    # group_prefix and group_members [B][m]
+    offs10 = (ctypes.c_size_t * 10)()
+    assert b.lib.pa_pipeline_input_bytes_prefix(3, 8, 2, 128, 5, b.PA_BF16, 0, offs10) == total
+    sizes10 = sizes + [3 * 8, 3 * 4, 3 * 4, 3 * 6 * 4]
+    total10 = b.lib.pa_pipeline_input_bytes_prefix(3, 8, 2, 128, 5, b.PA_BF16, 6, offs10)
+    assert list(offs10) == [sum(up(s) for s in sizes10[:i]) for i in range(10)]
+    assert total10 == sum(up(s) for s in sizes10)
+    for m in (-1, 33):
+        assert b.lib.pa_pipeline_input_bytes_prefix(3, 8, 2, 128, 5, b.PA_BF16, m, None) == 0
 
     a = b.Allocator(8, 4)
     h = ctypes.c_void_p()
     desc = b.pa_pipeline_desc()  # all zero: B = 0, no buffers
     assert b.lib.pa_pipeline_create(a._h, ctypes.byref(desc), ctypes.byref(h)) == b.PA_ERR_INVALID_ARG
     assert not h.value
+    desc.shared_prefix_members = 33  # out of range as well
+    assert b.lib.pa_pipeline_create(a._h, ctypes.byref(desc), ctypes.byref(h)) == b.PA_ERR_INVALID_ARG
     assert b.lib.pa_pipeline_create(None, ctypes.byref(desc), ctypes.byref(h)) == b.PA_ERR_INVALID_ARG
     slot = ctypes.c_int()
     assert b.lib.pa_pipeline_next_slot(None, ctypes.byref(slot)) == b.PA_ERR_INVALID_ARG

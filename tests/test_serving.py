@@ -150,11 +150,66 @@ def test_serving_trace_matches_oracle_replay(name):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("name", ["serve_bs16_g8", "serve_bs8_g4", "serve_bs32_g2"])
+def test_serving_trace_shared_prefix_matches_oracle_replay(name):
+    """The same traces through PagedKVCache.step_shared_prefix: each step groups the
+    sequences that share a prompt's blocks and reads those blocks once per group.  Every
+    step's output matches the oracle replay, the pools end bit-identical and the free list
+    equal."""
+    import paged_kv_cache_350_b200 as pa
+    tr = TRACES[name]()
+    outs, _, ref_kp, ref_vp, ref_alloc = _oracle_replay(tr)
+
+    def dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+
+    def host(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+    cache = pa.PagedKVCache(tr.num_blocks, tr.block_size, tr.Hkv, tr.D, shuffle_seed=tr.alloc_seed,
+                            k_pool=dev(tr.pool("k")), v_pool=dev(tr.pool("v")))
+    maxm = min(32, 64 // (tr.Hq // tr.Hkv))
+    live, groups = [], 0
+    w = workloads.independent([1], dtype="bf16")
+    for t, ev in enumerate(tr.events):
+        for e in ev:
+            if e[0] == "admit":
+                pk, pv = tr.prompt_kv(e[1], e[2])
+                cache.admit(e[1], host(pk), host(pv))
+                live.append(e[1])
+            elif e[0] == "fork":
+                cache.fork(e[1], e[2])
+                live.append(e[2])
+            elif e[0] == "select":
+                cache.beam_select(e[1], e[2])
+            elif e[0] == "truncate":
+                cache.truncate(e[1], e[2])
+            else:
+                cache.retire(e[1])
+                live.remove(e[1])
+        ids = sorted(live)
+        q, nk, nv = tr.step_inputs(t, len(ids))
+        out = torch.empty((len(ids), tr.Hq, tr.D), dtype=torch.bfloat16).pin_memory()
+        cache.step_shared_prefix(ids, host(q).pin_memory(), host(nk).pin_memory(),
+                                 host(nv).pin_memory(), out, tr.scale, tr.max_blocks, maxm)
+        groups += cache.last_prefix_groups
+        assert_close(w, out.clone(), outs[t])
+    assert groups > 0
+    cache.check_device_errors()
+    kd = cache.k_pool.view(torch.int16).cpu().numpy().view(np.uint16)
+    vd = cache.v_pool.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(kd, ref_kp) and np.array_equal(vd, ref_vp)
+    assert cache.alloc.free_list() == list(ref_alloc.free)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("members", [0, 8])
 @pytest.mark.parametrize("depth", [1, 2, 3])
-def test_step_pipeline_matches_oracle_step_by_step(depth):
+def test_step_pipeline_matches_oracle_step_by_step(depth, members):
     """StepPipeline: steps queued back to back over `depth` staging slots, with different
     inputs every step and copy-on-write in the first; each step's output (read one step
-    late, as a serving loop would) must match the oracle, the final pools bit for bit."""
+    late, as a serving loop would) must match the oracle, the final pools bit for bit.
+    members > 0: the shared-prefix steps (fork groups of up to `members` samples)."""
     import paged_kv_cache_350_b200 as pa
     w = workloads.prefix_cow(prompts=2, prompt_len=100)
     steps = 7
@@ -198,7 +253,7 @@ def test_step_pipeline_matches_oracle_step_by_step(depth):
     setup_pairs = workloads.run_setup(w, cache.alloc)
     pa.pa_copy_blocks(cache.k_pool, cache.v_pool,
                       torch.tensor(setup_pairs, dtype=torch.int32, device="cuda").reshape(-1, 2))
-    pipe = cache.pipeline(B, w.Hq, MB, depth=depth)
+    pipe = cache.pipeline(B, w.Hq, MB, depth=depth, shared_prefix_members=members)
     got = []
     lag = min(1, depth - 1)  # a slot holds its output until it is reused
     for t in range(steps):
