@@ -426,9 +426,11 @@ typedef struct pa_pipeline_desc {
   pa_stream_t compute;        /* kernels */
   pa_stream_t copy_in;        /* host->device copies */
   pa_stream_t copy_out;       /* device->host copies */
-  int shared_prefix_members;  /* 0: pa_decode_append; 1 .. 32 (and * Hq/Hkv <= 64): the
-                                 shared-prefix step, workspace of
-                                 pa_decode_shared_prefix_workspace_size(B, .., B / 2) bytes */
+  int shared_prefix_members;  /* 0: pa_decode_append; 1 .. 32: the shared-prefix step, for
+                                 shapes pa_decode_shared_prefix takes (bf16, members *
+                                 Hq/Hkv <= 64, ...) and a workspace of at least
+                                 pa_decode_shared_prefix_workspace_size(B, .., B / 2) bytes
+                                 (checked by pa_pipeline_create: PA_ERR_INVALID_ARG) */
 } pa_pipeline_desc;
 
 /* Bytes of one input slot; offsets[6] (nullable) receives the byte offsets of its

@@ -58,6 +58,21 @@ bool valid_desc(const pa_pipeline_desc* d) {
          d->v_pool && d->host_in && d->dev_in && d->host_out && d->dev_out;
 }
 
+// The shared-prefix step's shape and workspace, checked when the pipeline is made, so that
+// no submit can fail in the decode after the cache write was queued.
+bool prefix_desc_ok(const pa_pipeline_desc* d) {
+  const int m = d->shared_prefix_members, G = d->Hq / d->Hkv;
+  if (m == 0) return true;
+  if (d->dtype != PA_BF16 || (d->D != 64 && d->D != 128) || G > 16 || m * G > 64 ||
+      (d->block_size != 8 && d->block_size != 16 && d->block_size != 32) || !d->workspace ||
+      reinterpret_cast<uintptr_t>(d->workspace) % 256 != 0)
+    return false;
+  // a group has two members or more, so a step has at most B / 2 of them
+  const size_t need = pa_decode_shared_prefix_workspace_size(d->B, d->Hq, d->Hkv, d->D,
+                                                             d->block_size, d->B / 2);
+  return need != static_cast<size_t>(-1) && d->workspace_bytes >= need;
+}
+
 void destroy_events(pa_pipeline* p) {
   for (auto* v : {&p->h2d_done, &p->kern_done, &p->d2h_done})
     for (cudaEvent_t e : *v)
@@ -103,7 +118,7 @@ pa_status pa_pipeline_create(pa_allocator* alloc, const pa_pipeline_desc* desc,
                              pa_pipeline** out) {
   if (!out) return PA_ERR_INVALID_ARG;
   *out = nullptr;
-  if (!alloc || !valid_desc(desc)) return PA_ERR_INVALID_ARG;
+  if (!alloc || !valid_desc(desc) || !prefix_desc_ok(desc)) return PA_ERR_INVALID_ARG;
   const int depth = desc->depth;
   for (int k = 0; k < depth; ++k)
     if (!desc->host_in[k] || !desc->dev_in[k] || !desc->host_out[k] || !desc->dev_out[k] ||

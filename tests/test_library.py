@@ -267,6 +267,15 @@ def test_pipeline_layout_and_argument_errors_before_any_cuda_call():
     assert not h.value
     desc.shared_prefix_members = 33  # out of range as well
     assert b.lib.pa_pipeline_create(a._h, ctypes.byref(desc), ctypes.byref(h)) == b.PA_ERR_INVALID_ARG
+    # a shared-prefix descriptor the decode would refuse (fp32; 16 members x G = 8 > 64
+    # rows; no workspace) is refused when the pipeline is made, before any CUDA call
+    bufs = (ctypes.c_void_p * 1)(16)
+    for dtype, m, ws in ((b.PA_F32, 4, 256), (b.PA_BF16, 16, 256), (b.PA_BF16, 4, None)):
+        d2 = b.pa_pipeline_desc(4, 16, 2, 128, 16, 8, 64, dtype, 1, 16, 16, ws, 1 << 30, None,
+                                bufs, bufs, bufs, bufs, None, None, None, m)
+        assert b.lib.pa_pipeline_create(a._h, ctypes.byref(d2), ctypes.byref(h)) == \
+            b.PA_ERR_INVALID_ARG
+        assert not h.value
     assert b.lib.pa_pipeline_create(None, ctypes.byref(desc), ctypes.byref(h)) == b.PA_ERR_INVALID_ARG
     slot = ctypes.c_int()
     assert b.lib.pa_pipeline_next_slot(None, ctypes.byref(slot)) == b.PA_ERR_INVALID_ARG
