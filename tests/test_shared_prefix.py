@@ -86,6 +86,13 @@ CASES = {
     # long prompts: units span several CTAs, so cut units are merged across CTAs
     "long_prompt_m8": (lambda: workloads.prefix(prompts=4, n=8, prompt_len=2000,
                                                 max_private=300), 8),
+    # G = 2 (2 rows a member) and G = 16 (a member fills a sub-partition)
+    "prefix_g2_m16": (lambda: workloads.prefix(prompts=2, n=16, prompt_len=140, max_private=60,
+                                               Hq=16, Hkv=8), 16),
+    "prefix_g16_m4": (lambda: workloads.prefix(prompts=2, n=4, prompt_len=140, max_private=60,
+                                               Hq=32, Hkv=2), 4),
+    "prefix_g16_m2": (lambda: workloads.prefix(prompts=2, n=4, prompt_len=140, max_private=60,
+                                               Hq=32, Hkv=2), 2),
     # units of 64, 36, 24, 12 and 4 rows (and ungrouped sequences) in one launch, so a CTA
     # moves between units whose rows fill different numbers of sub-partitions
     "families_mixed_m16": (lambda: workloads.families(), 16),
