@@ -39,6 +39,24 @@ def test_prefix_refcounts_and_copy_counts():
     assert pairs.shape[0] == 32 * 7 and (lens == 1001).all()
 
 
+def test_families_mixed_sizes():
+    """Fork families of the given sizes share their prompt's full blocks (refcount = family
+    size); unforked sequences hold blocks of their own; every pool block fits."""
+    w = workloads.families()
+    sizes, solo, P = w.meta["sizes"], w.meta["solo"], w.meta["prompt_len"]
+    assert w.B == sum(sizes) + solo
+    alloc = RefAllocator(w.num_blocks, w.block_size, shuffle_seed=w.alloc_seed)
+    workloads.run_setup(w, alloc)
+    first = 0
+    for n in sizes:
+        table, _ = alloc.block_table(first)
+        assert all(alloc.refcount(b) == n for b in table[:P // w.block_size])
+        first += n
+    _, pairs, tables, lens = workloads.run_step_allocation(w, alloc)
+    assert (lens[:sum(sizes)] >= P + 1).all() and (lens[sum(sizes):] >= 1).all()
+    assert tables.shape[1] <= w.max_blocks and alloc.num_free() >= 0
+
+
 def test_length_distributions():
     w = workloads.gqa()
     L = np.array(w.meta["decode_lens"])
