@@ -21,6 +21,7 @@
 
 #include <cuda_runtime.h>
 
+#include <cstdint>
 #include <new>
 #include <vector>
 
@@ -67,7 +68,13 @@ bool prefix_desc_ok(const pa_pipeline_desc* d) {
       (d->block_size != 8 && d->block_size != 16 && d->block_size != 32) || !d->workspace ||
       reinterpret_cast<uintptr_t>(d->workspace) % 256 != 0)
     return false;
-  // a group has two members or more, so a step has at most B / 2 of them
+  // a group has two members or more, so a step has at most B / 2 of them; the decode
+  // takes B + ngroups <= 8192 rows and fewer than 2^31 row chunks (32 tokens each)
+  const int64_t rows = static_cast<int64_t>(d->B) + d->B / 2;
+  const int64_t chunks_per_row =
+      (static_cast<int64_t>(d->max_blocks) * d->block_size + PA_SHARED_PREFIX_ALIGN - 1) /
+      PA_SHARED_PREFIX_ALIGN;
+  if (rows > 8192 || rows * d->Hkv * chunks_per_row >= (int64_t(1) << 31)) return false;
   const size_t need = pa_decode_shared_prefix_workspace_size(d->B, d->Hq, d->Hkv, d->D,
                                                              d->block_size, d->B / 2);
   return need != static_cast<size_t>(-1) && d->workspace_bytes >= need;
