@@ -203,15 +203,17 @@ def test_serving_trace_shared_prefix_matches_oracle_replay(name):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("members", [0, 8])
+@pytest.mark.parametrize("wl, members", [("cow", 0), ("cow", 8), ("solo", 4)])
 @pytest.mark.parametrize("depth", [1, 2, 3])
-def test_step_pipeline_matches_oracle_step_by_step(depth, members):
+def test_step_pipeline_matches_oracle_step_by_step(depth, wl, members):
     """StepPipeline: steps queued back to back over `depth` staging slots, with different
     inputs every step and copy-on-write in the first; each step's output (read one step
     late, as a serving loop would) must match the oracle, the final pools bit for bit.
-    members > 0: the shared-prefix steps (fork groups of up to `members` samples)."""
+    members > 0: the shared-prefix steps (fork groups of up to `members` samples; "solo":
+    unforked sequences, so that no group forms in any step)."""
     import paged_kv_cache_350_b200 as pa
-    w = workloads.prefix_cow(prompts=2, prompt_len=100)
+    w = (workloads.prefix_cow(prompts=2, prompt_len=100) if wl == "cow"
+         else workloads.gqa(B=6, median=100, lo=1, hi=200))
     steps = 7
     MB = w.max_blocks + steps // w.block_size + 2
     B = len(w.step_seqs)
@@ -233,7 +235,7 @@ def test_step_pipeline_matches_oracle_step_by_step(depth, members):
             slots.append(slot)
             if src >= 0:
                 pairs.append((src, dst))
-        if t == 0:
+        if t == 0 and wl == "cow":
             assert pairs, "the first step copies on write"
         kp, vp = ref_copy_blocks(kp, vp, pairs)
         kp, vp = ref_reshape_and_cache(nk, nv, kp, vp, np.array(slots))
