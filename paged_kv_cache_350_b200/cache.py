@@ -136,8 +136,11 @@ class PagedKVCache:
         tensors as ``step``; returns (h2d_bytes, d2h_bytes), and ``last_prefix_groups`` is the
         number of groups formed.
         """
-        stream = stream or torch.cuda.current_stream(self.device)
         B, Hq, D = q_host.shape
+        # refused before the allocator or the pools change
+        if not (1 <= max_members <= 32 and max_members * (Hq // self.Hkv) <= 64):
+            raise _b.PAError(_b.PA_ERR_UNSUPPORTED, "step_shared_prefix: max_members")
+        stream = stream or torch.cuda.current_stream(self.device)
         ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
         slots_h = self._pinned(("slots",), (B,), torch.int64)
         pairs_h = self._pinned(("pairs",), (B, 2), torch.int32)

@@ -294,3 +294,20 @@ def test_pipeline_layout_and_argument_errors_before_any_cuda_call():
     assert chk(np.array([5], dtype=np.int64), 3) == b.PA_ERR_NOT_FOUND
     free = a.num_free()
     assert free == 8 - 1 - 2 and a.block_table(1)[1] == 8   # the checks changed nothing
+
+
+def test_step_shared_prefix_refuses_bad_group_size_before_any_change():
+    """PagedKVCache.step_shared_prefix: a group size the decode cannot take (over 32
+    members, or members x Hq/Hkv over 64 rows) is refused before the allocator changes."""
+    import torch
+    import paged_kv_cache_350_b200 as pa
+    cache = pa.PagedKVCache(16, 16, 2, 128, device="cpu")
+    cache.alloc.add_seq(0, 20)
+    cache.alloc.fork(0, 1)
+    free = cache.alloc.num_free()
+    q = torch.zeros((2, 16, 128), dtype=torch.bfloat16)
+    kv = torch.zeros((2, 2, 128), dtype=torch.bfloat16)
+    for m in (0, 33, 9):  # 9 members x G = 8 is 72 rows
+        with pytest.raises(pa.PAError):
+            cache.step_shared_prefix([0, 1], q, kv, kv, torch.empty_like(q), 0.1, 4, m)
+        assert cache.alloc.num_free() == free
