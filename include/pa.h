@@ -214,9 +214,13 @@ pa_status pa_decode_append(void* out, const void* q, const void* k_new, const vo
  * pa_alloc_prefix_groups builds these from the allocator.  bf16 tensor-core shapes only
  * (PA_ERR_UNSUPPORTED otherwise); max_members <= 32, max_members * (Hq/Hkv) <= 64;
  * B + ngroups <= 8192.
- * One launch: a persistent kernel with one CTA per SM.  A unit split between CTAs is
- * merged by the CTA that finishes its last piece (the pieces' partials and a per-call
- * tagged counter live in the workspace; no CTA waits for another).
+ * One launch: a persistent kernel with one CTA per SM, the tile math on the 5th-generation
+ * tensor cores.  A unit split between CTAs is merged by the CTA holding its first chunk
+ * (its owner): each later CTA publishes its piece's partial (per-row max, sum and
+ * unnormalised output) in the workspace with a flag tagged for this call, and the owner
+ * waits for those flags (bounded: every CTA of the grid is resident), merges, writes the
+ * rows and clears the flags it consumed, so that a replay of a captured launch waits for
+ * fresh partials.
  * Workspace: pa_decode_shared_prefix_workspace_size (on the current device); its contents
  * need no initialisation, and calls whose kernels may overlap on the GPU must not share
  * one. */
