@@ -306,12 +306,19 @@ __global__ void __launch_bounds__(C::THREADS, C::MIN_CTAS)
           flag_error(p.err, PA_DEVERR_BAD_BLOCK_ID);
           phys = 0;
         }
+        if constexpr (C::BPS == 1) {
+          // chunk c lands at c * CHUNK_BYTES (CHUNK_BYTES = BOXR rows of 128 bytes)
+          static_assert(C::BOXR == C::TILE_T, "one box spans the stage's rows");
+          tma_load_5d(kt, &tmk, 0, row0, 0, kv, phys, fb, policy);
+          tma_load_5d(vt, &tmv, 0, row0, 0, kv, phys, fb, policy);
+        } else {
 #pragma unroll
-        for (int c = 0; c < C::DCH; ++c) {
-          tma_load_4d(kt + c * C::CHUNK_BYTES + sub * C::BOXR * 128, &tmk, c * 64, kv, row0,
-                      phys, fb, policy);
-          tma_load_4d(vt + c * C::CHUNK_BYTES + sub * C::BOXR * 128, &tmv, c * 64, kv, row0,
-                      phys, fb, policy);
+          for (int c = 0; c < C::DCH; ++c) {
+            tma_load_4d(kt + c * C::CHUNK_BYTES + sub * C::BOXR * 128, &tmk, c * 64, kv, row0,
+                        phys, fb, policy);
+            tma_load_4d(vt + c * C::CHUNK_BYTES + sub * C::BOXR * 128, &tmv, c * 64, kv, row0,
+                        phys, fb, policy);
+          }
         }
       }
     }
@@ -563,9 +570,15 @@ template <class C>
 cudaError_t launch_stream_cfg(const StreamParams& sp, int grid, cudaStream_t stream) {
   CUtensorMap tmk, tmv;
   const DecodeParams& p = sp.d;
-  if (!make_pool_map(&tmk, p.k_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BOXR) ||
-      !make_pool_map(&tmv, p.v_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BOXR))
-    return cudaErrorInvalidValue;
+  // a stage of one block (or of part of one): one box of all D columns per stage and pool
+  // (the 5-D view lands in the stage's chunk-major layout); several blocks a stage: one
+  // box per block and 64-column chunk
+  const bool ok = C::BPS == 1
+      ? make_pool_map_rows(&tmk, p.k_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BOXR) &&
+        make_pool_map_rows(&tmv, p.v_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BOXR)
+      : make_pool_map(&tmk, p.k_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BOXR) &&
+        make_pool_map(&tmv, p.v_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BOXR);
+  if (!ok) return cudaErrorInvalidValue;
   const size_t smem = stream_smem_bytes<C>(p.B);
   cudaError_t e = cudaFuncSetAttribute(decode_stream_kernel<C>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,

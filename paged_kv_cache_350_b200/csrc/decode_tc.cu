@@ -276,6 +276,28 @@ bool make_pool_map(CUtensorMap* map, const void* pool, int NB, int BS, int Hkv, 
   return r == CUDA_SUCCESS;
 }
 
+// The same pool as a 5-D tensor (64 columns, rows, D / 64 column chunks, heads, blocks)
+// whose box is box_rows rows of one head and all D columns, landing as
+// [D / 64][box_rows][64] (128-byte swizzled): one box where the 4-D view needs D / 64.
+bool make_pool_map_rows(CUtensorMap* map, const void* pool, int NB, int BS, int Hkv, int D,
+                        int box_rows) {
+  auto encode = get_encode_fn();
+  if (!encode || D % 64 != 0) return false;
+  cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(BS), static_cast<cuuint64_t>(D / 64),
+                        static_cast<cuuint64_t>(Hkv), static_cast<cuuint64_t>(NB)};
+  cuuint64_t strides[4] = {static_cast<cuuint64_t>(Hkv) * D * 2, 128,
+                           static_cast<cuuint64_t>(D) * 2,
+                           static_cast<cuuint64_t>(BS) * Hkv * D * 2};
+  cuuint32_t box[5] = {64, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(D / 64),
+                       1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(pool), dims,
+                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool make_q_map(CUtensorMap* map, const void* q, int B, int Hq, int D, int G) {
   auto encode = get_encode_fn();
   if (!encode || G < 1 || G > 256) return false;

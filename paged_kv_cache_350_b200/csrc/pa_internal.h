@@ -78,6 +78,10 @@ cudaError_t launch_decode_prefix(const PrefixParams& pp, int grid, cudaStream_t 
 // block starting at a row coordinate) x 64 columns of one head.
 bool make_pool_map(CUtensorMap* map, const void* pool, int NB, int BS, int Hkv, int D,
                    int box_rows);
+// 5-D TMA view of the same pool: box = box_rows rows of one head with all D columns,
+// landing as [D / 64][box_rows][64], 128-byte swizzled.
+bool make_pool_map_rows(CUtensorMap* map, const void* pool, int NB, int BS, int Hkv, int D,
+                        int box_rows);
 // Tensor map over q viewed as [B][Hq][D] (bf16): boxes of 64 columns x G heads of one
 // batch row, 128-byte swizzled.
 bool make_q_map(CUtensorMap* map, const void* q, int B, int Hq, int D, int G);
