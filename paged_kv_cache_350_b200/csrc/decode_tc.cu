@@ -151,10 +151,18 @@ __global__ void __launch_bounds__(C::THREADS)
           if (ok) {
             const uint32_t kt = smem_addr(smem + stage * C::STAGE_BYTES) + sub * BS * 128;
             const uint32_t vt = kt + C::TILE_BYTES;
+            if constexpr (C::BPS == 1) {
+              // a stage is one block: one box of all D columns per pool, chunk c landing
+              // at c * CHUNK_BYTES (CHUNK_BYTES = BS rows of 128 bytes)
+              static_assert(C::TILE_T == BS, "one block a stage");
+              tma_load_5d(kt, &tmk, 0, 0, 0, kvh, phys, fb, policy);
+              tma_load_5d(vt, &tmv, 0, 0, 0, kvh, phys, fb, policy);
+            } else {
 #pragma unroll
-            for (int c = 0; c < C::DCH; ++c) {
-              tma_load_4d(kt + c * C::CHUNK_BYTES, &tmk, c * 64, kvh, 0, phys, fb, policy);
-              tma_load_4d(vt + c * C::CHUNK_BYTES, &tmv, c * 64, kvh, 0, phys, fb, policy);
+              for (int c = 0; c < C::DCH; ++c) {
+                tma_load_4d(kt + c * C::CHUNK_BYTES, &tmk, c * 64, kvh, 0, phys, fb, policy);
+                tma_load_4d(vt + c * C::CHUNK_BYTES, &tmv, c * 64, kvh, 0, phys, fb, policy);
+              }
             }
           }
         }
@@ -318,8 +326,13 @@ namespace {
 template <class C>
 cudaError_t launch_cfg(const DecodeParams& p, cudaStream_t stream) {
   CUtensorMap tmk, tmv;
-  if (!make_pool_map(&tmk, p.k_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BS) ||
-      !make_pool_map(&tmv, p.v_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BS))
+  // a stage of one block: the 5-D view (one box per pool); several: one box per chunk
+  const bool maps = C::BPS == 1
+      ? make_pool_map_rows(&tmk, p.k_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BS) &&
+        make_pool_map_rows(&tmv, p.v_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BS)
+      : make_pool_map(&tmk, p.k_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BS) &&
+        make_pool_map(&tmv, p.v_pool, p.num_blocks, C::BS, p.Hkv, C::D, C::BS);
+  if (!maps)
     return cudaErrorInvalidValue;
   auto kern = decode_tc_kernel<C>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
