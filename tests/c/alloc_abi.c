@@ -63,6 +63,36 @@ int main(void) {
 
   CHECK(strcmp(pa_status_string(PA_ERR_OUT_OF_BLOCKS), "no free block left in the pool") == 0);
   pa_alloc_destroy(a);
+
+  /* parallel sampling ("深入解析 PagedAttention", 多序列共享): a 34-token prompt in blocks
+   * of 4 forked twice; the step's appends copy the shared partial block for two of the
+   * three, and the grouping for the shared-prefix decode finds the 32 shared tokens */
+  CHECK(pa_alloc_create(32, 4, 0, &a) == PA_OK);
+  CHECK(pa_alloc_add_seq(a, 0, 34) == PA_OK);
+  CHECK(pa_alloc_fork(a, 0, 1) == PA_OK && pa_alloc_fork(a, 0, 2) == PA_OK);
+  const int64_t ids[3] = {0, 1, 2};
+  int64_t slots[3];
+  int32_t pairs[6];
+  int npairs = -1;
+  CHECK(pa_alloc_append_slots(a, ids, 3, slots, pairs, &npairs) == PA_OK && npairs == 2);
+  int32_t group_of[3], group_prefix[3], group_members[3 * 4];
+  int ngroups = -1;
+  CHECK(pa_alloc_prefix_groups(a, ids, 3, 4, PA_SHARED_PREFIX_ALIGN, group_of, group_prefix,
+                               group_members, &ngroups) == PA_OK);
+  CHECK(ngroups == 1 && group_prefix[0] == 32);
+  CHECK(group_of[0] == 0 && group_of[1] == 0 && group_of[2] == 0);
+  CHECK(group_members[0] == 0 && group_members[1] == 1 && group_members[2] == 2 &&
+        group_members[3] == -1);
+  pa_alloc_destroy(a);
+
+  /* the step pipeline's input slot: the shared-prefix layout extends the plain one */
+  size_t off6[6], off10[10];
+  const size_t plain = pa_pipeline_input_bytes(3, 8, 2, 128, 16, PA_BF16, off6);
+  const size_t sp = pa_pipeline_input_bytes_prefix(3, 8, 2, 128, 16, PA_BF16, 4, off10);
+  CHECK(plain > 0 && sp > plain && off10[6] == plain);
+  for (int i = 0; i < 6; ++i) CHECK(off10[i] == off6[i]);
+  CHECK(pa_pipeline_input_bytes_prefix(3, 8, 2, 128, 16, PA_BF16, 0, NULL) == plain);
+  CHECK(pa_pipeline_input_bytes_prefix(3, 8, 2, 128, 16, PA_BF16, 33, NULL) == 0);
   printf("ok\n");
   return 0;
 }

@@ -217,7 +217,8 @@ def test_binding_rejects_host_tensors_before_the_c_call():
 
 def test_header_compiles_as_c_and_the_allocator_runs_from_plain_c(tmp_path):
     """include/pa.h is a C header (strict C11) and the library serves a C client: the
-    allocator's copy-on-write story run from tests/c/alloc_abi.c, no Python in the path."""
+    allocator's copy-on-write story, the fork grouping for the shared-prefix decode and the
+    pipeline's slot layout, run from tests/c/alloc_abi.c, no Python in the path."""
     import shutil
     import subprocess
     cc = shutil.which("gcc") or shutil.which("cc")
